@@ -1,0 +1,186 @@
+"""CPU oracle for the forward pass of a Laguna-style token-choice MoE layer.
+
+TEST INFRASTRUCTURE.  This module is the independent checker of the CUDA
+library, not part of it.  Only the test suite, the smoke check in
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it.
+It shares no code with the CUDA path: it takes plain numpy arrays (bfloat16
+inputs as uint16 bit patterns, or float arrays) and computes in float64.
+
+What the layer computes, and where the pages say so:
+
+* Router: sigmoid scores over the experts, token-choice top-k, and
+  normalisation of the selected scores to sum to one
+  (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1:
+  "sigmoid router with post-top-k normalization"; Laguna-M.1-base spec sheet,
+  Mixture of experts: "Router score: sigmoid", "Renormalize top-k: Yes").
+* Experts: SwiGLU feed-forward blocks without bias
+  (Laguna-M.1-base spec sheet, Feed-forward: "Activation: SwiGLU",
+  "FFN bias: No", gate_proj / up_proj / down_proj projections).
+* Combine: the routed sum is multiplied by the modulation factor 2.5 and then
+  added to an always-on shared expert
+  (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1;
+  Laguna-M.1-base spec sheet, Mixture of experts, "Routed scaling factor":
+  1 for M.1, 2.5 introduced in XS.2).
+* Expert order: tokens are laid out expert by expert before the grouped GEMM
+  (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1.2,
+  Fig. 2: tokens are copied "in expert order").
+
+Readings where the pages are silent (each one listed in the design doc):
+
+* SwiGLU(x) = W_down (silu(W_gate x) * (W_up x)), silu(z) = z * sigmoid(z).
+* One shared expert of the same SwiGLU form, ungated, added after the 2.5.
+* An optional router bias b (a workload device) is added to the logits
+  before the sigmoid; it changes selection and weights alike.
+* Top-k is taken on the scores; since the sigmoid is strictly increasing this
+  is the same as taking it on the logits.  Exact ties go to the lower expert
+  index.  The selected list is ordered by descending score.
+* Normalisation runs over the k selected experts only, with no epsilon.
+
+Every function is a direct transcription of these definitions; numpy's
+matmul is the only library step.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def bf16_to_f64(a):
+    """Exact widening of bfloat16 bit patterns (uint16) to float64.
+
+    Float arrays are passed through as float64 unchanged.
+    """
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def sigmoid(z):
+    """Logistic function 1 / (1 + exp(-z)), float64."""
+    z = np.asarray(z, dtype=np.float64)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def silu(z):
+    """SiLU (swish) z * sigmoid(z), the gate nonlinearity of SwiGLU."""
+    z = np.asarray(z, dtype=np.float64)
+    return z * sigmoid(z)
+
+
+def router_logits(x, w_router, bias=None):
+    """l[t, e] = sum_i x[t, i] * W_r[e, i]  (+ b[e]).
+
+    x: [T, d]; w_router: [E, d] (nn.Linear [out, in] layout); bias: [E] or None.
+    """
+    X = bf16_to_f64(x)
+    W = bf16_to_f64(w_router)
+    logits = X @ W.T
+    if bias is not None:
+        logits = logits + np.asarray(bias, dtype=np.float64)[None, :]
+    return logits
+
+
+def select_topk(logits, k):
+    """Indices of the k largest logits per row, largest first.
+
+    Equal values keep ascending expert order, so an exact tie at the k-th
+    place goes to the lower expert index.
+    """
+    logits = np.asarray(logits, dtype=np.float64)
+    order = np.argsort(-logits, axis=1, kind="stable")
+    return order[:, :k].astype(np.int64)
+
+
+def normalise(selected_scores, norm_topk_prob=True):
+    """w_j = s_j / sum_j' s_j' over the selected experts (no epsilon)."""
+    s = np.asarray(selected_scores, dtype=np.float64)
+    if not norm_topk_prob:
+        return s.copy()
+    return s / s.sum(axis=1, keepdims=True)
+
+
+def route(x, w_router, bias, k, norm_topk_prob=True):
+    """Sigmoid router with post-top-k normalisation.
+
+    Returns (topk_idx [T,k] int64, topk_w [T,k] f64, scores [T,E] f64, logits [T,E] f64).
+    """
+    logits = router_logits(x, w_router, bias)
+    scores = sigmoid(logits)
+    idx = select_topk(logits, k)
+    sel = np.take_along_axis(scores, idx, axis=1)
+    return idx, normalise(sel, norm_topk_prob), scores, logits
+
+
+def swiglu_ffn(x, w_gate, w_up, w_down):
+    """down(silu(gate x) * (up x)) without bias, float64.
+
+    x: [n, d]; w_gate, w_up: [F, d]; w_down: [d, F]  (nn.Linear layouts).
+    """
+    X = bf16_to_f64(x)
+    g = X @ bf16_to_f64(w_gate).T
+    u = X @ bf16_to_f64(w_up).T
+    h = silu(g) * u
+    return h @ bf16_to_f64(w_down).T
+
+
+def expert_order(topk_idx, E):
+    """Layout of the (token, slot) pairs in expert order.
+
+    counts[e]  = number of tokens that selected expert e;
+    offsets    = exclusive prefix sum of counts, length E + 1;
+    perm[r]    = t * k + j for the r-th row in expert order, where rows of
+                 one expert are sorted by token t, then by slot j.
+    """
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    T, k = idx.shape
+    counts = np.zeros(E, dtype=np.int64)
+    for e in idx.reshape(-1):
+        counts[e] += 1
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.empty(T * k, dtype=np.int64)
+    fill = offsets[:-1].copy()
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            perm[fill[e]] = t * k + j
+            fill[e] += 1
+    return counts, offsets, perm
+
+
+def moe_forward(x, w_router, w_gate, w_up, w_down, k, *, router_bias=None,
+                ws_gate=None, ws_up=None, ws_down=None,
+                routed_scaling_factor=2.5, norm_topk_prob=True, routing=None):
+    """y_t = S(x_t) + scale * sum_j w_{t,j} * E_{e_{t,j}}(x_t), in float64.
+
+    x: [T, d]; w_router: [E, d]; w_gate, w_up: [E, F, d]; w_down: [E, d, F];
+    ws_gate, ws_up: [Fs, d]; ws_down: [d, Fs] (None: no shared expert).
+    ``routing`` may pass a precomputed (topk_idx, topk_w) pair from ``route``.
+
+    Returns a dict with y, the routed sum R (before the scale), the shared
+    output Sh, and the routing (topk_idx, topk_w, scores, logits).
+    """
+    X = bf16_to_f64(x)
+    T, d = X.shape
+    if routing is None:
+        idx, w, scores, logits = route(x, w_router, router_bias, k, norm_topk_prob)
+    else:
+        idx, w = routing
+        scores = logits = None
+    E = np.asarray(w_gate).shape[0]
+    # contrib[t, j] = w_{t,j} * E_{e_{t,j}}(x_t); each expert evaluated on its tokens.
+    contrib = np.zeros((T, k, d), dtype=np.float64)
+    for e in range(E):
+        tt, jj = np.nonzero(idx == e)
+        if tt.size == 0:
+            continue
+        o = swiglu_ffn(X[tt], w_gate[e], w_up[e], w_down[e])
+        contrib[tt, jj, :] = w[tt, jj][:, None] * o
+    R = contrib.sum(axis=1)
+    if ws_gate is not None:
+        Sh = swiglu_ffn(X, ws_gate, ws_up, ws_down)
+    else:
+        Sh = np.zeros((T, d), dtype=np.float64)
+    y = routed_scaling_factor * R + Sh
+    return {"y": y, "R": R, "Sh": Sh, "topk_idx": idx, "topk_w": w,
+            "scores": scores, "logits": logits}
