@@ -1,0 +1,168 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) forward pass of a Laguna-style
+ * token-choice mixture-of-experts layer.
+ *
+ * The layer (Laguna M.1/XS.2 Technical Report summary, Key claims, report
+ * §3.1; Laguna-M.1-base spec sheet, "Feed-forward" and "Mixture of experts"):
+ *
+ *   logits_t,e = x_t . W_r[e]  (+ b_e)            sigmoid router, scores s = sigmoid(logits)
+ *   S_t        = the k experts of largest score    token-choice top-k, ties -> lower index
+ *   w_t,j      = s_t,e_j / sum_j' s_t,e_j'         post-top-k normalisation
+ *   E_e(x)     = W_down[e] (silu(W_gate[e] x) * (W_up[e] x))   SwiGLU, no bias
+ *   y_t        = Sh(x_t) + routed_scaling_factor * sum_j w_t,j E_e_j(x_t)
+ *
+ * with Sh an always-on shared expert of the same SwiGLU form, and
+ * routed_scaling_factor the routed-expert modulation (2.5 in XS.2, 1 in M.1).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Pointers are caller-owned DEVICE memory unless stated otherwise; the
+ *   library allocates nothing per call.  bf16 tensors are passed as `const
+ *   void *` and hold IEEE bfloat16 bit patterns, row-major.
+ * - Weight layouts follow nn.Linear ([out, in], so the reduction dimension
+ *   is contiguous): w_router [E, d]; w_gate, w_up [E, F, d]; w_down [E, d, F];
+ *   ws_gate, ws_up [Fs, d]; ws_down [d, Fs].
+ * - Calls are asynchronous on `stream` (a cudaStream_t passed as void *; NULL
+ *   is the legacy default stream).  No call synchronises the host except
+ *   moe_read_device_status, so the sequence can be captured in a CUDA graph.
+ * - Every device pointer must be 16-byte aligned.  Shape limits: d_model a
+ *   multiple of 128; F and Fs multiples of 64 (Fs = 0: no shared expert);
+ *   1 <= k <= min(E, 16); E <= 512.  Anything else returns
+ *   MOE_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ * - T = 0 is a no-op that returns MOE_OK.
+ * - Errors: argument errors return synchronously and launch nothing; a failed
+ *   launch returns MOE_ERR_CUDA.  Errors found on the device (a bounded wait
+ *   that gave up, an out-of-range expert index) are written to a status word
+ *   at the start of the workspace; moe_read_device_status returns them.  The
+ *   library never aborts, exits or traps.
+ * - The workspace `ws` (size from moe_workspace_size) is scratch owned by the
+ *   caller.  Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,        /* NULL pointer, bad struct_size, misaligned pointer */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* dims outside the limits above */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+    MOE_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = 5,     /* a device-side wait gave up (see moe_read_device_status) */
+    MOE_ERR_DEVICE_BOUNDS = 6       /* a device-side index check failed (e.g. expert id >= E) */
+} moe_status;
+
+/* Layer dimensions.  Field names follow the model-config keys listed on the
+ * Laguna-M.1-base spec sheet ("Mixture of experts"). */
+typedef struct {
+    uint32_t struct_size;            /* sizeof(moe_dims_t) */
+    int32_t T;                       /* tokens in this call */
+    int32_t d_model;                 /* d */
+    int32_t num_experts;             /* E */
+    int32_t num_experts_per_tok;     /* k */
+    int32_t moe_intermediate_size;   /* F, width of one routed expert */
+    int32_t shared_intermediate_size;/* Fs, width of the shared expert; 0 = none */
+    float routed_scaling_factor;     /* routed-expert modulation, 2.5 for XS.2 */
+    int32_t norm_topk_prob;          /* 1: w = s / sum over the selected (both models); 0: w = s */
+    int32_t flags;                   /* MOE_FLAG_* below; 0 = automatic choices */
+} moe_dims_t;
+
+/* flags: force one of the two router implementations (both compute the same
+ * selection rule; the choice only changes speed). */
+#define MOE_FLAG_ROUTER_CUDA_CORE 1   /* fp32 FMA logits + warp-per-token top-k */
+#define MOE_FLAG_ROUTER_TENSOR    2   /* tcgen05 logits with the top-k in the epilogue */
+
+typedef struct {
+    const void *w_router;      /* [E, d] bf16 */
+    const float *router_bias;  /* [E] fp32 added to the logits, or NULL */
+    const void *w_gate;        /* [E, F, d] bf16 */
+    const void *w_up;          /* [E, F, d] bf16 */
+    const void *w_down;        /* [E, d, F] bf16 */
+    const void *ws_gate;       /* [Fs, d] bf16, NULL if Fs = 0 */
+    const void *ws_up;         /* [Fs, d] bf16 */
+    const void *ws_down;       /* [d, Fs] bf16 */
+} moe_weights_t;
+
+/* Routing outputs of moe_forward (caller-owned device memory, all required). */
+typedef struct {
+    int32_t *topk_idx;  /* [T, k] selected experts, descending score */
+    float *topk_w;      /* [T, k] normalised weights, same order */
+    int32_t *counts;    /* [E] rows per expert */
+    int32_t *offsets;   /* [E + 1] exclusive prefix sum of counts */
+    int32_t *perm;      /* [T * k] perm[r] = t * k + j for row r in expert order */
+} moe_routing_t;
+
+/* Bytes of scratch that moe_route / moe_permute / moe_forward need for these
+ * dims (0 if the dims are invalid).  The workspace must be 256-byte aligned. */
+size_t moe_workspace_size(const moe_dims_t *dims);
+
+/* Router: sigmoid scores, top-k with ties to the lower expert index, and
+ * post-top-k normalisation (Laguna M.1/XS.2 Technical Report summary, Key
+ * claims, report §3.1; Laguna-M.1-base spec sheet, Mixture of experts:
+ * "Router score", "Renormalize top-k").  Selection is made on fp32 logits
+ * (equivalent to selection on the scores, since the sigmoid is increasing).
+ * x: [T, d] bf16.  router_bias may be NULL.  Outputs topk_idx [T, k] int32 and
+ * topk_w [T, k] fp32, both in descending-score order. */
+moe_status moe_route(const moe_dims_t *dims, const void *x, const void *w_router,
+                     const float *router_bias, int32_t *topk_idx, float *topk_w,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/* Expert order of the (token, slot) pairs, the layout in which tokens are
+ * handed to the grouped expert GEMM (Laguna M.1/XS.2 Technical Report
+ * summary, Key claims, report §3.1.2, Fig. 2: tokens copied "in expert
+ * order").  counts[e] = rows of expert e; offsets = exclusive prefix sum
+ * ([E + 1]); perm[r] = t * k + j, rows of one expert in ascending (t, j).
+ * If x and x_perm are both non-NULL the gathered rows are also materialised:
+ * x_perm[r, :] = x[perm[r] / k, :] ([T * k, d] bf16).  An expert id outside
+ * [0, E) sets MOE_ERR_DEVICE_BOUNDS in the status word. */
+moe_status moe_permute(const moe_dims_t *dims, const int32_t *topk_idx, int32_t *counts,
+                       int32_t *offsets, int32_t *perm, const void *x, void *x_perm,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* The whole layer: route, permute, the SwiGLU experts as tcgen05 grouped
+ * GEMMs (gather of the permuted rows fused into the operand load), the shared
+ * expert, the routed_scaling_factor modulation and the weighted combine.
+ * x: [T, d] bf16 in; y: [T, d] bf16 out.  `routing` receives the router and
+ * permutation results.  Accumulation is fp32; the SwiGLU activation h is
+ * rounded to bf16 before the down projection, and y is rounded to bf16. */
+moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *weights, const void *x,
+                       void *y, const moe_routing_t *routing, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* Synchronises `stream`, then returns the device-side status word of `ws`
+ * (MOE_OK if no kernel reported an error) and, if site != NULL, the id of the
+ * place that reported it.  The status word is cleared by each moe_route /
+ * moe_permute / moe_forward call. */
+moe_status moe_read_device_status(const void *ws, void *stream, int32_t *site);
+
+/* Self-test of the device timeout path: launches one kernel that waits, with
+ * a bound of `limit_us` microseconds, on a flag nothing sets; it must give up
+ * and write MOE_ERR_DEVICE_TIMEOUT to the status word.  Used by the tests. */
+moe_status moe_selftest_bounded_wait(void *ws, size_t ws_bytes, uint32_t limit_us, void *stream);
+
+/* Stage timing for benchmarks: arms the NEXT moe_forward call on this host
+ * thread to record events (cudaEvent_t handles passed as void *, created by
+ * the caller) on its stream at the six stage boundaries: before the router,
+ * before the index builder, before the gate/up GEMM, before the down GEMM,
+ * before the combine, and after the combine.  Events beyond n_events are not
+ * recorded.  Pass events = NULL to disarm. */
+moe_status moe_profile_next_forward(void **events, int32_t n_events);
+
+/* Human-readable name of a status code (static string). */
+const char *moe_status_string(moe_status s);
+
+/* Number of kernel launches the last successful call on this host thread
+ * issued (for launch accounting in benchmarks). */
+int32_t moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

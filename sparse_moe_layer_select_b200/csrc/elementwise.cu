@@ -1,0 +1,115 @@
+// elementwise.cu -- the HBM-bound kernels of the layer.
+//
+//   gather_rows_kernel  x_perm[r, :] = x[perm[r] / k, :]   (materialised expert-order
+//                       activations; the forward pass fuses this gather into the GEMM
+//                       operand load instead)
+//   combine_kernel      y[t, :] = bf16( sum_j slot[t, j, :] ) over the k routed slots
+//                       (already scaled by routed_scaling_factor * w_t,j) and the
+//                       shared-expert slot: the combine of the routed sum with the
+//                       always-on shared expert (Laguna M.1/XS.2 Technical Report
+//                       summary, Key claims, report §3.1)
+//   selftest_wait_kernel  a bounded wait on a flag nothing sets (timeout self-test)
+//
+// All three move 16-byte vectors with one thread per vector, grid-stride.
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "status.cuh"
+
+namespace moe {
+
+namespace {
+
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ perm, int n_rows,
+                       int k, int vec_per_row, uint4 *__restrict__ x_perm) {
+  const size_t total = static_cast<size_t>(n_rows) * vec_per_row;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / vec_per_row);
+    const int c = static_cast<int>(i - static_cast<size_t>(r) * vec_per_row);
+    const int t = perm[r] / k;
+    x_perm[i] = x[static_cast<size_t>(t) * vec_per_row + c];
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    combine_kernel(const uint4 *__restrict__ slots, int T, int nslots, int vec_per_row,
+                   uint4 *__restrict__ y) {
+  const size_t total = static_cast<size_t>(T) * vec_per_row;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t t = i / vec_per_row;
+    const size_t c = i - t * vec_per_row;
+    const uint4 *src = slots + t * nslots * vec_per_row + c;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < nslots; ++j) {
+      const uint4 v = src[static_cast<size_t>(j) * vec_per_row];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += __uint_as_float(w[q] << 16);
+        acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+      o[q] = *reinterpret_cast<uint32_t *>(&b);
+    }
+    y[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+__global__ void selftest_wait_kernel(int *status, long long limit_cycles) {
+  // The flag lives in this CTA's shared memory and nothing ever sets it.
+  __shared__ volatile int flag;
+  if (threadIdx.x == 0) flag = 0;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const long long t0 = clock64();
+  while (flag == 0) {
+    if (clock64() - t0 > limit_cycles) {
+      record_status(status, MOE_ERR_DEVICE_TIMEOUT, SITE_SELFTEST_FLAG);
+      return;
+    }
+  }
+}
+
+int grid_for(size_t work, int threads) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t want = (work + threads - 1) / threads;
+  const size_t cap = static_cast<size_t>(sms) * 8;
+  return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_rows, int k, int d,
+                               uint16_t *x_perm, cudaStream_t s) {
+  const int vpr = d / 8;
+  const size_t work = static_cast<size_t>(n_rows) * vpr;
+  gather_rows_kernel<<<grid_for(work, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(x), perm,
+                                                         n_rows, k, vpr,
+                                                         reinterpret_cast<uint4 *>(x_perm));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t *slots, int T, int nslots, int d, uint16_t *y,
+                           cudaStream_t s) {
+  const int vpr = d / 8;
+  const size_t work = static_cast<size_t>(T) * vpr;
+  combine_kernel<<<grid_for(work, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(slots), T,
+                                                     nslots, vpr, reinterpret_cast<uint4 *>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(status, limit_cycles);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,75 @@
+// kernels.h -- internal launch interface between the C ABI (moe_api.cu) and
+// the device kernels.  Not part of the public boundary.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace moe {
+
+// Row tile of the grouped GEMMs: `nrows` (<= 128) consecutive rows starting
+// at `row0` of group `group` (an expert id, or E for the shared expert,
+// whose rows are token ids).
+struct Tile {
+  int group;
+  int row0;
+  int nrows;
+  int pad;
+};
+
+constexpr int kBlockM = 128;        // rows per tile (tcgen05 M)
+constexpr int kBlockK = 64;         // K elements per pipeline stage (one 128-byte swizzle row)
+constexpr int kStages = 4;          // shared-memory pipeline depth
+constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kIndexChunk = 1024;   // (token, slot) entries per index-builder chunk
+
+enum GemmMode : int { MODE_ROUTER = 0, MODE_GEMM1 = 1, MODE_GEMM2 = 2 };
+
+struct GemmParams {
+  int *status;              // workspace header (status word)
+  const Tile *tiles;        // GEMM1/GEMM2: tile list
+  const int *n_tiles_dev;   // GEMM1/GEMM2: number of tiles (device)
+  int n_tiles_host;         // ROUTER: number of row tiles
+  int n_ntiles;             // N tiles per row tile (max over groups)
+  int T, d, E, k, F, Fs;
+  int n_half;               // GEMM1: gate (and up) columns per N tile
+  int n_tile;               // MMA N of this launch
+  int slots;                // GEMM2: slots per token (k, plus one if shared)
+  uint32_t a_bytes;         // bytes of one A stage (ROUTER, GEMM2 routed rows)
+  uint32_t a_sh_bytes;      // bytes of one A stage for shared-expert rows (GEMM2)
+  float routed_scale;       // GEMM2: routed_scaling_factor
+  int norm_topk;            // ROUTER
+  const int *perm;          // GEMM1/GEMM2: expert-order rows -> t * k + j
+  const float *topk_w;      // GEMM2
+  const float *bias;        // ROUTER (may be null)
+  int *topk_idx;            // ROUTER out
+  float *topk_w_out;        // ROUTER out
+  uint16_t *h;              // GEMM1 out: [T*k, F] bf16 (expert-order rows)
+  uint16_t *h_shared;       // GEMM1 out: [T, Fs] bf16
+  uint16_t *slot_out;       // GEMM2 out: [T, slots, d] bf16
+};
+
+struct GemmMaps {
+  CUtensorMap a, b0, b1, a_sh, b0_sh, b1_sh;
+};
+
+size_t gemm_smem_bytes();
+cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int grid,
+                        cudaStream_t s);
+
+cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
+                             float *logits, int T, int d, int E, cudaStream_t s);
+cudaError_t launch_topk_from_logits(const float *logits, int T, int E, int k, int norm_topk,
+                                    int32_t *topk_idx, float *topk_w, cudaStream_t s);
+
+cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
+                         int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
+                         int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches);
+cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_rows, int k, int d,
+                               uint16_t *x_perm, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t *slots, int T, int nslots, int d, uint16_t *y,
+                           cudaStream_t s);
+cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,466 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument checks,
+// workspace layout, TMA tensor maps and the launch sequence of the layer.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstddef>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+#include "status.cuh"
+
+namespace moe {
+cudaError_t gemm_set_attributes();
+}
+
+namespace {
+
+using namespace moe;
+
+thread_local int32_t g_last_launches = 0;
+thread_local void **g_prof_events = nullptr;
+thread_local int32_t g_prof_n = 0;
+
+// Records the next armed profiling event (if any) on stream s.
+struct EventMarker {
+  cudaStream_t s;
+  int next = 0;
+  bool on;
+  explicit EventMarker(cudaStream_t st) : s(st), on(g_prof_events != nullptr) {}
+  void mark() {
+    if (on && next < g_prof_n)
+      cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[next]), s);
+    ++next;
+  }
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int g_sms[kMaxDevices] = {0};
+bool g_attrs[kMaxDevices] = {false};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Per-device one-time set-up: SM count, shared-memory limits of the GEMM kernels.
+cudaError_t device_setup(int *sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return e != cudaSuccess ? e : cudaErrorNotSupported;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (!g_attrs[dev]) {
+    e = cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = gemm_set_attributes();
+    if (e != cudaSuccess) return e;
+    g_attrs[dev] = true;
+  }
+  *sms = g_sms[dev];
+  return cudaSuccess;
+}
+
+// 2-D bf16 tensor [rows, cols] (row-major), 128-byte swizzle, box 64 x box_rows.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBlockK), box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Dims {
+  int T, d, E, k, F, Fs, slots, flags, norm;
+  float scale;
+};
+
+struct WsLayout {
+  size_t header, chunk_hist, tiles, logits, h, h_sh, slots, total;
+  int max_tiles;
+};
+
+WsLayout ws_layout(const Dims &D) {
+  WsLayout L;
+  const size_t n = static_cast<size_t>(D.T) * D.k;
+  const size_t nchunks = (n + kIndexChunk - 1) / kIndexChunk;
+  L.max_tiles = static_cast<int>((n + kBlockM - 1) / kBlockM + D.E + (D.T + kBlockM - 1) / kBlockM);
+  size_t off = 0;
+  L.header = off;
+  off += align256(sizeof(WsHeader));
+  L.chunk_hist = off;
+  off += align256(std::max<size_t>(nchunks, 1) * D.E * 4);
+  L.tiles = off;
+  off += align256(static_cast<size_t>(L.max_tiles) * sizeof(Tile));
+  L.logits = off;
+  off += align256(static_cast<size_t>(D.T) * D.E * 4);
+  L.h = off;
+  off += align256(n * D.F * 2);
+  L.h_sh = off;
+  off += align256(static_cast<size_t>(D.T) * D.Fs * 2);
+  L.slots = off;
+  off += align256(static_cast<size_t>(D.T) * D.slots * D.d * 2);
+  L.total = off;
+  return L;
+}
+
+moe_status check_dims(const moe_dims_t *dims, Dims *D) {
+  if (dims == nullptr || dims->struct_size != sizeof(moe_dims_t)) return MOE_ERR_INVALID_ARG;
+  D->T = dims->T;
+  D->d = dims->d_model;
+  D->E = dims->num_experts;
+  D->k = dims->num_experts_per_tok;
+  D->F = dims->moe_intermediate_size;
+  D->Fs = dims->shared_intermediate_size;
+  D->scale = dims->routed_scaling_factor;
+  D->norm = dims->norm_topk_prob ? 1 : 0;
+  D->flags = dims->flags;
+  if (D->T < 0) return MOE_ERR_INVALID_ARG;
+  if (D->d < 128 || D->d % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D->E < 1 || D->E > 512) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D->k < 1 || D->k > 16 || D->k > D->E) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D->F < 64 || D->F % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D->Fs < 0 || D->Fs % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(D->T) * D->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(D->E) * std::max(D->F, D->d) >= (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((dims->flags & MOE_FLAG_ROUTER_TENSOR) && (D->E % 16 != 0 || D->E > 256))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  D->slots = D->k + (D->Fs > 0 ? 1 : 0);
+  return MOE_OK;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+moe_status check_ws(const Dims &D, const void *ws, size_t ws_bytes) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(D).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return MOE_OK;
+}
+
+inline char *wsp(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
+
+bool use_tensor_router(const Dims &D) {
+  if (D.flags & MOE_FLAG_ROUTER_CUDA_CORE) return false;
+  const bool fits = D.E % 16 == 0 && D.E <= 256;
+  if (D.flags & MOE_FLAG_ROUTER_TENSOR) return fits;
+  return fits && D.T >= 1024;
+}
+
+moe_status route_impl(const Dims &D, const void *x, const void *w_router, const float *bias,
+                      int32_t *topk_idx, float *topk_w, void *ws, cudaStream_t s, int sms,
+                      int *launches) {
+  const WsLayout L = ws_layout(D);
+  if (use_tensor_router(D)) {
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.status = reinterpret_cast<int *>(wsp(ws, L.header));
+    p.n_tiles_host = (D.T + kBlockM - 1) / kBlockM;
+    p.n_ntiles = 1;
+    p.T = D.T;
+    p.d = D.d;
+    p.E = D.E;
+    p.k = D.k;
+    p.F = D.F;
+    p.Fs = D.Fs;
+    p.n_tile = D.E;
+    p.norm_topk = D.norm;
+    p.bias = bias;
+    p.topk_idx = topk_idx;
+    p.topk_w_out = topk_w;
+    const uint32_t a_rows = static_cast<uint32_t>(std::min(D.T, kBlockM));
+    p.a_bytes = a_rows * kBlockK * 2;
+    GemmMaps m;
+    std::memset(&m, 0, sizeof(m));
+    if (!make_map(&m.a, x, D.T, D.d, a_rows)) return MOE_ERR_CUDA;
+    if (!make_map(&m.b0, w_router, D.E, D.d, D.E)) return MOE_ERR_CUDA;
+    m.b1 = m.b0;
+    m.a_sh = m.a;
+    m.b0_sh = m.b0;
+    m.b1_sh = m.b0;
+    const int grid = std::min(sms, p.n_tiles_host);
+    if (launch_gemm(MODE_ROUTER, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+    *launches += 1;
+    return MOE_OK;
+  }
+  float *logits = reinterpret_cast<float *>(wsp(ws, L.logits));
+  if (launch_router_cc(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(w_router),
+                       bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_topk_from_logits(logits, D.T, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *launches += 2;
+  return MOE_OK;
+}
+
+moe_status clear_header(void *ws, cudaStream_t s) {
+  return cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_dims_t *dims) {
+  Dims D;
+  if (check_dims(dims, &D) != MOE_OK) return 0;
+  return ws_layout(D).total;
+}
+
+moe_status moe_route(const moe_dims_t *dims, const void *x, const void *w_router,
+                     const float *router_bias, int32_t *topk_idx, float *topk_w, void *ws,
+                     size_t ws_bytes, void *stream) {
+  Dims D;
+  moe_status st = check_dims(dims, &D);
+  if (st != MOE_OK) return st;
+  if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(topk_idx) || !aligned16(topk_w) ||
+      (router_bias && !aligned16(router_bias)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(D, ws, ws_bytes)) != MOE_OK) return st;
+  g_last_launches = 0;
+  if (D.T == 0) return MOE_OK;
+  int sms = 0;
+  if (device_setup(&sms) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_header(ws, s)) != MOE_OK) return st;
+  int launches = 0;
+  st = route_impl(D, x, w_router, router_bias, topk_idx, topk_w, ws, s, sms, &launches);
+  g_last_launches = launches;
+  return st;
+}
+
+moe_status moe_permute(const moe_dims_t *dims, const int32_t *topk_idx, int32_t *counts,
+                       int32_t *offsets, int32_t *perm, const void *x, void *x_perm, void *ws,
+                       size_t ws_bytes, void *stream) {
+  Dims D;
+  moe_status st = check_dims(dims, &D);
+  if (st != MOE_OK) return st;
+  if (!topk_idx || !counts || !offsets || !perm) return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_idx) || !aligned16(counts) || !aligned16(offsets) || !aligned16(perm) ||
+      (x && (!aligned16(x) || !aligned16(x_perm))))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(D, ws, ws_bytes)) != MOE_OK) return st;
+  g_last_launches = 0;
+  if (D.T == 0) return MOE_OK;
+  int sms = 0;
+  if (device_setup(&sms) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_header(ws, s)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(D);
+  int launches = 0;
+  if (launch_index(topk_idx, D.T, D.k, D.E, D.Fs > 0, reinterpret_cast<int *>(wsp(ws, L.chunk_hist)),
+                   reinterpret_cast<Tile *>(wsp(ws, L.tiles)),
+                   reinterpret_cast<int *>(wsp(ws, L.header)), counts, offsets, perm, s,
+                   &launches) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (x) {
+    if (launch_gather_rows(static_cast<const uint16_t *>(x), perm, D.T * D.k, D.k, D.d,
+                           static_cast<uint16_t *>(x_perm), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    launches += 1;
+  }
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const void *x, void *y,
+                       const moe_routing_t *routing, void *ws, size_t ws_bytes, void *stream) {
+  Dims D;
+  moe_status st = check_dims(dims, &D);
+  if (st != MOE_OK) return st;
+  if (!w || !x || !y || !routing) return MOE_ERR_INVALID_ARG;
+  if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (D.Fs > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down)) return MOE_ERR_INVALID_ARG;
+  if (!routing->topk_idx || !routing->topk_w || !routing->counts || !routing->offsets ||
+      !routing->perm)
+    return MOE_ERR_INVALID_ARG;
+  const void *ptrs[] = {x, y, w->w_router, w->w_gate, w->w_up, w->w_down, routing->topk_idx,
+                        routing->topk_w, routing->counts, routing->offsets, routing->perm};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (w->router_bias && !aligned16(w->router_bias)) return MOE_ERR_INVALID_ARG;
+  if (D.Fs > 0 && (!aligned16(w->ws_gate) || !aligned16(w->ws_up) || !aligned16(w->ws_down)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(D, ws, ws_bytes)) != MOE_OK) return st;
+  g_last_launches = 0;
+  if (D.T == 0) return MOE_OK;
+  int sms = 0;
+  if (device_setup(&sms) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_header(ws, s)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(D);
+  int *header = reinterpret_cast<int *>(wsp(ws, L.header));
+  Tile *tiles = reinterpret_cast<Tile *>(wsp(ws, L.tiles));
+  uint16_t *h = reinterpret_cast<uint16_t *>(wsp(ws, L.h));
+  uint16_t *h_sh = reinterpret_cast<uint16_t *>(wsp(ws, L.h_sh));
+  uint16_t *slots = reinterpret_cast<uint16_t *>(wsp(ws, L.slots));
+  int launches = 0;
+  EventMarker ev(s);
+  g_prof_events = nullptr;  // one call only
+
+  // 1. router
+  ev.mark();
+  st = route_impl(D, x, w->w_router, w->router_bias, routing->topk_idx, routing->topk_w, ws, s,
+                  sms, &launches);
+  if (st != MOE_OK) return st;
+  // 2. expert order + tile list
+  ev.mark();
+  if (launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0,
+                   reinterpret_cast<int *>(wsp(ws, L.chunk_hist)), tiles, header, routing->counts,
+                   routing->offsets, routing->perm, s, &launches) != cudaSuccess)
+    return MOE_ERR_CUDA;
+
+  const int n_rows = D.T * D.k;
+  const int n_half = (D.F % 128 == 0 && D.Fs % 128 == 0) ? 128 : 64;
+  const int n2 = (D.d % 256 == 0) ? 256 : 128;
+
+  GemmParams base;
+  std::memset(&base, 0, sizeof(base));
+  base.status = header;
+  base.tiles = tiles;
+  base.n_tiles_dev = header + offsetof(WsHeader, n_tiles) / sizeof(int);
+  base.T = D.T;
+  base.d = D.d;
+  base.E = D.E;
+  base.k = D.k;
+  base.F = D.F;
+  base.Fs = D.Fs;
+  base.slots = D.slots;
+  base.routed_scale = D.scale;
+  base.norm_topk = D.norm;
+  base.perm = routing->perm;
+  base.topk_w = routing->topk_w;
+  base.h = h;
+  base.h_shared = h_sh;
+  base.slot_out = slots;
+
+  // 3. GEMM1: gathered x rows . [W_gate | W_up]^T -> SwiGLU -> h (bf16)
+  {
+    GemmParams p = base;
+    p.n_half = n_half;
+    p.n_tile = 2 * n_half;
+    p.n_ntiles = std::max(D.F, D.Fs) / n_half;
+    p.a_bytes = kBlockM * kBlockK * 2;
+    p.a_sh_bytes = p.a_bytes;
+    GemmMaps m;
+    std::memset(&m, 0, sizeof(m));
+    if (!make_map(&m.a, x, D.T, D.d, 1)) return MOE_ERR_CUDA;
+    if (!make_map(&m.b0, w->w_gate, static_cast<uint64_t>(D.E) * D.F, D.d, n_half)) return MOE_ERR_CUDA;
+    if (!make_map(&m.b1, w->w_up, static_cast<uint64_t>(D.E) * D.F, D.d, n_half)) return MOE_ERR_CUDA;
+    m.a_sh = m.a;
+    if (D.Fs > 0) {
+      if (!make_map(&m.b0_sh, w->ws_gate, D.Fs, D.d, n_half)) return MOE_ERR_CUDA;
+      if (!make_map(&m.b1_sh, w->ws_up, D.Fs, D.d, n_half)) return MOE_ERR_CUDA;
+    } else {
+      m.b0_sh = m.b0;
+      m.b1_sh = m.b1;
+    }
+    const int grid = sms;
+    ev.mark();
+    if (launch_gemm(MODE_GEMM1, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+    launches += 1;
+  }
+  // 4. GEMM2: h . W_down^T -> x (routed_scaling_factor * w) -> slot rows
+  {
+    GemmParams p = base;
+    p.n_tile = n2;
+    p.n_ntiles = D.d / n2;
+    const uint32_t a_rows = static_cast<uint32_t>(std::min(n_rows, kBlockM));
+    const uint32_t a_sh_rows = static_cast<uint32_t>(std::min(D.T, kBlockM));
+    p.a_bytes = a_rows * kBlockK * 2;
+    p.a_sh_bytes = a_sh_rows * kBlockK * 2;
+    GemmMaps m;
+    std::memset(&m, 0, sizeof(m));
+    if (!make_map(&m.a, h, n_rows, D.F, a_rows)) return MOE_ERR_CUDA;
+    if (!make_map(&m.b0, w->w_down, static_cast<uint64_t>(D.E) * D.d, D.F, n2)) return MOE_ERR_CUDA;
+    m.b1 = m.b0;
+    if (D.Fs > 0) {
+      if (!make_map(&m.a_sh, h_sh, D.T, D.Fs, a_sh_rows)) return MOE_ERR_CUDA;
+      if (!make_map(&m.b0_sh, w->ws_down, D.d, D.Fs, n2)) return MOE_ERR_CUDA;
+    } else {
+      m.a_sh = m.a;
+      m.b0_sh = m.b0;
+    }
+    m.b1_sh = m.b0_sh;
+    const int grid = sms;
+    ev.mark();
+    if (launch_gemm(MODE_GEMM2, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+    launches += 1;
+  }
+  // 5. combine: y = bf16(sum of the scaled routed slots + shared slot)
+  ev.mark();
+  if (launch_combine(slots, D.T, D.slots, D.d, static_cast<uint16_t *>(y), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  launches += 1;
+  ev.mark();
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_read_device_status(const void *ws, void *stream, int32_t *site) {
+  if (ws == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int hdr[2] = {0, 0};
+  if (cudaMemcpyAsync(hdr, ws, sizeof(hdr), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (site) *site = hdr[1];
+  return static_cast<moe_status>(hdr[0]);
+}
+
+moe_status moe_selftest_bounded_wait(void *ws, size_t ws_bytes, uint32_t limit_us, void *stream) {
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  int dev = 0, khz = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  moe_status st = clear_header(ws, s);
+  if (st != MOE_OK) return st;
+  const long long cycles = static_cast<long long>(limit_us) * (khz / 1000);
+  if (launch_selftest_wait(static_cast<int *>(ws), cycles, s) != cudaSuccess) return MOE_ERR_CUDA;
+  g_last_launches = 1;
+  return MOE_OK;
+}
+
+const char *moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+moe_status moe_profile_next_forward(void **events, int32_t n_events) {
+  if (events != nullptr && n_events < 1) return MOE_ERR_INVALID_ARG;
+  g_prof_events = events;
+  g_prof_n = events ? n_events : 0;
+  return MOE_OK;
+}
+
+}  // extern "C"

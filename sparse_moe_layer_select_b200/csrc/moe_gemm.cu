@@ -1,0 +1,495 @@
+// moe_gemm.cu -- persistent, warp-specialised tcgen05 GEMM for the MoE layer.
+//
+// One kernel template serves the three contractions of the layer:
+//
+//   MODE_ROUTER  logits[128 tokens, E] = x_tile . W_r^T, fp32 in TMEM; the
+//                epilogue keeps each token's top-k in registers and writes the
+//                normalised sigmoid weights (sigmoid router with post-top-k
+//                normalisation: Laguna M.1/XS.2 Technical Report summary, Key
+//                claims, report §3.1).
+//   MODE_GEMM1   [gate | up] = X_perm . [W_gate | W_up]^T for one expert and
+//                one column block; the rows of X_perm are gathered from x by
+//                TMA (tile::gather4) through the expert-order permutation, so
+//                the permuted activations are never written out.  The
+//                epilogue applies SwiGLU, h = silu(gate) * up, and stores h in
+//                bf16 (Laguna-M.1-base spec sheet, Feed-forward: SwiGLU, no bias).
+//   MODE_GEMM2   o = h . W_down^T for one expert and one d-column block; the
+//                epilogue multiplies each row by routed_scaling_factor * w
+//                (the 2.5 modulation of the routed sum: Technical Report
+//                summary, report §3.1) and writes it to that (token, slot)'s
+//                row of the slot buffer; shared-expert rows go to the last
+//                slot with scale 1.
+//
+// Roles inside a CTA (192 threads, one CTA per SM, persistent over items):
+//   warp 0      TMA producer: fills a kStages-deep ring of (A, B) stages.
+//   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma
+//               (M=128, N<=256, K=16 per instruction) into one of two
+//               accumulator buffers and commits stage releases.
+//   warps 2..5  epilogue: tcgen05.ld the finished accumulator (each thread
+//               owns one row), compute, store; release the buffer, so the
+//               MMA of the next item overlaps this epilogue.
+// Every wait is bounded (status.cuh); on expiry the kernel records
+// MOE_ERR_DEVICE_TIMEOUT, drains what it issued, frees TMEM and returns.
+#include <cuda_bf16.h>
+
+#include <cfloat>
+
+#include "kernels.h"
+#include "ptx.cuh"
+#include "status.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kABytes = kBlockM * kBlockK * 2;  // 16 KB: 128 rows x 128 bytes
+constexpr int kBBytesMax = 256 * kBlockK * 2;   // 32 KB: up to 256 rows
+constexpr int kTmemCols = 512;                  // two accumulators of up to 256 columns
+constexpr int kAccStride = 256;
+
+struct SmemLayout {
+  static constexpr int a_off = 0;
+  static constexpr int b_off = a_off + kStages * kABytes;
+  static constexpr int bar_off = b_off + kStages * kBBytesMax;
+  // full[S], empty[S], acc_full[2], acc_empty[2], drain
+  static constexpr int n_bars = 2 * kStages + 5;
+  static constexpr int tmem_slot_off = bar_off + n_bars * 8;
+  static constexpr int bias_off = (tmem_slot_off + 16 + 15) / 16 * 16;
+  static constexpr int total = bias_off + 512 * 4;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Per-item description shared by all roles.
+struct Item {
+  int group;   // expert id, E = shared expert, -1 = router tile
+  int row0;    // first row (expert-order row, token for shared/router)
+  int nrows;   // valid rows (<= 128)
+  int j;       // N tile index
+  int nk;      // K blocks
+  bool skip;   // no work (N tile beyond this group's width)
+};
+
+template <int MODE>
+__device__ __forceinline__ Item decode_item(const GemmParams &p, int item) {
+  Item it;
+  if (MODE == MODE_ROUTER) {
+    it.group = -1;
+    it.row0 = item * kBlockM;
+    it.nrows = min(kBlockM, p.T - it.row0);
+    it.j = 0;
+    it.nk = p.d / kBlockK;
+    it.skip = false;
+    return it;
+  }
+  const int ti = item / p.n_ntiles;
+  it.j = item - ti * p.n_ntiles;
+  const int4 t = *reinterpret_cast<const int4 *>(&p.tiles[ti]);
+  it.group = t.x;
+  it.row0 = t.y;
+  it.nrows = t.z;
+  const bool shared = it.group == p.E;
+  if (MODE == MODE_GEMM1) {
+    const int width = shared ? p.Fs : p.F;
+    it.skip = it.j * p.n_half >= width;
+    it.nk = p.d / kBlockK;
+  } else {
+    it.skip = false;
+    it.nk = (shared ? p.Fs : p.F) / kBlockK;
+  }
+  return it;
+}
+
+template <int KM>
+__device__ __forceinline__ void topk_insert(float (&bv)[KM], int (&bi)[KM], float v, int i) {
+  // Sorted descending; a candidate displaces only a strictly smaller value,
+  // and candidates arrive in ascending expert order, so equal logits keep
+  // the lower expert index first.
+#pragma unroll
+  for (int q = 0; q < KM; ++q) {
+    if (v > bv[q]) {
+      const float tv = bv[q];
+      const int ti = bi[q];
+      bv[q] = v;
+      bi[q] = i;
+      v = tv;
+      i = ti;
+    }
+  }
+}
+
+template <int KM>
+__device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item &it, uint32_t taddr,
+                                                int row_local, const float *bias_s) {
+  float bv[KM];
+  int bi[KM];
+#pragma unroll
+  for (int q = 0; q < KM; ++q) {
+    bv[q] = -FLT_MAX;
+    bi[q] = 0x7fffffff;
+  }
+  for (int c = 0; c < p.E; c += 32) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + c, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float v = __uint_as_float(r[i]) + bias_s[c + i];
+      if (c + i < p.E && v > bv[KM - 1]) topk_insert<KM>(bv, bi, v, c + i);
+    }
+  }
+  if (row_local < it.nrows) {
+    const size_t t = static_cast<size_t>(it.row0 + row_local);
+    float s[KM];
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < KM; ++q) {
+      s[q] = 1.f / (1.f + expf(-bv[q]));
+      if (q < p.k) sum += s[q];
+    }
+#pragma unroll
+    for (int q = 0; q < KM; ++q) {
+      if (q < p.k) {
+        p.topk_idx[t * p.k + q] = bi[q];
+        p.topk_w_out[t * p.k + q] = p.norm_topk ? s[q] / sum : s[q];
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item &it,
+                                                uint32_t taddr, int row_local) {
+  const bool shared = it.group == p.E;
+  const bool valid = row_local < it.nrows;
+  uint16_t *dst = shared ? p.h_shared + static_cast<size_t>(it.row0 + row_local) * p.Fs
+                         : p.h + static_cast<size_t>(it.row0 + row_local) * p.F;
+  dst += it.j * p.n_half;
+  for (int c = 0; c < p.n_half; c += 32) {
+    uint32_t g[32], u[32];
+    tmem_ld_32x32b_x32(taddr + c, g);
+    tmem_ld_32x32b_x32(taddr + p.n_half + c, u);
+    tmem_ld_wait();
+    uint32_t packed[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+      const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+      const float h0 = g0 / (1.f + __expf(-g0)) * u0;
+      const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+      packed[i] = pack_bf16x2(h0, h1);
+    }
+    if (valid) {
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        d4[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void slot_epilogue(const GemmParams &p, const Item &it, uint32_t taddr,
+                                              int row_local) {
+  const bool shared = it.group == p.E;
+  const bool valid = row_local < it.nrows;
+  float scale = 1.f;
+  size_t dst_row = 0;
+  if (valid) {
+    if (shared) {
+      const size_t t = static_cast<size_t>(it.row0 + row_local);
+      dst_row = t * p.slots + p.k;
+    } else {
+      const int pt = p.perm[it.row0 + row_local];
+      const int t = pt / p.k;
+      const int jslot = pt - t * p.k;
+      scale = p.routed_scale * p.topk_w[pt];
+      dst_row = static_cast<size_t>(t) * p.slots + jslot;
+    }
+  }
+  uint16_t *dst = p.slot_out + dst_row * p.d + static_cast<size_t>(it.j) * p.n_tile;
+  for (int c = 0; c < p.n_tile; c += 32) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + c, r);
+    tmem_ld_wait();
+    if (valid) {
+      uint32_t packed[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * scale,
+                                __uint_as_float(r[2 * i + 1]) * scale);
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        d4[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+    }
+  }
+}
+
+}  // namespace
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b0,
+                    const __grid_constant__ CUtensorMap tm_b1,
+                    const __grid_constant__ CUtensorMap tm_a_sh,
+                    const __grid_constant__ CUtensorMap tm_b0_sh,
+                    const __grid_constant__ CUtensorMap tm_b1_sh) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem + SmemLayout::a_off;
+  uint8_t *sB = smem + SmemLayout::b_off;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SmemLayout::bar_off);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + kStages;
+  uint64_t *acc_full = bars + 2 * kStages;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *drain = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot_off);
+  float *bias_s = reinterpret_cast<float *>(smem + SmemLayout::bias_off);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4 * 32);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (MODE == MODE_ROUTER) {
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) bias_s[e] = p.bias ? p.bias[e] : 0.f;
+    for (int e = p.E + threadIdx.x; e < 512; e += blockDim.x) bias_s[e] = 0.f;
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b0);
+    if (MODE == MODE_GEMM1) prefetch_tmap(&tm_b1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int n_items = (MODE == MODE_ROUTER) ? p.n_tiles_host : (*p.n_tiles_dev) * p.n_ntiles;
+  const uint32_t idesc = idesc_bf16_f32(kBlockM, p.n_tile);
+  int *status = p.status;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int s = 0;
+    uint32_t ph = 0;
+    long long issued = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const Item it = decode_item<MODE>(p, item);
+      if (it.skip) continue;
+      if (status_is_set(status)) break;
+      const bool shared = it.group == p.E;
+      // GEMM1: each lane gathers 4 of the tile's 128 rows (token ids).
+      int tok[4] = {0, 0, 0, 0};
+      if (MODE == MODE_GEMM1) {
+        int first;
+        if (shared) {
+          first = it.row0;
+        } else {
+          first = p.perm[it.row0] / p.k;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int r = 4 * lane + q;
+          int t = first;
+          if (r < it.nrows) t = shared ? it.row0 + r : p.perm[it.row0 + r] / p.k;
+          tok[q] = t;
+        }
+      }
+      // A boxes shorter than 128 rows (tensors with fewer rows) fill only
+      // their rows; the rest of the stage feeds accumulator rows that the
+      // epilogue discards.
+      uint32_t bytes;
+      if (MODE == MODE_ROUTER) bytes = p.a_bytes + p.E * 128;
+      else if (MODE == MODE_GEMM1) bytes = kABytes + 2 * p.n_half * 128;
+      else bytes = (shared ? p.a_sh_bytes : p.a_bytes) + p.n_tile * 128;
+      for (int kb = 0; kb < it.nk; ++kb) {
+        int good = 1;
+        if (lane == 0) {
+          good = mbar_wait(&empty[s], ph ^ 1, status, SITE_GEMM_PRODUCER_EMPTY);
+          if (good) mbar_arrive_expect_tx(&full[s], bytes);
+        }
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
+          ok = false;
+          break;
+        }
+        uint8_t *a_dst = sA + s * kABytes;
+        uint8_t *b_dst = sB + s * kBBytesMax;
+        const int kc = kb * kBlockK;
+        if (MODE == MODE_GEMM1) {
+          tma_gather4(a_dst + lane * 4 * 128, &tm_a, &full[s], kc, tok[0], tok[1], tok[2], tok[3]);
+          if (lane == 0) {
+            const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
+            tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
+            tma_load_2d(b_dst + p.n_half * 128, shared ? &tm_b1_sh : &tm_b1, &full[s], kc, brow);
+          }
+        } else if (lane == 0) {
+          if (MODE == MODE_ROUTER) {
+            tma_load_2d(a_dst, &tm_a, &full[s], kc, it.row0);
+            tma_load_2d(b_dst, &tm_b0, &full[s], kc, 0);
+          } else {
+            tma_load_2d(a_dst, shared ? &tm_a_sh : &tm_a, &full[s], kc, it.row0);
+            const int brow = (shared ? 0 : it.group * p.d) + it.j * p.n_tile;
+            tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
+          }
+        }
+        ++issued;
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+    // Drain: every stage this warp filled must have landed before the CTA exits.
+    if (lane == 0) {
+      for (long long n = (issued > kStages ? issued - kStages : 0); n < issued; ++n)
+        if (!mbar_wait(&full[n % kStages], static_cast<uint32_t>((n / kStages) & 1), status,
+                       SITE_GEMM_DRAIN))
+          break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const Item it = decode_item<MODE>(p, item);
+        if (it.skip) continue;
+        if (status_is_set(status)) break;
+        if (!mbar_wait(&acc_empty[acc], aph ^ 1, status, SITE_GEMM_MMA_ACC_EMPTY)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kAccStride;
+        for (int kb = 0; kb < it.nk; ++kb) {
+          if (!mbar_wait(&full[s], ph, status, SITE_GEMM_MMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kABytes);
+          const uint32_t b0 = smem_u32(sB + s * kBBytesMax);
+#pragma unroll
+          for (int kk = 0; kk < kBlockK / 16; ++kk) {
+            umma_bf16_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+                         idesc, (kb | kk) != 0);
+          }
+          umma_commit(&empty[s]);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1;
+        }
+      }
+      // All MMAs issued by this thread complete before TMEM is released.
+      umma_commit(drain);
+      mbar_wait(drain, 0, status, SITE_GEMM_DRAIN);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_local = q * 32 + lane;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const Item it = decode_item<MODE>(p, item);
+      if (it.skip) continue;
+      if (status_is_set(status)) break;
+      if (!mbar_wait(&acc_full[acc], aph, status, SITE_GEMM_EPI_ACC_FULL)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccStride;
+      if (MODE == MODE_ROUTER) {
+        if (p.k <= 4) router_epilogue<4>(p, it, taddr, row_local, bias_s);
+        else if (p.k <= 8) router_epilogue<8>(p, it, taddr, row_local, bias_s);
+        else router_epilogue<16>(p, it, taddr, row_local, bias_s);
+      } else if (MODE == MODE_GEMM1) {
+        swiglu_epilogue(p, it, taddr, row_local);
+      } else {
+        slot_epilogue(p, it, taddr, row_local);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
+
+cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int grid,
+                        cudaStream_t s) {
+  const size_t smem = gemm_smem_bytes();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  switch (mode) {
+    case MODE_ROUTER:
+      return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_ROUTER>, p, m.a, m.b0, m.b1, m.a_sh,
+                                m.b0_sh, m.b1_sh);
+    case MODE_GEMM1:
+      return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM1>, p, m.a, m.b0, m.b1, m.a_sh,
+                                m.b0_sh, m.b1_sh);
+    default:
+      return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM2>, p, m.a, m.b0, m.b1, m.a_sh,
+                                m.b0_sh, m.b1_sh);
+  }
+}
+
+// Raise the dynamic shared-memory limit of the three instantiations (once per device).
+cudaError_t gemm_set_attributes() {
+  const int smem = static_cast<int>(gemm_smem_bytes());
+  cudaError_t e;
+  e = cudaFuncSetAttribute(moe_gemm_kernel<MODE_ROUTER>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM1>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM2>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+}  // namespace moe

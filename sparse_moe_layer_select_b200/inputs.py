@@ -238,6 +238,16 @@ def generate_numpy(shape, seed: int, tensor_id: int, sigma: float, start: int = 
     return f64_to_bf16_bits(z * float(sigma)).reshape(shape)
 
 
+def generate_numpy_chunked(shape, seed: int, tensor_id: int, sigma: float, chunk: int = 1 << 24):
+    """generate_numpy for large tensors, drawn in slices to bound host memory."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    for s in range(0, n, chunk):
+        m = min(chunk, n - s)
+        out[s:s + m] = generate_numpy((m,), seed, tensor_id, sigma, start=s)
+    return out.reshape(shape)
+
+
 def zipf_rank(E: int):
     """Popularity rank r_e in 1..E of each expert: a seed-1 Philox permutation."""
     e = np.arange(E, dtype=np.uint64)

@@ -1,0 +1,249 @@
+"""Python binding of the C ABI in include/moe.h (argument marshalling only).
+
+Every step of the layer runs in the CUDA kernels of libmoe_b200.so; this
+module only turns torch tensors into device pointers and checks status
+codes.  There is no fallback: if the library is missing, importing the
+functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED_SHAPE = 2
+MOE_ERR_WORKSPACE_TOO_SMALL = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE_TIMEOUT = 5
+MOE_ERR_DEVICE_BOUNDS = 6
+
+MOE_FLAG_ROUTER_CUDA_CORE = 1
+MOE_FLAG_ROUTER_TENSOR = 2
+
+# Every symbol the header declares (checked by the CPU tests).
+EXPORTED = ["moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
+            "moe_read_device_status", "moe_selftest_bounded_wait", "moe_status_string",
+            "moe_last_launch_count", "moe_profile_next_forward"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+class moe_dims_t(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("T", ctypes.c_int32),
+                ("d_model", ctypes.c_int32), ("num_experts", ctypes.c_int32),
+                ("num_experts_per_tok", ctypes.c_int32), ("moe_intermediate_size", ctypes.c_int32),
+                ("shared_intermediate_size", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float), ("norm_topk_prob", ctypes.c_int32),
+                ("flags", ctypes.c_int32)]
+
+
+class moe_weights_t(ctypes.Structure):
+    _fields_ = [("w_router", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+                ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
+                ("w_down", ctypes.c_void_p), ("ws_gate", ctypes.c_void_p),
+                ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p)]
+
+
+class moe_routing_t(ctypes.Structure):
+    _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p),
+                ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("perm", ctypes.c_void_p)]
+
+
+_LIB = None
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} "
+                               "(run python -m sparse_moe_layer_select_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        D = ctypes.POINTER(moe_dims_t)
+        L.moe_workspace_size.restype = ctypes.c_size_t
+        L.moe_workspace_size.argtypes = [D]
+        L.moe_route.restype = ctypes.c_int
+        L.moe_route.argtypes = [D, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_permute.restype = ctypes.c_int
+        L.moe_permute.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_forward.restype = ctypes.c_int
+        L.moe_forward.argtypes = [D, ctypes.POINTER(moe_weights_t), P, P,
+                                  ctypes.POINTER(moe_routing_t), P, ctypes.c_size_t, P]
+        L.moe_read_device_status.restype = ctypes.c_int
+        L.moe_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+        L.moe_selftest_bounded_wait.restype = ctypes.c_int
+        L.moe_selftest_bounded_wait.argtypes = [P, ctypes.c_size_t, ctypes.c_uint32, P]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_last_launch_count.restype = ctypes.c_int32
+        L.moe_last_launch_count.argtypes = []
+        L.moe_profile_next_forward.restype = ctypes.c_int
+        L.moe_profile_next_forward.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+        _LIB = L
+    return _LIB
+
+
+def status_string(code: int) -> str:
+    return lib().moe_status_string(code).decode()
+
+
+def make_dims(T, d_model, num_experts, num_experts_per_tok, moe_intermediate_size,
+              shared_intermediate_size, routed_scaling_factor=2.5, norm_topk_prob=1, flags=0):
+    return moe_dims_t(ctypes.sizeof(moe_dims_t), T, d_model, num_experts, num_experts_per_tok,
+                      moe_intermediate_size, shared_intermediate_size, routed_scaling_factor,
+                      norm_topk_prob, flags)
+
+
+def dims_for(w, T=None, flags=0):
+    """moe_dims_t of an inputs.Workload (optionally with another token count)."""
+    return make_dims(w.T if T is None else T, w.d_model, w.E, w.k, w.F, w.Fs,
+                     w.routed_scaling_factor, 1, flags)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code, where):
+    if code != MOE_OK:
+        raise MoeError(code, where)
+
+
+def workspace_size(dims) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(dims)))
+
+
+def alloc_workspace(dims, device="cuda"):
+    import torch
+    n = workspace_size(dims)
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def route(dims, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
+    _check(lib().moe_route(ctypes.byref(dims), _p(x), _p(w_router), _p(bias), _p(topk_idx),
+                           _p(topk_w), _p(ws), ws.numel(), _stream(stream)), "moe_route")
+
+
+def permute(dims, topk_idx, counts, offsets, perm, ws, x=None, x_perm=None, stream=None):
+    _check(lib().moe_permute(ctypes.byref(dims), _p(topk_idx), _p(counts), _p(offsets), _p(perm),
+                             _p(x), _p(x_perm), _p(ws), ws.numel(), _stream(stream)),
+           "moe_permute")
+
+
+def weights_struct(W):
+    return moe_weights_t(*[None if W.get(k) is None else W[k].data_ptr() for k in
+                           ("w_router", "router_bias", "w_gate", "w_up", "w_down", "ws_gate",
+                            "ws_up", "ws_down")])
+
+
+def routing_struct(R):
+    return moe_routing_t(*[R[k].data_ptr() for k in ("topk_idx", "topk_w", "counts", "offsets",
+                                                     "perm")])
+
+
+def forward(dims, weights, x, y, routing, ws, stream=None):
+    """moe_forward on torch tensors; weights/routing are dicts of tensors (or prebuilt structs)."""
+    ws_s = weights if isinstance(weights, moe_weights_t) else weights_struct(weights)
+    r_s = routing if isinstance(routing, moe_routing_t) else routing_struct(routing)
+    _check(lib().moe_forward(ctypes.byref(dims), ctypes.byref(ws_s), _p(x), _p(y),
+                             ctypes.byref(r_s), _p(ws), ws.numel(), _stream(stream)),
+           "moe_forward")
+
+
+def alloc_routing(dims, device="cuda"):
+    import torch
+    T, k, E = dims.T, dims.num_experts_per_tok, dims.num_experts
+    return {"topk_idx": torch.empty((T, k), dtype=torch.int32, device=device),
+            "topk_w": torch.empty((T, k), dtype=torch.float32, device=device),
+            "counts": torch.empty(E, dtype=torch.int32, device=device),
+            "offsets": torch.empty(E + 1, dtype=torch.int32, device=device),
+            "perm": torch.empty(T * k, dtype=torch.int32, device=device)}
+
+
+def read_device_status(ws, stream=None):
+    site = ctypes.c_int32(0)
+    code = lib().moe_read_device_status(_p(ws), _stream(stream), ctypes.byref(site))
+    return int(code), int(site.value)
+
+
+def selftest_bounded_wait(ws, limit_us, stream=None):
+    _check(lib().moe_selftest_bounded_wait(_p(ws), ws.numel(), limit_us, _stream(stream)),
+           "moe_selftest_bounded_wait")
+
+
+def profile_next_forward(events):
+    """Arm per-kernel event recording for the next forward call (torch.cuda.Event list)."""
+    if events is None:
+        _check(lib().moe_profile_next_forward(None, 0), "moe_profile_next_forward")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    profile_next_forward._keep = arr
+    _check(lib().moe_profile_next_forward(arr, len(events)), "moe_profile_next_forward")
+
+
+# Stage names of the kernel-marker intervals recorded by moe_forward, in order.
+FORWARD_STAGES = ("router", "index", "gemm1_swiglu", "gemm2_down_scale", "combine")
+
+
+def last_launch_count() -> int:
+    return int(lib().moe_last_launch_count())
+
+
+class MoeLayer:
+    """A layer instance: device weights, routing buffers and workspace, reused across calls."""
+
+    def __init__(self, weights: dict, d_model, num_experts, num_experts_per_tok,
+                 moe_intermediate_size, shared_intermediate_size, routed_scaling_factor=2.5,
+                 max_tokens=1, flags=0, device="cuda"):
+        self.W = weights
+        self.cfg = dict(d_model=d_model, num_experts=num_experts,
+                        num_experts_per_tok=num_experts_per_tok,
+                        moe_intermediate_size=moe_intermediate_size,
+                        shared_intermediate_size=shared_intermediate_size,
+                        routed_scaling_factor=routed_scaling_factor, flags=flags)
+        self.device = device
+        self._ws_struct = weights_struct(weights)
+        self._reserve(max_tokens)
+
+    def dims(self, T):
+        c = self.cfg
+        return make_dims(T, c["d_model"], c["num_experts"], c["num_experts_per_tok"],
+                         c["moe_intermediate_size"], c["shared_intermediate_size"],
+                         c["routed_scaling_factor"], 1, c["flags"])
+
+    def _reserve(self, T):
+        self.max_tokens = T
+        d = self.dims(T)
+        self.ws = alloc_workspace(d, self.device)
+        self.routing = alloc_routing(d, self.device)
+        self._r_struct = routing_struct(self.routing)
+
+    def forward(self, x, y=None, stream=None):
+        import torch
+        T = x.shape[0]
+        if T > self.max_tokens:
+            self._reserve(T)
+        if y is None:
+            y = torch.empty_like(x)
+        d = self.dims(T)
+        forward(d, self._ws_struct, x, y, self._r_struct, self.ws, stream)
+        return y

@@ -1,0 +1,107 @@
+"""The C ABI library: it builds, loads, exports every declared symbol, and its
+host-side argument checks return the documented codes (no GPU needed: these
+paths return before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_moe_layer_select_b200 import build as B
+from sparse_moe_layer_select_b200 import moe as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return M.lib()
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared_functions()
+    assert "moe_forward" in declared and "moe_route" in declared and "moe_permute" in declared
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(M.EXPORTED) == declared
+
+
+def test_generator_library_exports(L):
+    import sparse_moe_layer_select_b200.inputs as I
+    assert hasattr(I._gen_lib(), "moe_gen_normal_bf16")
+
+
+def test_status_strings(L):
+    for code, name in [(0, "MOE_OK"), (1, "MOE_ERR_INVALID_ARG"), (2, "MOE_ERR_UNSUPPORTED_SHAPE"),
+                       (3, "MOE_ERR_WORKSPACE_TOO_SMALL"), (4, "MOE_ERR_CUDA"),
+                       (5, "MOE_ERR_DEVICE_TIMEOUT"), (6, "MOE_ERR_DEVICE_BOUNDS")]:
+        assert M.status_string(code) == name
+
+
+def test_workspace_size_and_shape_limits(L):
+    ok = M.make_dims(4096, 2048, 256, 8, 512, 512)
+    n = M.workspace_size(ok)
+    # slots alone: T * (k + 1) * d * 2 bytes
+    assert n >= 4096 * 9 * 2048 * 2 and n % 256 == 0
+    bad = [M.make_dims(64, 100, 16, 4, 128, 128),      # d not a multiple of 128
+           M.make_dims(64, 256, 16, 17, 128, 128),     # k > 16
+           M.make_dims(64, 256, 4, 5, 128, 128),       # k > E
+           M.make_dims(64, 256, 1024, 4, 128, 128),    # E > 512
+           M.make_dims(64, 256, 16, 4, 96, 128),       # F not a multiple of 64
+           M.make_dims(64, 256, 16, 4, 128, 32)]       # Fs not a multiple of 64
+    for d in bad:
+        assert M.workspace_size(d) == 0
+    d = M.make_dims(64, 256, 16, 4, 128, 128)
+    d.struct_size = 4
+    assert M.workspace_size(d) == 0
+
+
+def _call_forward(dims, x=256, y=512, ws=4096, ws_bytes=1 << 40, weights=None, routing=None):
+    w = weights or M.moe_weights_t(1024, None, 2048, 4096, 8192, 16384, 32768, 65536)
+    r = routing or M.moe_routing_t(1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20)
+    return M.lib().moe_forward(ctypes.byref(dims), ctypes.byref(w), ctypes.c_void_p(x),
+                               ctypes.c_void_p(y), ctypes.byref(r), ctypes.c_void_p(ws), ws_bytes,
+                               None)
+
+
+def test_argument_errors_return_before_any_launch(L):
+    d = M.make_dims(64, 256, 16, 4, 128, 128)
+    # fake device addresses are never dereferenced on these paths
+    assert _call_forward(d, x=0) == M.MOE_ERR_INVALID_ARG
+    assert _call_forward(d, x=256 + 8) == M.MOE_ERR_INVALID_ARG          # misaligned
+    assert _call_forward(d, ws=4096 + 16) == M.MOE_ERR_INVALID_ARG       # ws not 256-aligned
+    assert _call_forward(d, ws_bytes=1024) == M.MOE_ERR_WORKSPACE_TOO_SMALL
+    bad = M.make_dims(64, 256, 16, 4, 128, 32)
+    assert _call_forward(bad) == M.MOE_ERR_UNSUPPORTED_SHAPE
+    w = M.moe_weights_t(1024, None, 2048, 4096, 8192, None, None, None)  # shared missing
+    assert _call_forward(d, weights=w) == M.MOE_ERR_INVALID_ARG
+    r = M.moe_routing_t(1 << 20, 2 << 20, 0, 4 << 20, 5 << 20)
+    assert _call_forward(d, routing=r) == M.MOE_ERR_INVALID_ARG
+    # forced tensor-core router with an E it cannot take
+    f = M.make_dims(64, 256, 24, 4, 128, 128, flags=M.MOE_FLAG_ROUTER_TENSOR)
+    assert _call_forward(f) == M.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+def test_zero_tokens_is_a_noop(L):
+    d = M.make_dims(0, 256, 16, 4, 128, 128)
+    assert _call_forward(d) == M.MOE_OK
+    rc = L.moe_route(ctypes.byref(d), ctypes.c_void_p(256), ctypes.c_void_p(512), None,
+                     ctypes.c_void_p(768), ctypes.c_void_p(1024), ctypes.c_void_p(4096),
+                     1 << 30, None)
+    assert rc == M.MOE_OK
+    rc = L.moe_permute(ctypes.byref(d), ctypes.c_void_p(256), ctypes.c_void_p(512),
+                       ctypes.c_void_p(768), ctypes.c_void_p(1024), None, None,
+                       ctypes.c_void_p(4096), 1 << 30, None)
+    assert rc == M.MOE_OK
+    rc = L.moe_permute(ctypes.byref(d), ctypes.c_void_p(256), ctypes.c_void_p(512),
+                       ctypes.c_void_p(768), ctypes.c_void_p(1024), ctypes.c_void_p(256), None,
+                       ctypes.c_void_p(4096), 1 << 30, None)
+    assert rc == M.MOE_ERR_INVALID_ARG  # x without x_perm

@@ -1,0 +1,297 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Selection: bit-exact index sets and counts except the exempt near-ties
+(tests/parity.py); weights within 1e-5; output within relative Frobenius
+1e-2 and |dy| <= 2e-2 (|y| + 0.05) per element.  Permutation: bit-exact.
+"""
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+from sparse_moe_layer_select_b200 import inputs as I
+from sparse_moe_layer_select_b200 import moe as M
+from tests import gpu_common as G
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    torch.cuda.set_device(0)
+    from sparse_moe_layer_select_b200 import build as B
+    B.build()
+    yield
+
+
+# ------------------------------------------------------------------ generator
+
+def test_cuda_generator_matches_numpy_bit_for_bit():
+    import torch
+    for tid, sigma, start in [(0, 1.0, 0), (3, 0.02, 12345), (5, 0.015, 7), (101, 1.0, 0)]:
+        n = 1 << 20
+        t = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        I.generate_cuda(t, 0, tid, sigma, start=start)
+        got = P.to_numpy_bf16(t)
+        ref = I.generate_numpy((n,), 0, tid, sigma, start=start)
+        assert np.array_equal(got, ref), (tid, int((got != ref).sum()))
+
+
+# ------------------------------------------------------------------ tiny workload
+
+def _small(w):
+    h = I.host_inputs(w)
+    return h, G.host_to_device(h)
+
+
+def test_tiny_forward_matches_oracle():
+    w = I.get("c1_tiny")
+    h, dev = _small(w)
+    y, routing, _ = G.run_forward(w, dev)
+    ref = G.oracle_forward(w, h)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
+    G.check_output(G.y_numpy(y), ref["y"], what="c1")
+    counts, offsets, perm = O.expert_order(ref["topk_idx"], w.E)
+    assert np.array_equal(routing["counts"].cpu().numpy(), counts)
+    assert np.array_equal(routing["offsets"].cpu().numpy(), offsets)
+    assert np.array_equal(routing["perm"].cpu().numpy(), perm)
+
+
+@pytest.mark.parametrize("flags", [M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR])
+@pytest.mark.parametrize("T", [1, 64, 127, 128, 129, 1000])
+def test_router_paths_match_oracle(flags, T):
+    import torch
+    w = I.get("c1_tiny").with_(T=T)
+    h, dev = _small(w)
+    dims = M.dims_for(w, flags=flags)
+    ws = M.alloc_workspace(dims)
+    idx = torch.empty((T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((T, w.k), dtype=torch.float32, device="cuda")
+    M.route(dims, dev["x"], dev["w_router"], None, idx, wt, ws)
+    torch.cuda.synchronize()
+    assert M.read_device_status(ws)[0] == 0
+    ridx, rw, scores, _ = O.route(h["x"], h["w_router"], None, w.k)
+    ref = {"topk_idx": ridx, "topk_w": rw, "scores": scores}
+    G.check_routing(idx.cpu().numpy(), wt.cpu().numpy(), ref, w.k)
+
+
+@pytest.mark.parametrize("T", [1, 127, 128, 129, 1000])
+def test_ragged_and_multi_tile_forward(T):
+    w = I.get("c1_tiny").with_(T=T)
+    h, dev = _small(w)
+    y, routing, _ = G.run_forward(w, dev)
+    ref = G.oracle_forward(w, h)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
+    G.check_output(G.y_numpy(y), ref["y"], what=f"T={T}")
+
+
+def test_permute_materialised_gather_and_counts():
+    import torch
+    w = I.get("c1_tiny").with_(T=1000)
+    h, dev = _small(w)
+    ridx = O.route(h["x"], h["w_router"], None, w.k)[0]
+    dims = M.dims_for(w)
+    ws = M.alloc_workspace(dims)
+    idx = torch.from_numpy(ridx.astype(np.int32)).cuda()
+    counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(w.T * w.k, dtype=torch.int32, device="cuda")
+    xp = torch.empty((w.T * w.k, w.d_model), dtype=torch.bfloat16, device="cuda")
+    M.permute(dims, idx, counts, offsets, perm, ws, x=dev["x"], x_perm=xp)
+    torch.cuda.synchronize()
+    assert M.read_device_status(ws)[0] == 0
+    c, o, p = O.expert_order(ridx, w.E)
+    assert np.array_equal(counts.cpu().numpy(), c)
+    assert np.array_equal(offsets.cpu().numpy(), o)
+    assert np.array_equal(perm.cpu().numpy(), p)
+    assert np.array_equal(P.to_numpy_bf16(xp), h["x"][p // w.k])
+
+
+def test_bad_expert_id_sets_bounds_status():
+    import torch
+    w = I.get("c1_tiny")
+    dims = M.dims_for(w)
+    ws = M.alloc_workspace(dims)
+    idx = torch.zeros((w.T, w.k), dtype=torch.int32, device="cuda")
+    idx[5, 2] = w.E  # out of range
+    counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(w.T * w.k, dtype=torch.int32, device="cuda")
+    M.permute(dims, idx, counts, offsets, perm, ws)
+    code, site = M.read_device_status(ws)
+    assert code == M.MOE_ERR_DEVICE_BOUNDS and site == 20
+
+
+def test_device_wait_timeout_is_reported_and_context_survives():
+    import torch
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    M.selftest_bounded_wait(ws, 2000)
+    code, site = M.read_device_status(ws)
+    assert code == M.MOE_ERR_DEVICE_TIMEOUT and site == 90
+    # the context is still usable: a normal layer call succeeds afterwards
+    w = I.get("c1_tiny")
+    h, dev = _small(w)
+    y, _, _ = G.run_forward(w, dev)
+    G.check_output(G.y_numpy(y), G.oracle_forward(w, h)["y"], what="after timeout")
+
+
+# ------------------------------------------------------------------ special cases
+
+def test_no_shared_expert():
+    w = I.get("c1_tiny").with_(T=300, shared_intermediate_size=0)
+    h, dev = _small(w)
+    y, _, _ = G.run_forward(w, dev)
+    ref = G.oracle_forward(w, h)
+    assert np.array_equal(ref["Sh"], np.zeros_like(ref["Sh"]))
+    G.check_output(G.y_numpy(y), ref["y"], what="Fs=0")
+
+
+def test_zero_shared_weights_isolate_routed_path():
+    import torch
+    w = I.get("c1_tiny").with_(T=200)
+    h, dev = _small(w)
+    for key in ("ws_gate", "ws_up", "ws_down"):
+        h[key] = np.zeros_like(h[key])
+        dev[key] = torch.zeros_like(dev[key])
+    y, _, _ = G.run_forward(w, dev)
+    ref = G.oracle_forward(w, h)
+    G.check_output(G.y_numpy(y), 2.5 * ref["R"], what="shared=0")
+
+
+@pytest.mark.parametrize("E,k", [(2, 1), (2, 2), (4, 1), (4, 3), (8, 1), (8, 4), (8, 8), (16, 16)])
+def test_small_expert_counts_and_k_extremes(E, k):
+    w = I.get("c1_tiny").with_(T=257, num_experts=E, num_experts_per_tok=k)
+    h, dev = _small(w)
+    y, routing, _ = G.run_forward(w, dev)
+    ref = G.oracle_forward(w, h)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, k)
+    G.check_output(G.y_numpy(y), ref["y"], what=f"E={E},k={k}")
+
+
+def test_exact_ties_go_to_lower_expert_index():
+    w = I.get("c1_tiny").with_(T=256)
+    h, _ = _small(w)
+    wr = h["w_router"].copy()
+    wr[9] = wr[2]   # experts 2 and 9, and 5 and 14, have identical logits for every token
+    wr[14] = wr[5]
+    h["w_router"] = wr
+    dev = G.host_to_device(h)
+    for flags in (M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR):
+        y, routing, _ = G.run_forward(w, dev, flags=flags)
+        idx = routing["topk_idx"].cpu().numpy()
+        ref = G.oracle_forward(w, h)
+        for t in range(w.T):
+            s = set(idx[t].tolist())
+            assert not (9 in s and 2 not in s) and not (14 in s and 5 not in s), (t, idx[t])
+        G.check_routing(idx, routing["topk_w"].cpu().numpy(), ref, w.k)
+        G.check_output(G.y_numpy(y), ref["y"], what="ties")
+
+
+def test_maximum_skew_all_tokens_on_the_same_experts():
+    import torch
+    w = I.get("c1_tiny").with_(T=1000)
+    h, dev = _small(w)
+    bias = np.zeros(w.E, dtype=np.float32)
+    bias[[3, 7, 11, 12]] = 100.0   # every token selects experts 3, 7, 11, 12
+    h["router_bias"] = bias
+    dev["router_bias"] = torch.from_numpy(bias).cuda()
+    y, routing, _ = G.run_forward(w, dev)
+    counts = routing["counts"].cpu().numpy()
+    assert counts[[3, 7, 11, 12]].tolist() == [1000] * 4 and counts.sum() == 4000
+    ref = G.oracle_forward(w, h)
+    G.check_output(G.y_numpy(y), ref["y"], what="max skew")
+
+
+def test_output_guard_bands_untouched():
+    import torch
+    w = I.get("c1_tiny").with_(T=300)
+    h, dev = _small(w)
+    big = torch.full((w.T + 2, w.d_model), 7.0, dtype=torch.bfloat16, device="cuda")
+    y_view = big[1:w.T + 1]
+    dims = M.dims_for(w)
+    ws = M.alloc_workspace(dims)
+    routing = M.alloc_routing(dims)
+    M.forward(dims, dev, dev["x"], y_view, routing, ws)
+    torch.cuda.synchronize()
+    assert bool((big[0] == 7.0).all()) and bool((big[-1] == 7.0).all())
+    G.check_output(G.y_numpy(y_view), G.oracle_forward(w, h)["y"], what="guard")
+
+
+def test_redundant_runs_are_bit_identical():
+    """The same inputs five times: routing, permutation and y identical bit for bit."""
+    import torch
+    w = I.get("c1_tiny").with_(T=1000)
+    _, dev = _small(w)
+    outs = []
+    for _ in range(5):
+        y, routing, _ = G.run_forward(w, dev)
+        outs.append((P.to_numpy_bf16(y), routing["topk_idx"].cpu().numpy(),
+                     routing["topk_w"].cpu().numpy(), routing["perm"].cpu().numpy()))
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _device_workload(w):
+    dev = I.device_inputs(w)
+    h = G.device_to_host(dev)
+    return h, dev
+
+
+def test_xs2_dims_multi_tile_full_oracle():
+    """XS.2 widths at T=1000: every token through the oracle (ragged tiles everywhere)."""
+    w = I.get("c2_xs2_small").with_(T=1000)
+    h, dev = _device_workload(w)
+    y, routing, _ = G.run_forward(w, dev)
+    ref = G.oracle_forward(w, h)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
+    same = P.same_selection_mask(routing["topk_idx"].cpu().numpy(), ref["topk_idx"])
+    G.check_output(G.y_numpy(y), ref["y"], rows_ok=same, what="xs2 T=1000")
+
+
+@pytest.mark.parametrize("name,n_sample", [("c2_xs2_small", 1024), ("c3_xs2_prefill_zipf", 1024),
+                                           ("c4_m1_width", 256)])
+def test_full_size_workloads(name, n_sample):
+    """Routing and counts on every token; y on a seeded sample of tokens."""
+    w = I.get(name)
+    h, dev = _device_workload(w)
+    y, routing, _ = G.run_forward(w, dev)
+    gidx = routing["topk_idx"].cpu().numpy()
+    gw = routing["topk_w"].cpu().numpy()
+    ridx, rw, scores, _ = O.route(h["x"], h["w_router"], h["router_bias"], w.k)
+    n_ex, n_diff = G.check_routing(gidx, gw, {"topk_idx": ridx, "topk_w": rw, "scores": scores},
+                                   w.k)
+    c, o, p = O.expert_order(gidx, w.E)   # the permutation of the (accepted) GPU selection
+    assert np.array_equal(routing["counts"].cpu().numpy(), c)
+    assert np.array_equal(routing["offsets"].cpu().numpy(), o)
+    assert np.array_equal(routing["perm"].cpu().numpy(), p)
+    if n_diff == 0:
+        assert np.array_equal(c, np.bincount(ridx.reshape(-1), minlength=w.E))
+    rng = np.random.default_rng(1234)
+    rows = np.sort(rng.choice(w.T, size=n_sample, replace=False))
+    ref = G.oracle_forward(w, h, rows=rows)
+    same = P.same_selection_mask(gidx[rows], ref["topk_idx"])
+    G.check_output(G.y_numpy(y)[rows], ref["y"], rows_ok=same, what=name)
+
+
+def test_decode_fresh_batches():
+    import torch
+    w = I.get("c5_decode")
+    dev = I.device_inputs(w)
+    h = G.device_to_host(dev)
+    layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
+                       max_tokens=w.T)
+    ring = I.device_decode_ring(w, 3)
+    for i in range(3):
+        y = layer.forward(ring[i])
+        torch.cuda.synchronize()
+        hx = dict(h, x=P.to_numpy_bf16(ring[i]))
+        assert np.array_equal(hx["x"], I.decode_batch_host(w, i))
+        ref = G.oracle_forward(w, hx)
+        idx = layer.routing["topk_idx"][:w.T].cpu().numpy()
+        G.check_routing(idx, layer.routing["topk_w"][:w.T].cpu().numpy(), ref, w.k)
+        same = P.same_selection_mask(idx, ref["topk_idx"])
+        G.check_output(G.y_numpy(y), ref["y"], rows_ok=same, what=f"decode batch {i}")
