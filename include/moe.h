@@ -77,6 +77,13 @@ typedef struct {
  * selection rule; the choice only changes speed). */
 #define MOE_FLAG_ROUTER_CUDA_CORE 1   /* fp32 FMA logits + warp-per-token top-k */
 #define MOE_FLAG_ROUTER_TENSOR    2   /* tcgen05 logits with the top-k in the epilogue */
+/* The caller passes fp16 copies of the down projections (w_down_f16,
+ * ws_down_f16, made once by moe_prepare_down_f16); without this flag
+ * moe_forward converts them into the workspace on every call. */
+#define MOE_FLAG_DOWN_F16         4
+/* Both router paths also write the fp32 logits (bias included) to the
+ * workspace, at the byte offset returned by moe_logits_offset. */
+#define MOE_FLAG_WRITE_LOGITS     8
 
 typedef struct {
     const void *w_router;      /* [E, d] bf16 */
@@ -87,6 +94,8 @@ typedef struct {
     const void *ws_gate;       /* [Fs, d] bf16, NULL if Fs = 0 */
     const void *ws_up;         /* [Fs, d] bf16 */
     const void *ws_down;       /* [d, Fs] bf16 */
+    const void *w_down_f16;    /* [E, d, F] fp16 copy of w_down (with MOE_FLAG_DOWN_F16) */
+    const void *ws_down_f16;   /* [d, Fs] fp16 copy of ws_down (with MOE_FLAG_DOWN_F16) */
 } moe_weights_t;
 
 /* Routing outputs of moe_forward (caller-owned device memory, all required). */
@@ -129,11 +138,30 @@ moe_status moe_permute(const moe_dims_t *dims, const int32_t *topk_idx, int32_t 
  * GEMMs (gather of the permuted rows fused into the operand load), the shared
  * expert, the routed_scaling_factor modulation and the weighted combine.
  * x: [T, d] bf16 in; y: [T, d] bf16 out.  `routing` receives the router and
- * permutation results.  Accumulation is fp32; the SwiGLU activation h is
- * rounded to bf16 before the down projection, and y is rounded to bf16. */
+ * permutation results.  Precision: all accumulation is fp32; the SwiGLU
+ * activation h enters the down projection as fp16 (against an fp16 copy of
+ * W_down), each scaled routed contribution and the shared output are held in
+ * fp16 before the fp32 combine, and y is rounded to bf16.  A value beyond the
+ * fp16 range (|v| > 65504) in h or in a contribution sets
+ * MOE_ERR_DEVICE_BOUNDS in the status word. */
 moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *weights, const void *x,
                        void *y, const moe_routing_t *routing, void *ws, size_t ws_bytes,
                        void *stream);
+
+/* One-time preparation of the down projections for moe_forward: fp16 copies
+ * w_down_f16 [E, d, F] and ws_down_f16 [d, Fs] (NULL if Fs = 0) of the bf16
+ * weights, rounded to nearest even (exact for 2^-14 <= |w| <= 65504; smaller
+ * values become fp16 subnormals, absolute error <= 2^-25).  A weight beyond
+ * the fp16 range sets MOE_ERR_DEVICE_BOUNDS in the status word of ws (which
+ * needs only moe_workspace_size's first 256 bytes here).  Pass the copies in
+ * moe_weights_t together with MOE_FLAG_DOWN_F16. */
+moe_status moe_prepare_down_f16(const moe_dims_t *dims, const void *w_down, const void *ws_down,
+                                void *w_down_f16, void *ws_down_f16, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* Byte offset of the fp32 router logits [T, E] inside the workspace (written
+ * when MOE_FLAG_WRITE_LOGITS is set, and by the CUDA-core router). */
+size_t moe_logits_offset(const moe_dims_t *dims);
 
 /* Synchronises `stream`, then returns the device-side status word of `ws`
  * (MOE_OK if no kernel reported an error) and, if site != NULL, the id of the

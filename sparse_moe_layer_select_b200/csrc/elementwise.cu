@@ -3,15 +3,18 @@
 //   gather_rows_kernel  x_perm[r, :] = x[perm[r] / k, :]   (materialised expert-order
 //                       activations; the forward pass fuses this gather into the GEMM
 //                       operand load instead)
-//   combine_kernel      y[t, :] = bf16( sum_j slot[t, j, :] ) over the k routed slots
-//                       (already scaled by routed_scaling_factor * w_t,j) and the
-//                       shared-expert slot: the combine of the routed sum with the
-//                       always-on shared expert (Laguna M.1/XS.2 Technical Report
+//   combine_kernel      y[t, :] = bf16( sum_j slot[t, j, :] ) in fp32 over the k routed
+//                       fp16 slots (already scaled by routed_scaling_factor * w_t,j)
+//                       and the shared-expert slot: the combine of the routed sum with
+//                       the always-on shared expert (Laguna M.1/XS.2 Technical Report
 //                       summary, Key claims, report §3.1)
+//   bf16_to_f16_kernel  fp16 copy of the down-projection weights (round to nearest
+//                       even; values beyond the fp16 range are reported)
 //   selftest_wait_kernel  a bounded wait on a flag nothing sets (timeout self-test)
 //
 // All three move 16-byte vectors with one thread per vector, grid-stride.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "status.cuh"
@@ -48,8 +51,9 @@ __global__ void __launch_bounds__(256)
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        acc[2 * q] += __uint_as_float(w[q] << 16);
-        acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[q]));
+        acc[2 * q] += f.x;
+        acc[2 * q + 1] += f.y;
       }
     }
     uint32_t o[4];
@@ -60,6 +64,28 @@ __global__ void __launch_bounds__(256)
     }
     y[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
+}
+
+__global__ void __launch_bounds__(256)
+    bf16_to_f16_kernel(const uint4 *__restrict__ src, size_t n_vec, uint4 *__restrict__ dst,
+                       int *status) {
+  bool over = false;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = __uint_as_float(w[q] << 16);
+      const float b = __uint_as_float(w[q] & 0xFFFF0000u);
+      over |= fabsf(a) > 65504.f || fabsf(b) > 65504.f;
+      __half2 h = __floats2half2_rn(a, b);
+      o[q] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (over) record_status(status, MOE_ERR_DEVICE_BOUNDS, SITE_WEIGHT_FP16_RANGE);
 }
 
 __global__ void selftest_wait_kernel(int *status, long long limit_cycles) {
@@ -78,9 +104,14 @@ __global__ void selftest_wait_kernel(int *status, long long limit_cycles) {
 }
 
 int grid_for(size_t work, int threads) {
-  int dev = 0, sms = 148;
+  static int cached[64] = {0};
+  int dev = 0;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int sms = (dev >= 0 && dev < 64) ? cached[dev] : 0;
+  if (sms == 0) {
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (dev >= 0 && dev < 64) cached[dev] = sms;
+  }
   const size_t want = (work + threads - 1) / threads;
   const size_t cap = static_cast<size_t>(sms) * 8;
   return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
@@ -104,6 +135,15 @@ cudaError_t launch_combine(const uint16_t *slots, int T, int nslots, int d, uint
   const size_t work = static_cast<size_t>(T) * vpr;
   combine_kernel<<<grid_for(work, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(slots), T,
                                                      nslots, vpr, reinterpret_cast<uint4 *>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int *status,
+                               cudaStream_t s) {
+  const size_t n_vec = n / 8;  // n is a multiple of 64 (d and F are)
+  bf16_to_f16_kernel<<<grid_for(n_vec, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(src),
+                                                          n_vec, reinterpret_cast<uint4 *>(dst),
+                                                          status);
   return cudaGetLastError();
 }
 

@@ -45,9 +45,10 @@ struct GemmParams {
   const float *bias;        // ROUTER (may be null)
   int *topk_idx;            // ROUTER out
   float *topk_w_out;        // ROUTER out
-  uint16_t *h;              // GEMM1 out: [T*k, F] bf16 (expert-order rows)
-  uint16_t *h_shared;       // GEMM1 out: [T, Fs] bf16
-  uint16_t *slot_out;       // GEMM2 out: [T, slots, d] bf16
+  float *logits_out;        // ROUTER out (optional): [T, E] fp32 logits incl. bias
+  uint16_t *h;              // GEMM1 out: [T*k, F] fp16 (expert-order rows)
+  uint16_t *h_shared;       // GEMM1 out: [T, Fs] fp16
+  uint16_t *slot_out;       // GEMM2 out: [T, slots, d] fp16
 };
 
 struct GemmMaps {
@@ -70,6 +71,8 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_row
                                uint16_t *x_perm, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *slots, int T, int nslots, int d, uint16_t *y,
                            cudaStream_t s);
+cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int *status,
+                               cudaStream_t s);
 cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s);
 
 }  // namespace moe

@@ -33,7 +33,7 @@ struct EventMarker {
   bool on;
   explicit EventMarker(cudaStream_t st) : s(st), on(g_prof_events != nullptr) {}
   void mark() {
-    if (on && next < g_prof_n)
+    if (on && next < g_prof_n && g_prof_events[next] != nullptr)
       cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[next]), s);
     ++next;
   }
@@ -71,13 +71,14 @@ cudaError_t device_setup(int *sms) {
   return cudaSuccess;
 }
 
-// 2-D bf16 tensor [rows, cols] (row-major), 128-byte swizzle, box 64 x box_rows.
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D 16-bit tensor [rows, cols] (row-major), 128-byte swizzle, box 64 x box_rows.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(kBlockK), box_rows};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+  CUresult r = g_encode(m, dtype, 2, const_cast<void *>(ptr), dims,
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -92,7 +93,7 @@ struct Dims {
 };
 
 struct WsLayout {
-  size_t header, chunk_hist, tiles, logits, h, h_sh, slots, total;
+  size_t header, chunk_hist, tiles, logits, h, h_sh, slots, down16, down16_sh, total;
   int max_tiles;
 };
 
@@ -116,6 +117,12 @@ WsLayout ws_layout(const Dims &D) {
   off += align256(static_cast<size_t>(D.T) * D.Fs * 2);
   L.slots = off;
   off += align256(static_cast<size_t>(D.T) * D.slots * D.d * 2);
+  L.down16 = L.down16_sh = off;
+  if (!(D.flags & MOE_FLAG_DOWN_F16)) {  // per-call fp16 copy of the down projections
+    off += align256(static_cast<size_t>(D.E) * D.d * D.F * 2);
+    L.down16_sh = off;
+    off += align256(static_cast<size_t>(D.d) * D.Fs * 2);
+  }
   L.total = off;
   return L;
 }
@@ -184,6 +191,7 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     p.bias = bias;
     p.topk_idx = topk_idx;
     p.topk_w_out = topk_w;
+    if (D.flags & MOE_FLAG_WRITE_LOGITS) p.logits_out = reinterpret_cast<float *>(wsp(ws, L.logits));
     const uint32_t a_rows = static_cast<uint32_t>(std::min(D.T, kBlockM));
     p.a_bytes = a_rows * kBlockK * 2;
     GemmMaps m;
@@ -299,6 +307,10 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   if (w->router_bias && !aligned16(w->router_bias)) return MOE_ERR_INVALID_ARG;
   if (D.Fs > 0 && (!aligned16(w->ws_gate) || !aligned16(w->ws_up) || !aligned16(w->ws_down)))
     return MOE_ERR_INVALID_ARG;
+  if (D.flags & MOE_FLAG_DOWN_F16) {
+    if (!w->w_down_f16 || !aligned16(w->w_down_f16)) return MOE_ERR_INVALID_ARG;
+    if (D.Fs > 0 && (!w->ws_down_f16 || !aligned16(w->ws_down_f16))) return MOE_ERR_INVALID_ARG;
+  }
   if ((st = check_ws(D, ws, ws_bytes)) != MOE_OK) return st;
   g_last_launches = 0;
   if (D.T == 0) return MOE_OK;
@@ -327,6 +339,26 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
                    reinterpret_cast<int *>(wsp(ws, L.chunk_hist)), tiles, header, routing->counts,
                    routing->offsets, routing->perm, s, &launches) != cudaSuccess)
     return MOE_ERR_CUDA;
+
+  // fp16 down projections: caller-prepared, or converted here every call
+  const void *wd16 = w->w_down_f16;
+  const void *wsd16 = w->ws_down_f16;
+  if (!(D.flags & MOE_FLAG_DOWN_F16)) {
+    uint16_t *dst = reinterpret_cast<uint16_t *>(wsp(ws, L.down16));
+    if (launch_bf16_to_f16(static_cast<const uint16_t *>(w->w_down),
+                           static_cast<size_t>(D.E) * D.d * D.F, dst, header, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    wd16 = dst;
+    launches += 1;
+    if (D.Fs > 0) {
+      uint16_t *dsh = reinterpret_cast<uint16_t *>(wsp(ws, L.down16_sh));
+      if (launch_bf16_to_f16(static_cast<const uint16_t *>(w->ws_down),
+                             static_cast<size_t>(D.d) * D.Fs, dsh, header, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      wsd16 = dsh;
+      launches += 1;
+    }
+  }
 
   const int n_rows = D.T * D.k;
   const int n_half = (D.F % 128 == 0 && D.Fs % 128 == 0) ? 128 : 64;
@@ -389,12 +421,14 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     p.a_sh_bytes = a_sh_rows * kBlockK * 2;
     GemmMaps m;
     std::memset(&m, 0, sizeof(m));
-    if (!make_map(&m.a, h, n_rows, D.F, a_rows)) return MOE_ERR_CUDA;
-    if (!make_map(&m.b0, w->w_down, static_cast<uint64_t>(D.E) * D.d, D.F, n2)) return MOE_ERR_CUDA;
+    const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&m.a, h, n_rows, D.F, a_rows, f16)) return MOE_ERR_CUDA;
+    if (!make_map(&m.b0, wd16, static_cast<uint64_t>(D.E) * D.d, D.F, n2, f16))
+      return MOE_ERR_CUDA;
     m.b1 = m.b0;
     if (D.Fs > 0) {
-      if (!make_map(&m.a_sh, h_sh, D.T, D.Fs, a_sh_rows)) return MOE_ERR_CUDA;
-      if (!make_map(&m.b0_sh, w->ws_down, D.d, D.Fs, n2)) return MOE_ERR_CUDA;
+      if (!make_map(&m.a_sh, h_sh, D.T, D.Fs, a_sh_rows, f16)) return MOE_ERR_CUDA;
+      if (!make_map(&m.b0_sh, wsd16, D.d, D.Fs, n2, f16)) return MOE_ERR_CUDA;
     } else {
       m.a_sh = m.a;
       m.b0_sh = m.b0;
@@ -413,6 +447,44 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   ev.mark();
   g_last_launches = launches;
   return MOE_OK;
+}
+
+moe_status moe_prepare_down_f16(const moe_dims_t *dims, const void *w_down, const void *ws_down,
+                                void *w_down_f16, void *ws_down_f16, void *ws, size_t ws_bytes,
+                                void *stream) {
+  Dims D;
+  moe_status st = check_dims(dims, &D);
+  if (st != MOE_OK) return st;
+  if (!w_down || !w_down_f16 || !aligned16(w_down) || !aligned16(w_down_f16))
+    return MOE_ERR_INVALID_ARG;
+  if (D.Fs > 0 && (!ws_down || !ws_down_f16 || !aligned16(ws_down) || !aligned16(ws_down_f16)))
+    return MOE_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  if (device_setup(&sms) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_header(ws, s)) != MOE_OK) return st;
+  int *status = static_cast<int *>(ws);
+  int launches = 0;
+  if (launch_bf16_to_f16(static_cast<const uint16_t *>(w_down), static_cast<size_t>(D.E) * D.d * D.F,
+                         static_cast<uint16_t *>(w_down_f16), status, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  ++launches;
+  if (D.Fs > 0) {
+    if (launch_bf16_to_f16(static_cast<const uint16_t *>(ws_down), static_cast<size_t>(D.d) * D.Fs,
+                           static_cast<uint16_t *>(ws_down_f16), status, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    ++launches;
+  }
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+size_t moe_logits_offset(const moe_dims_t *dims) {
+  Dims D;
+  if (check_dims(dims, &D) != MOE_OK) return 0;
+  return ws_layout(D).logits;
 }
 
 moe_status moe_read_device_status(const void *ws, void *stream, int32_t *site) {

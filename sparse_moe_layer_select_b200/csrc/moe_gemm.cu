@@ -12,13 +12,14 @@
 //                TMA (tile::gather4) through the expert-order permutation, so
 //                the permuted activations are never written out.  The
 //                epilogue applies SwiGLU, h = silu(gate) * up, and stores h in
-//                bf16 (Laguna-M.1-base spec sheet, Feed-forward: SwiGLU, no bias).
-//   MODE_GEMM2   o = h . W_down^T for one expert and one d-column block; the
+//                fp16 (Laguna-M.1-base spec sheet, Feed-forward: SwiGLU, no bias).
+//   MODE_GEMM2   o = h . W_down^T (fp16 operands, fp32 accumulation) for one
+//                expert and one d-column block; the
 //                epilogue multiplies each row by routed_scaling_factor * w
 //                (the 2.5 modulation of the routed sum: Technical Report
-//                summary, report §3.1) and writes it to that (token, slot)'s
-//                row of the slot buffer; shared-expert rows go to the last
-//                slot with scale 1.
+//                summary, report §3.1) and writes it, in fp16, to that
+//                (token, slot)'s row of the slot buffer; shared-expert rows go
+//                to the last slot with scale 1.
 //
 // Roles inside a CTA (192 threads, one CTA per SM, persistent over items):
 //   warp 0      TMA producer: fills a kStages-deep ring of (A, B) stages.
@@ -31,6 +32,7 @@
 // Every wait is bounded (status.cuh); on expiry the kernel records
 // MOE_ERR_DEVICE_TIMEOUT, drains what it issued, frees TMEM and returns.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cfloat>
 
@@ -58,10 +60,12 @@ struct SmemLayout {
   static constexpr int total = bias_off + 512 * 4;
 };
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
 }
+
+constexpr float kF16Max = 65504.f;
 
 // Per-item description shared by all roles.
 struct Item {
@@ -131,6 +135,7 @@ __device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item 
     bv[q] = -FLT_MAX;
     bi[q] = 0x7fffffff;
   }
+  const bool valid = row_local < it.nrows;
   for (int c = 0; c < p.E; c += 32) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(taddr + c, r);
@@ -140,8 +145,14 @@ __device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item 
       const float v = __uint_as_float(r[i]) + bias_s[c + i];
       if (c + i < p.E && v > bv[KM - 1]) topk_insert<KM>(bv, bi, v, c + i);
     }
+    if (p.logits_out != nullptr && valid) {
+      float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E + c;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (c + i < p.E) dst[i] = __uint_as_float(r[i]) + bias_s[c + i];
+    }
   }
-  if (row_local < it.nrows) {
+  if (valid) {
     const size_t t = static_cast<size_t>(it.row0 + row_local);
     float s[KM];
     float sum = 0.f;
@@ -173,14 +184,17 @@ __device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item 
     tmem_ld_32x32b_x32(taddr + p.n_half + c, u);
     tmem_ld_wait();
     uint32_t packed[16];
+    float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
       const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
       const float h0 = g0 / (1.f + __expf(-g0)) * u0;
       const float h1 = g1 / (1.f + __expf(-g1)) * u1;
-      packed[i] = pack_bf16x2(h0, h1);
+      amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
+      packed[i] = pack_f16x2(h0, h1);
     }
+    if (valid && amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_H_FP16_RANGE);
     if (valid) {
       uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
 #pragma unroll
@@ -215,10 +229,15 @@ __device__ __forceinline__ void slot_epilogue(const GemmParams &p, const Item &i
     tmem_ld_wait();
     if (valid) {
       uint32_t packed[16];
+      float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * scale,
-                                __uint_as_float(r[2 * i + 1]) * scale);
+      for (int i = 0; i < 16; ++i) {
+        const float v0 = __uint_as_float(r[2 * i]) * scale;
+        const float v1 = __uint_as_float(r[2 * i + 1]) * scale;
+        amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));
+        packed[i] = pack_f16x2(v0, v1);
+      }
+      if (amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_SLOT_FP16_RANGE);
       uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
 #pragma unroll
       for (int v = 0; v < 4; ++v)
@@ -285,7 +304,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int n_items = (MODE == MODE_ROUTER) ? p.n_tiles_host : (*p.n_tiles_dev) * p.n_ntiles;
-  const uint32_t idesc = idesc_bf16_f32(kBlockM, p.n_tile);
+  // The down projection multiplies fp16 h by fp16 W_down; the others are bf16.
+  const uint32_t idesc =
+      MODE == MODE_GEMM2 ? idesc_f16_f32(kBlockM, p.n_tile) : idesc_bf16_f32(kBlockM, p.n_tile);
   int *status = p.status;
 
   if (warp == 0) {
@@ -393,7 +414,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b0 = smem_u32(sB + s * kBBytesMax);
 #pragma unroll
           for (int kk = 0; kk < kBlockK / 16; ++kk) {
-            umma_bf16_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+            umma_f16_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
                          idesc, (kb | kk) != 0);
           }
           umma_commit(&empty[s]);

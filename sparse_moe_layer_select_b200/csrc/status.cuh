@@ -18,6 +18,9 @@ enum Site : int {
   SITE_GEMM_EPI_ACC_FULL = 13,
   SITE_GEMM_DRAIN = 14,
   SITE_PERMUTE_EXPERT_ID = 20,
+  SITE_H_FP16_RANGE = 30,        // SwiGLU activation beyond the fp16 range
+  SITE_SLOT_FP16_RANGE = 31,     // scaled expert contribution beyond the fp16 range
+  SITE_WEIGHT_FP16_RANGE = 32,   // down-projection weight beyond the fp16 range
   SITE_SELFTEST_FLAG = 90,
 };
 

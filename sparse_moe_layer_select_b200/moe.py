@@ -23,11 +23,14 @@ MOE_ERR_DEVICE_BOUNDS = 6
 
 MOE_FLAG_ROUTER_CUDA_CORE = 1
 MOE_FLAG_ROUTER_TENSOR = 2
+MOE_FLAG_DOWN_F16 = 4
+MOE_FLAG_WRITE_LOGITS = 8
 
 # Every symbol the header declares (checked by the CPU tests).
 EXPORTED = ["moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
             "moe_read_device_status", "moe_selftest_bounded_wait", "moe_status_string",
-            "moe_last_launch_count", "moe_profile_next_forward"]
+            "moe_last_launch_count", "moe_profile_next_forward", "moe_prepare_down_f16",
+            "moe_logits_offset"]
 
 
 class MoeError(RuntimeError):
@@ -49,7 +52,8 @@ class moe_weights_t(ctypes.Structure):
     _fields_ = [("w_router", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
                 ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
                 ("w_down", ctypes.c_void_p), ("ws_gate", ctypes.c_void_p),
-                ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p)]
+                ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p),
+                ("w_down_f16", ctypes.c_void_p), ("ws_down_f16", ctypes.c_void_p)]
 
 
 class moe_routing_t(ctypes.Structure):
@@ -88,6 +92,10 @@ def lib():
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_last_launch_count.restype = ctypes.c_int32
         L.moe_last_launch_count.argtypes = []
+        L.moe_prepare_down_f16.restype = ctypes.c_int
+        L.moe_prepare_down_f16.argtypes = [D, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_logits_offset.restype = ctypes.c_size_t
+        L.moe_logits_offset.argtypes = [D]
         L.moe_profile_next_forward.restype = ctypes.c_int
         L.moe_profile_next_forward.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
         _LIB = L
@@ -152,7 +160,26 @@ def permute(dims, topk_idx, counts, offsets, perm, ws, x=None, x_perm=None, stre
 def weights_struct(W):
     return moe_weights_t(*[None if W.get(k) is None else W[k].data_ptr() for k in
                            ("w_router", "router_bias", "w_gate", "w_up", "w_down", "ws_gate",
-                            "ws_up", "ws_down")])
+                            "ws_up", "ws_down", "w_down_f16", "ws_down_f16")])
+
+
+def prepare_down_f16(dims, W, stream=None):
+    """fp16 copies of the down projections (moe_prepare_down_f16); adds them to W and
+    returns the device status of the conversion."""
+    import torch
+    W["w_down_f16"] = torch.empty(W["w_down"].shape, dtype=torch.float16, device=W["w_down"].device)
+    if W.get("ws_down") is not None:
+        W["ws_down_f16"] = torch.empty(W["ws_down"].shape, dtype=torch.float16,
+                                       device=W["ws_down"].device)
+    hdr = torch.zeros(256, dtype=torch.uint8, device=W["w_down"].device)
+    _check(lib().moe_prepare_down_f16(ctypes.byref(dims), _p(W["w_down"]), _p(W.get("ws_down")),
+                                      _p(W["w_down_f16"]), _p(W.get("ws_down_f16")), _p(hdr), 256,
+                                      _stream(stream)), "moe_prepare_down_f16")
+    return read_device_status(hdr, stream)
+
+
+def logits_offset(dims) -> int:
+    return int(lib().moe_logits_offset(ctypes.byref(dims)))
 
 
 def routing_struct(R):
@@ -195,6 +222,12 @@ def profile_next_forward(events):
     if events is None:
         _check(lib().moe_profile_next_forward(None, 0), "moe_profile_next_forward")
         return
+    import torch
+    for e in events:  # torch creates the CUDA event handle on first record
+        if e.cuda_event == 0:
+            e.record(torch.cuda.current_stream())
+    if any(e.cuda_event == 0 for e in events):
+        raise RuntimeError("profile_next_forward: CUDA events were not created")
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     profile_next_forward._keep = arr
     _check(lib().moe_profile_next_forward(arr, len(events)), "moe_profile_next_forward")
@@ -213,15 +246,20 @@ class MoeLayer:
 
     def __init__(self, weights: dict, d_model, num_experts, num_experts_per_tok,
                  moe_intermediate_size, shared_intermediate_size, routed_scaling_factor=2.5,
-                 max_tokens=1, flags=0, device="cuda"):
-        self.W = weights
+                 max_tokens=1, flags=0, device="cuda", prepare=True):
+        self.W = dict(weights)
         self.cfg = dict(d_model=d_model, num_experts=num_experts,
                         num_experts_per_tok=num_experts_per_tok,
                         moe_intermediate_size=moe_intermediate_size,
                         shared_intermediate_size=shared_intermediate_size,
                         routed_scaling_factor=routed_scaling_factor, flags=flags)
         self.device = device
-        self._ws_struct = weights_struct(weights)
+        if prepare:  # one-time fp16 copy of the down projections (model-load step)
+            self.cfg["flags"] |= MOE_FLAG_DOWN_F16
+            code, site = prepare_down_f16(self.dims(1), self.W)
+            if code != MOE_OK:
+                raise MoeError(code, f"moe_prepare_down_f16 (site {site})")
+        self._ws_struct = weights_struct(self.W)
         self._reserve(max_tokens)
 
     def dims(self, T):

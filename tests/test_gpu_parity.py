@@ -169,7 +169,9 @@ def test_small_expert_counts_and_k_extremes(E, k):
     G.check_output(G.y_numpy(y), ref["y"], what=f"E={E},k={k}")
 
 
-def test_exact_ties_go_to_lower_expert_index():
+@pytest.mark.parametrize("flags", [M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR])
+def test_exact_ties_go_to_lower_expert_index(flags):
+    import torch
     w = I.get("c1_tiny").with_(T=256)
     h, _ = _small(w)
     wr = h["w_router"].copy()
@@ -177,15 +179,67 @@ def test_exact_ties_go_to_lower_expert_index():
     wr[14] = wr[5]
     h["w_router"] = wr
     dev = G.host_to_device(h)
-    for flags in (M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR):
-        y, routing, _ = G.run_forward(w, dev, flags=flags)
-        idx = routing["topk_idx"].cpu().numpy()
-        ref = G.oracle_forward(w, h)
-        for t in range(w.T):
-            s = set(idx[t].tolist())
-            assert not (9 in s and 2 not in s) and not (14 in s and 5 not in s), (t, idx[t])
-        G.check_routing(idx, routing["topk_w"].cpu().numpy(), ref, w.k)
-        G.check_output(G.y_numpy(y), ref["y"], what="ties")
+    y, routing, ws = G.run_forward(w, dev, flags=flags | M.MOE_FLAG_WRITE_LOGITS)
+    off = M.logits_offset(M.dims_for(w, flags=flags | M.MOE_FLAG_WRITE_LOGITS))
+    logits = ws[off:off + w.T * w.E * 4].view(torch.float32).view(w.T, w.E).cpu().numpy()
+    assert np.array_equal(logits[:, 2], logits[:, 9]) and np.array_equal(logits[:, 5], logits[:, 14])
+    idx = routing["topk_idx"].cpu().numpy()
+    ref = G.oracle_forward(w, h)
+    for t in range(w.T):
+        s_ = set(idx[t].tolist())
+        assert not (9 in s_ and 2 not in s_) and not (14 in s_ and 5 not in s_), (t, idx[t])
+    G.check_routing(idx, routing["topk_w"].cpu().numpy(), ref, w.k)
+    G.check_output(G.y_numpy(y), ref["y"], what="ties")
+
+
+@pytest.mark.parametrize("flags", [M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR])
+def test_router_logits_error_against_float64(flags):
+    """fp32 logits of both router paths against the oracle's float64 logits (XS.2 widths)."""
+    import torch
+    w = I.get("c2_xs2_small").with_(T=2048)
+    dev = {"x": torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda"),
+           "w_router": torch.empty((w.E, w.d_model), dtype=torch.bfloat16, device="cuda")}
+    I.generate_cuda(dev["x"], w.seed, I.TID_X, w.sigma_x)
+    I.generate_cuda(dev["w_router"], w.seed, I.TID_W_ROUTER, w.sigma_router)
+    dims = M.dims_for(w, flags=flags | M.MOE_FLAG_WRITE_LOGITS)
+    ws = M.alloc_workspace(dims)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((w.T, w.k), dtype=torch.float32, device="cuda")
+    M.route(dims, dev["x"], dev["w_router"], None, idx, wt, ws)
+    torch.cuda.synchronize()
+    off = M.logits_offset(dims)
+    got = ws[off:off + w.T * w.E * 4].view(torch.float32).view(w.T, w.E).cpu().numpy()
+    ref = O.router_logits(P.to_numpy_bf16(dev["x"]), P.to_numpy_bf16(dev["w_router"]), None)
+    err = float(np.abs(got - ref).max())
+    # a logit error below 4e-6 is a score error below 1e-6 (the sigmoid's slope is <= 1/4),
+    # so any selection it flips lies inside the near-tie exemption band
+    assert err < 4e-6, err
+
+
+def test_prepared_down_weights_match_per_call_conversion():
+    import torch
+    w = I.get("c1_tiny").with_(T=500)
+    h, dev = _small(w)
+    y1, _, _ = G.run_forward(w, dev)                      # converts W_down every call
+    layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
+                       max_tokens=w.T)                    # prepared once
+    y2 = layer.forward(dev["x"])
+    torch.cuda.synchronize()
+    assert np.array_equal(P.to_numpy_bf16(y1), P.to_numpy_bf16(y2))
+    wd = h["w_down"].astype(np.uint32) << 16
+    ref16 = wd.view(np.float32).astype(np.float16)
+    assert np.array_equal(layer.W["w_down_f16"].cpu().numpy(), ref16)
+
+
+def test_fp16_range_violation_is_reported():
+    import torch
+    w = I.get("c1_tiny")
+    h, dev = _small(w)
+    bad = dev["w_down"].clone()
+    bad[3, 5, 7] = 1.0e6
+    W = {"w_down": bad, "ws_down": dev["ws_down"]}
+    code, site = M.prepare_down_f16(M.dims_for(w), W)
+    assert code == M.MOE_ERR_DEVICE_BOUNDS and site == 32
 
 
 def test_maximum_skew_all_tokens_on_the_same_experts():
