@@ -80,14 +80,23 @@ class ClockSampler:
         self.proc = None
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+             "utilization.gpu")
         try:
             self.f = open(path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+
+    def wait_first_sample(self, timeout=3.0):
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < timeout:
+            self.f.flush()
+            if os.path.getsize(self.path) > 0:
+                return
+            time.sleep(0.05)
 
     def stop(self):
         if self.proc is None:
@@ -103,20 +112,25 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
+                    util = float(parts[9])
+                    clk = float(parts[1])
                     mx = float(parts[2])
                 except ValueError:
                     continue
+                if util < 50:  # idle samples say nothing about the clock under load
+                    continue
+                sm.append(clk)
                 for n, v in zip(names, parts[5:9]):
                     if v.lower().startswith("active"):
                         reasons.add(n)
         if not sm:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window": "warm-up start to end of timed region, "
+                                              "samples with utilization >= 50%"}
 
 
 # ----------------------------------------------------------------- CPU baseline
@@ -190,8 +204,18 @@ def run_ours(args):
             M.profile_next_forward(events)
         layer.forward(x_buf, y)
 
-    for i in range(args.warmup):
+    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                          if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
+                          else f"/tmp/clocks_rank{rank}.csv")
+    clocks.wait_first_sample()
+    # warm-up: at least W steps and at least 0.3 s, so clocks settle under load
+    t_w = time.time()
+    i = 0
+    while i < args.warmup or time.time() - t_w < 0.3:
         step(i)
+        i += 1
+        if i % 16 == 0:
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
     code, site = M.read_device_status(layer.ws)
     if code != 0:
@@ -200,9 +224,6 @@ def run_ours(args):
 
     n_st = len(M.FORWARD_STAGES)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)] for _ in range(args.steps)]
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                          if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
-                          else f"/tmp/clocks_rank{rank}.csv")
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

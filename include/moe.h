@@ -81,9 +81,6 @@ typedef struct {
  * ws_down_f16, made once by moe_prepare_down_f16); without this flag
  * moe_forward converts them into the workspace on every call. */
 #define MOE_FLAG_DOWN_F16         4
-/* Both router paths also write the fp32 logits (bias included) to the
- * workspace, at the byte offset returned by moe_logits_offset. */
-#define MOE_FLAG_WRITE_LOGITS     8
 
 typedef struct {
     const void *w_router;      /* [E, d] bf16 */
@@ -114,8 +111,10 @@ size_t moe_workspace_size(const moe_dims_t *dims);
 /* Router: sigmoid scores, top-k with ties to the lower expert index, and
  * post-top-k normalisation (Laguna M.1/XS.2 Technical Report summary, Key
  * claims, report §3.1; Laguna-M.1-base spec sheet, Mixture of experts:
- * "Router score", "Renormalize top-k").  Selection is made on fp32 logits
- * (equivalent to selection on the scores, since the sigmoid is increasing).
+ * "Router score", "Renormalize top-k").  Selection is made on the logits
+ * (equivalent to selection on the scores, since the sigmoid is increasing):
+ * fp32 logits, and for tokens whose k-th and (k+1)-th logits are closer than
+ * 2e-4, float64 logits for the experts at that boundary.
  * x: [T, d] bf16.  router_bias may be NULL.  Outputs topk_idx [T, k] int32 and
  * topk_w [T, k] fp32, both in descending-score order. */
 moe_status moe_route(const moe_dims_t *dims, const void *x, const void *w_router,
@@ -159,8 +158,8 @@ moe_status moe_prepare_down_f16(const moe_dims_t *dims, const void *w_down, cons
                                 void *w_down_f16, void *ws_down_f16, void *ws, size_t ws_bytes,
                                 void *stream);
 
-/* Byte offset of the fp32 router logits [T, E] inside the workspace (written
- * when MOE_FLAG_WRITE_LOGITS is set, and by the CUDA-core router). */
+/* Byte offset of the fp32 router logits [T, E] (bias included) that
+ * moe_route and moe_forward leave in the workspace. */
 size_t moe_logits_offset(const moe_dims_t *dims);
 
 /* Synchronises `stream`, then returns the device-side status word of `ws`

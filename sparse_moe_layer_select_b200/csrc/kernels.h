@@ -39,13 +39,11 @@ struct GemmParams {
   uint32_t a_bytes;         // bytes of one A stage (ROUTER, GEMM2 routed rows)
   uint32_t a_sh_bytes;      // bytes of one A stage for shared-expert rows (GEMM2)
   float routed_scale;       // GEMM2: routed_scaling_factor
-  int norm_topk;            // ROUTER
+  const uint16_t *x;        // GEMM1: token rows [T, d] bf16 (gathered by cp.async)
   const int *perm;          // GEMM1/GEMM2: expert-order rows -> t * k + j
   const float *topk_w;      // GEMM2
   const float *bias;        // ROUTER (may be null)
-  int *topk_idx;            // ROUTER out
-  float *topk_w_out;        // ROUTER out
-  float *logits_out;        // ROUTER out (optional): [T, E] fp32 logits incl. bias
+  float *logits_out;        // ROUTER out: [T, E] fp32 logits incl. bias
   uint16_t *h;              // GEMM1 out: [T*k, F] fp16 (expert-order rows)
   uint16_t *h_shared;       // GEMM1 out: [T, Fs] fp16
   uint16_t *slot_out;       // GEMM2 out: [T, slots, d] fp16
@@ -61,8 +59,9 @@ cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int gr
 
 cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
                              float *logits, int T, int d, int E, cudaStream_t s);
-cudaError_t launch_topk_from_logits(const float *logits, int T, int E, int k, int norm_topk,
-                                    int32_t *topk_idx, float *topk_w, cudaStream_t s);
+cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
+                                 const float *bias, int T, int d, int E, int k, int norm_topk,
+                                 int32_t *topk_idx, float *topk_w, cudaStream_t s);
 
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,

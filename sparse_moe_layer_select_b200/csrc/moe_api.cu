@@ -26,15 +26,20 @@ thread_local int32_t g_last_launches = 0;
 thread_local void **g_prof_events = nullptr;
 thread_local int32_t g_prof_n = 0;
 
-// Records the next armed profiling event (if any) on stream s.
+// Records the next armed profiling event (if any) on stream s.  Takes over
+// the armed event list, so only one call records into it.
 struct EventMarker {
   cudaStream_t s;
+  void **events;
+  int n;
   int next = 0;
-  bool on;
-  explicit EventMarker(cudaStream_t st) : s(st), on(g_prof_events != nullptr) {}
+  explicit EventMarker(cudaStream_t st) : s(st), events(g_prof_events), n(g_prof_n) {
+    g_prof_events = nullptr;
+    g_prof_n = 0;
+  }
   void mark() {
-    if (on && next < g_prof_n && g_prof_events[next] != nullptr)
-      cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[next]), s);
+    if (events != nullptr && next < n && events[next] != nullptr)
+      cudaEventRecord(static_cast<cudaEvent_t>(events[next]), s);
     ++next;
   }
 };
@@ -170,10 +175,13 @@ bool use_tensor_router(const Dims &D) {
   return fits && D.T >= 1024;
 }
 
+// Router: fp32 logits (tcgen05 GEMM or CUDA-core FMA) into the workspace,
+// then the warp-per-token selection kernel.
 moe_status route_impl(const Dims &D, const void *x, const void *w_router, const float *bias,
                       int32_t *topk_idx, float *topk_w, void *ws, cudaStream_t s, int sms,
                       int *launches) {
   const WsLayout L = ws_layout(D);
+  float *logits = reinterpret_cast<float *>(wsp(ws, L.logits));
   if (use_tensor_router(D)) {
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -187,11 +195,8 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     p.F = D.F;
     p.Fs = D.Fs;
     p.n_tile = D.E;
-    p.norm_topk = D.norm;
     p.bias = bias;
-    p.topk_idx = topk_idx;
-    p.topk_w_out = topk_w;
-    if (D.flags & MOE_FLAG_WRITE_LOGITS) p.logits_out = reinterpret_cast<float *>(wsp(ws, L.logits));
+    p.logits_out = logits;
     const uint32_t a_rows = static_cast<uint32_t>(std::min(D.T, kBlockM));
     p.a_bytes = a_rows * kBlockK * 2;
     GemmMaps m;
@@ -204,14 +209,14 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     m.b1_sh = m.b0;
     const int grid = std::min(sms, p.n_tiles_host);
     if (launch_gemm(MODE_ROUTER, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
-    *launches += 1;
-    return MOE_OK;
+  } else {
+    if (launch_router_cc(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(w_router),
+                         bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
-  float *logits = reinterpret_cast<float *>(wsp(ws, L.logits));
-  if (launch_router_cc(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(w_router),
-                       bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (launch_topk_from_logits(logits, D.T, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
+  if (launch_router_select(logits, static_cast<const uint16_t *>(x),
+                           static_cast<const uint16_t *>(w_router), bias, D.T, D.d, D.E, D.k,
+                           D.norm, topk_idx, topk_w, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   *launches += 2;
   return MOE_OK;
@@ -326,7 +331,6 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   uint16_t *slots = reinterpret_cast<uint16_t *>(wsp(ws, L.slots));
   int launches = 0;
   EventMarker ev(s);
-  g_prof_events = nullptr;  // one call only
 
   // 1. router
   ev.mark();
@@ -377,7 +381,6 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   base.Fs = D.Fs;
   base.slots = D.slots;
   base.routed_scale = D.scale;
-  base.norm_topk = D.norm;
   base.perm = routing->perm;
   base.topk_w = routing->topk_w;
   base.h = h;
@@ -390,6 +393,7 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     p.n_half = n_half;
     p.n_tile = 2 * n_half;
     p.n_ntiles = std::max(D.F, D.Fs) / n_half;
+    p.x = static_cast<const uint16_t *>(x);
     p.a_bytes = kBlockM * kBlockK * 2;
     p.a_sh_bytes = p.a_bytes;
     GemmMaps m;

@@ -2,14 +2,14 @@
 //
 // One kernel template serves the three contractions of the layer:
 //
-//   MODE_ROUTER  logits[128 tokens, E] = x_tile . W_r^T, fp32 in TMEM; the
-//                epilogue keeps each token's top-k in registers and writes the
-//                normalised sigmoid weights (sigmoid router with post-top-k
-//                normalisation: Laguna M.1/XS.2 Technical Report summary, Key
-//                claims, report §3.1).
+//   MODE_ROUTER  logits[128 tokens, E] = x_tile . W_r^T (+ b), fp32 in TMEM,
+//                written out for the warp-per-token selection (sigmoid router
+//                with post-top-k normalisation: Laguna M.1/XS.2 Technical
+//                Report summary, Key claims, report §3.1).
 //   MODE_GEMM1   [gate | up] = X_perm . [W_gate | W_up]^T for one expert and
-//                one column block; the rows of X_perm are gathered from x by
-//                TMA (tile::gather4) through the expert-order permutation, so
+//                one column block; the rows of X_perm are gathered from x
+//                through the expert-order permutation by 16-byte cp.async
+//                copies written straight into the swizzled operand layout, so
 //                the permuted activations are never written out.  The
 //                epilogue applies SwiGLU, h = silu(gate) * up, and stores h in
 //                fp16 (Laguna-M.1-base spec sheet, Feed-forward: SwiGLU, no bias).
@@ -22,7 +22,8 @@
 //                to the last slot with scale 1.
 //
 // Roles inside a CTA (192 threads, one CTA per SM, persistent over items):
-//   warp 0      TMA producer: fills a kStages-deep ring of (A, B) stages.
+//   warp 0      producer: fills a kStages-deep ring of (A, B) stages (TMA
+//               tiles; for GEMM1 the A rows by cp.async from all 32 lanes).
 //   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma
 //               (M=128, N<=256, K=16 per instruction) into one of two
 //               accumulator buffers and commits stage releases.
@@ -107,65 +108,30 @@ __device__ __forceinline__ Item decode_item(const GemmParams &p, int item) {
   return it;
 }
 
-template <int KM>
-__device__ __forceinline__ void topk_insert(float (&bv)[KM], int (&bi)[KM], float v, int i) {
-  // Sorted descending; a candidate displaces only a strictly smaller value,
-  // and candidates arrive in ascending expert order, so equal logits keep
-  // the lower expert index first.
-#pragma unroll
-  for (int q = 0; q < KM; ++q) {
-    if (v > bv[q]) {
-      const float tv = bv[q];
-      const int ti = bi[q];
-      bv[q] = v;
-      bi[q] = i;
-      v = tv;
-      i = ti;
-    }
-  }
-}
-
-template <int KM>
+// Router epilogue: each thread owns one token row and writes its E fp32
+// logits (bias added) as 16-byte vectors; selection happens in the
+// warp-per-token select kernel that follows.
 __device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item &it, uint32_t taddr,
                                                 int row_local, const float *bias_s) {
-  float bv[KM];
-  int bi[KM];
-#pragma unroll
-  for (int q = 0; q < KM; ++q) {
-    bv[q] = -FLT_MAX;
-    bi[q] = 0x7fffffff;
-  }
   const bool valid = row_local < it.nrows;
+  float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E;
   for (int c = 0; c < p.E; c += 32) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(taddr + c, r);
     tmem_ld_wait();
+    if (valid) {
+      if (c + 32 <= p.E) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float v = __uint_as_float(r[i]) + bias_s[c + i];
-      if (c + i < p.E && v > bv[KM - 1]) topk_insert<KM>(bv, bi, v, c + i);
-    }
-    if (p.logits_out != nullptr && valid) {
-      float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E + c;
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4 *>(dst + c + i) =
+              make_float4(__uint_as_float(r[i]) + bias_s[c + i],
+                          __uint_as_float(r[i + 1]) + bias_s[c + i + 1],
+                          __uint_as_float(r[i + 2]) + bias_s[c + i + 2],
+                          __uint_as_float(r[i + 3]) + bias_s[c + i + 3]);
+      } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (c + i < p.E) dst[i] = __uint_as_float(r[i]) + bias_s[c + i];
-    }
-  }
-  if (valid) {
-    const size_t t = static_cast<size_t>(it.row0 + row_local);
-    float s[KM];
-    float sum = 0.f;
-#pragma unroll
-    for (int q = 0; q < KM; ++q) {
-      s[q] = 1.f / (1.f + expf(-bv[q]));
-      if (q < p.k) sum += s[q];
-    }
-#pragma unroll
-    for (int q = 0; q < KM; ++q) {
-      if (q < p.k) {
-        p.topk_idx[t * p.k + q] = bi[q];
-        p.topk_w_out[t * p.k + q] = p.norm_topk ? s[q] / sum : s[q];
+        for (int i = 0; i < 32; ++i)
+          if (c + i < p.E) dst[c + i] = __uint_as_float(r[i]) + bias_s[c + i];
       }
     }
   }
@@ -275,7 +241,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      // GEMM1: one expect_tx arrival for the B tiles plus one cp.async
+      // completion arrival from each lane of the gathering warp.
+      mbar_init(&full[s], MODE == MODE_GEMM1 ? 1 + 32 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -320,21 +288,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (it.skip) continue;
       if (status_is_set(status)) break;
       const bool shared = it.group == p.E;
-      // GEMM1: each lane gathers 4 of the tile's 128 rows (token ids).
-      int tok[4] = {0, 0, 0, 0};
+      // GEMM1: lane l copies 16-byte chunk (l & 7) of rows (l >> 3) + 4 i,
+      // i = 0..31, so one warp instruction moves four whole 128-byte rows.
+      // Rows past the tile's valid count are not loaded (their accumulator
+      // rows are discarded by the epilogue).
+      int tok[32];
       if (MODE == MODE_GEMM1) {
-        int first;
-        if (shared) {
-          first = it.row0;
-        } else {
-          first = p.perm[it.row0] / p.k;
-        }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r = 4 * lane + q;
-          int t = first;
-          if (r < it.nrows) t = shared ? it.row0 + r : p.perm[it.row0 + r] / p.k;
-          tok[q] = t;
+        for (int i = 0; i < 32; ++i) {
+          const int r = (lane >> 3) + 4 * i;
+          tok[i] = -1;
+          if (r < it.nrows) tok[i] = shared ? it.row0 + r : p.perm[it.row0 + r] / p.k;
         }
       }
       // A boxes shorter than 128 rows (tensors with fewer rows) fill only
@@ -342,7 +306,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // epilogue discards.
       uint32_t bytes;
       if (MODE == MODE_ROUTER) bytes = p.a_bytes + p.E * 128;
-      else if (MODE == MODE_GEMM1) bytes = kABytes + 2 * p.n_half * 128;
+      else if (MODE == MODE_GEMM1) bytes = 2 * p.n_half * 128;  // A arrives by cp.async
       else bytes = (shared ? p.a_sh_bytes : p.a_bytes) + p.n_tile * 128;
       for (int kb = 0; kb < it.nk; ++kb) {
         int good = 1;
@@ -359,12 +323,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint8_t *b_dst = sB + s * kBBytesMax;
         const int kc = kb * kBlockK;
         if (MODE == MODE_GEMM1) {
-          tma_gather4(a_dst + lane * 4 * 128, &tm_a, &full[s], kc, tok[0], tok[1], tok[2], tok[3]);
           if (lane == 0) {
             const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
             tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
             tma_load_2d(b_dst + p.n_half * 128, shared ? &tm_b1_sh : &tm_b1, &full[s], kc, brow);
           }
+          // 128-byte swizzle: chunk c of row r sits at chunk (c ^ (r & 7)).
+          const int c = lane & 7;
+          const uint32_t a_base = smem_u32(a_dst);
+          const char *xsrc = reinterpret_cast<const char *>(p.x) + kc * 2 + c * 16;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int r = (lane >> 3) + 4 * i;
+            if (tok[i] >= 0)
+              cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4),
+                          xsrc + static_cast<size_t>(tok[i]) * p.d * 2);
+          }
+          cp_async_arrive_noinc(&full[s]);
         } else if (lane == 0) {
           if (MODE == MODE_ROUTER) {
             tma_load_2d(a_dst, &tm_a, &full[s], kc, it.row0);
@@ -383,6 +358,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     // Drain: every stage this warp filled must have landed before the CTA exits.
+    if (MODE == MODE_GEMM1) cp_async_wait_all();
     if (lane == 0) {
       for (long long n = (issued > kStages ? issued - kStages : 0); n < issued; ++n)
         if (!mbar_wait(&full[n % kStages], static_cast<uint32_t>((n / kStages) & 1), status,
@@ -409,6 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
+          if (MODE == MODE_GEMM1) fence_proxy_async_smem();  // A was written by cp.async
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kABytes);
           const uint32_t b0 = smem_u32(sB + s * kBBytesMax);
@@ -449,9 +426,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccStride;
       if (MODE == MODE_ROUTER) {
-        if (p.k <= 4) router_epilogue<4>(p, it, taddr, row_local, bias_s);
-        else if (p.k <= 8) router_epilogue<8>(p, it, taddr, row_local, bias_s);
-        else router_epilogue<16>(p, it, taddr, row_local, bias_s);
+        router_epilogue(p, it, taddr, row_local, bias_s);
       } else if (MODE == MODE_GEMM1) {
         swiglu_epilogue(p, it, taddr, row_local);
       } else {

@@ -3,7 +3,9 @@
 // core + tensor memory) instructions used by the expert and router GEMMs.
 //
 // Written from the PTX ISA descriptions of these instructions.  No cluster
-// multicast form is used anywhere in this library.
+// multicast form is used anywhere in this library.  (tile::gather4 is kept
+// for reference; the expert GEMM gathers rows with cp.async instead, which
+// moves 512 bytes per warp instruction against 512 bytes per TMA gather4.)
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -93,6 +95,28 @@ __device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, ui
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1),
       "r"(r2), "r"(r3)
       : "memory");
+}
+
+// 16-byte asynchronous global->shared copy (cp.async, L2-only caching).
+__device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");
+}
+
+// Arrive on `bar` once every cp.async issued so far by this thread has landed
+// (no increment of the pending count: the arrival is counted at init).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Orders this thread's view of shared memory written through the generic
+// proxy (cp.async) before its subsequent async-proxy reads (tcgen05.mma).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

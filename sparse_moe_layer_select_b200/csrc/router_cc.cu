@@ -1,5 +1,6 @@
-// router_cc.cu -- CUDA-core router for small token counts and shapes outside
-// the tensor-core router's limits (E not a multiple of 16, or E > 256).
+// router_cc.cu -- CUDA-core router logits (small token counts and shapes
+// outside the tensor-core router's limits) and the selection kernel that
+// both logit paths feed.
 //
 // Sigmoid router with post-top-k normalisation (Laguna M.1/XS.2 Technical
 // Report summary, Key claims, report §3.1; Laguna-M.1-base spec sheet,
@@ -9,10 +10,13 @@
 //                         8 token rows in shared memory; each warp computes
 //                         one expert's logits for those 8 tokens (16-byte
 //                         loads of W_r, fp32 FMA, warp butterfly reduction).
-//   topk_kernel           one warp per token: the E logits sit in registers
-//                         (E/32 per lane); k rounds of a warp arg-max (ties to
-//                         the lower expert index) pick the experts in
-//                         descending order; sigmoid and normalisation in fp32.
+//   router_select_kernel  one warp per token, for both logit paths: the E
+//                         logits sit in registers (E/32 per lane); k+1 rounds
+//                         of a warp arg-max (ties to the lower expert index)
+//                         pick the experts in descending order; tokens whose
+//                         k-th and (k+1)-th logits are within kRefineBand get
+//                         the experts near that boundary re-decided on float64
+//                         logits; sigmoid and normalisation in fp32.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -81,25 +85,93 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
 }
 
 constexpr int kMaxPerLane = 16;  // E <= 512
+constexpr int kSelectWarps = 8;
 
-__global__ void __launch_bounds__(256)
-    topk_kernel(const float *__restrict__ logits, int T, int E, int k, int norm_topk,
-                int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// Width of the ambiguous band around the k-th/(k+1)-th boundary, in logit
+// units.  It is far above twice the largest fp32 logit error of either logit
+// path at these widths (tensor-core accumulation up to 1.2e-5, CUDA-core FMA
+// below 4e-6), so every expert outside the band is on the right side of the
+// boundary, and the band is decided on float64 logits.
+constexpr float kRefineBand = 2e-4f;
+
+// float64 logits of up to four experts e[0..n) for one token: exact bf16
+// products, float64 sums (lane-strided, then a butterfly in fixed order), plus
+// the bias.  The token row is read once per group, all loads of the group
+// are independent, so the group costs about one memory round trip.
+__device__ __forceinline__ void logits_f64_x4(const uint16_t *__restrict__ x,
+                                              const uint16_t *__restrict__ w_router,
+                                              const float *__restrict__ bias, int t,
+                                              const int (&e)[4], int n, int d, int lane,
+                                              double (&out)[4]) {
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * d);
+  const uint4 *wr[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    wr[g] = reinterpret_cast<const uint4 *>(w_router + static_cast<size_t>(g < n ? e[g] : e[0]) * d);
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  const int nvec = d / 8;
+#pragma unroll 4
+  for (int c = lane; c < nvec; c += 32) {
+    float xf[8];
+    bf16x8_to_f32(xr[c], xf);
+    uint4 wv[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) wv[g] = wr[g][c];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float wf[8];
+      bf16x8_to_f32(wv[g], wf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        acc[g] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[g]);
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
+    out[g] = acc[g] + ((bias && g < n) ? static_cast<double>(bias[e[g]]) : 0.0);
+  }
+}
+
+__device__ __forceinline__ void warp_argmax(float &bv, int &be) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+    if (ov > bv || (ov == bv && oe < be)) {
+      bv = ov;
+      be = oe;
+    }
+  }
+}
+
+// One warp per token: register top-(k+1) of the fp32 logits (ties to the lower
+// expert index), float64 refinement of the experts near the boundary when the
+// k-th and (k+1)-th logits are closer than kRefineBand, then sigmoid scores
+// and post-top-k normalisation (Laguna M.1/XS.2 Technical Report summary, Key
+// claims, report §3.1; Laguna-M.1-base spec sheet, Mixture of experts).
+__global__ void __launch_bounds__(kSelectWarps * 32)
+    router_select_kernel(const float *__restrict__ logits, const uint16_t *__restrict__ x,
+                         const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
+                         int T, int d, int E, int k, int norm_topk,
+                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+  const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  const float *row = logits + static_cast<size_t>(warp) * E;
+  if (t >= T) return;
+  const float *row = logits + static_cast<size_t>(t) * E;
+  const float kNaN = __int_as_float(0x7fc00000);  // compares false: never selected
   float v[kMaxPerLane];
 #pragma unroll
   for (int i = 0; i < kMaxPerLane; ++i) {
     const int e = lane + 32 * i;
-    v[i] = e < E ? row[e] : __int_as_float(0x7fc00000);  // NaN: never selected
+    v[i] = e < E ? row[e] : kNaN;
   }
-  float my_s = 0.f;
+  float my_l = 0.f;  // lane j < k keeps the j-th selected logit and expert
   int my_e = 0;
-  float sum = 0.f;
-  for (int j = 0; j < k; ++j) {
-    // lane-local best (lowest index on ties: i ascending means e ascending)
+  float lk = 0.f, lk1 = -INFINITY;
+  const int rounds = k < E ? k + 1 : k;
+  for (int j = 0; j < rounds; ++j) {
     float bv = -INFINITY;
     int be = 0x7fffffff;
 #pragma unroll
@@ -110,30 +182,78 @@ __global__ void __launch_bounds__(256)
         be = e;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    // remove the winner (NaN compares false, so it is never picked again)
+    warp_argmax(bv, be);
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i)
-      if (lane + 32 * i == be) v[i] = __int_as_float(0x7fc00000);
-    const float s = 1.f / (1.f + expf(-bv));
-    sum += s;
-    if (lane == j) {
-      my_s = s;
+      if (lane + 32 * i == be) v[i] = kNaN;
+    if (j < k && lane == j) {
+      my_l = bv;
       my_e = be;
     }
+    if (j == k - 1) lk = bv;
+    if (j == k) lk1 = bv;
   }
+
+  if (k < E && lk - lk1 < kRefineBand) {
+    // Candidates: every expert whose fp32 logit reaches the lower band edge
+    // (the selected ones and the band below the boundary), in ascending id.
+    // Their float64 logits decide the top k among them.
+    const float lo = 0.5f * (lk + lk1) - kRefineBand;
+    double best_l[16];
+    int best_e[16];
+    int nbest = 0;
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int e_lane = lane + 32 * i;
+      const bool cand = e_lane < E && row[e_lane] >= lo;
+      unsigned m = __ballot_sync(0xffffffffu, cand);
+      while (m) {
+        int eg[4] = {0, 0, 0, 0};
+        int ng = 0;
+        while (m && ng < 4) {  // up to four candidates, ascending id
+          eg[ng++] = (__ffs(m) - 1) + 32 * i;
+          m &= m - 1;
+        }
+        double lg[4];
+        logits_f64_x4(x, w_router, bias, t, eg, ng, d, lane, lg);
+        if (lane == 0) {
+          for (int g = 0; g < ng; ++g) {
+            // sorted insert, descending logit, lower id first on ties (ids arrive ascending)
+            const double l = lg[g];
+            int pos = nbest < k ? nbest : k;
+            while (pos > 0 && l > best_l[pos - 1]) --pos;
+            if (pos < k) {
+              const int last = nbest < k ? nbest : k - 1;
+              for (int q = last; q > pos; --q) {
+                best_l[q] = best_l[q - 1];
+                best_e[q] = best_e[q - 1];
+              }
+              best_l[pos] = l;
+              best_e[pos] = eg[g];
+              if (nbest < k) ++nbest;
+            }
+          }
+        }
+      }
+    }
+    // hand the refined list to lanes 0..k-1
+    for (int q = 0; q < k; ++q) {
+      const float lq = __shfl_sync(0xffffffffu, lane == 0 ? static_cast<float>(best_l[q]) : 0.f, 0);
+      const int eq = __shfl_sync(0xffffffffu, lane == 0 ? best_e[q] : 0, 0);
+      if (lane == q) {
+        my_l = lq;
+        my_e = eq;
+      }
+    }
+  }
+
+  const float s = 1.f / (1.f + expf(-my_l));
+  float sum = lane < k ? s : 0.f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
   if (lane < k) {
-    const size_t o = static_cast<size_t>(warp) * k + lane;
+    const size_t o = static_cast<size_t>(t) * k + lane;
     topk_idx[o] = my_e;
-    topk_w[o] = norm_topk ? my_s / sum : my_s;
+    topk_w[o] = norm_topk ? s / sum : s;
   }
 }
 
@@ -157,11 +277,12 @@ cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const 
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk_from_logits(const float *logits, int T, int E, int k, int norm_topk,
-                                    int32_t *topk_idx, float *topk_w, cudaStream_t s) {
-  const int threads = 256;
-  const int blocks = (T * 32 + threads - 1) / threads;
-  topk_kernel<<<blocks, threads, 0, s>>>(logits, T, E, k, norm_topk, topk_idx, topk_w);
+cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
+                                 const float *bias, int T, int d, int E, int k, int norm_topk,
+                                 int32_t *topk_idx, float *topk_w, cudaStream_t s) {
+  const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
+  router_select_kernel<<<blocks, kSelectWarps * 32, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
+                                                           norm_topk, topk_idx, topk_w);
   return cudaGetLastError();
 }
 

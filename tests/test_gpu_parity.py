@@ -179,8 +179,8 @@ def test_exact_ties_go_to_lower_expert_index(flags):
     wr[14] = wr[5]
     h["w_router"] = wr
     dev = G.host_to_device(h)
-    y, routing, ws = G.run_forward(w, dev, flags=flags | M.MOE_FLAG_WRITE_LOGITS)
-    off = M.logits_offset(M.dims_for(w, flags=flags | M.MOE_FLAG_WRITE_LOGITS))
+    y, routing, ws = G.run_forward(w, dev, flags=flags)
+    off = M.logits_offset(M.dims_for(w, flags=flags))
     logits = ws[off:off + w.T * w.E * 4].view(torch.float32).view(w.T, w.E).cpu().numpy()
     assert np.array_equal(logits[:, 2], logits[:, 9]) and np.array_equal(logits[:, 5], logits[:, 14])
     idx = routing["topk_idx"].cpu().numpy()
@@ -201,7 +201,7 @@ def test_router_logits_error_against_float64(flags):
            "w_router": torch.empty((w.E, w.d_model), dtype=torch.bfloat16, device="cuda")}
     I.generate_cuda(dev["x"], w.seed, I.TID_X, w.sigma_x)
     I.generate_cuda(dev["w_router"], w.seed, I.TID_W_ROUTER, w.sigma_router)
-    dims = M.dims_for(w, flags=flags | M.MOE_FLAG_WRITE_LOGITS)
+    dims = M.dims_for(w, flags=flags)
     ws = M.alloc_workspace(dims)
     idx = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
     wt = torch.empty((w.T, w.k), dtype=torch.float32, device="cuda")
@@ -211,9 +211,10 @@ def test_router_logits_error_against_float64(flags):
     got = ws[off:off + w.T * w.E * 4].view(torch.float32).view(w.T, w.E).cpu().numpy()
     ref = O.router_logits(P.to_numpy_bf16(dev["x"]), P.to_numpy_bf16(dev["w_router"]), None)
     err = float(np.abs(got - ref).max())
-    # a logit error below 4e-6 is a score error below 1e-6 (the sigmoid's slope is <= 1/4),
-    # so any selection it flips lies inside the near-tie exemption band
-    assert err < 4e-6, err
+    # the select kernel re-decides, on float64 logits, every token whose k-th and
+    # (k+1)-th fp32 logits are within 2e-4; that is exact as long as the fp32
+    # logit error stays below half of it (measured: ~1.2e-5 tensor, < 4e-6 CUDA core)
+    assert err < 1e-4 / 4, err
 
 
 def test_prepared_down_weights_match_per_call_conversion():
