@@ -181,6 +181,28 @@ moe_status moe_selftest_bounded_wait(void *ws, size_t ws_bytes, uint32_t limit_u
  * recorded.  Pass events = NULL to disarm. */
 moe_status moe_profile_next_forward(void **events, int32_t n_events);
 
+/* Size of the library's static scratch array used by moe_permute_static. */
+#define MOE_STATIC_SCRATCH_BYTES (512u * 1024u)
+
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory (code that runs inside another runtime's memory pool, plugins whose
+ * host process owns all device memory, or work being captured into a CUDA
+ * graph where an allocation would break the capture).  The paper has no
+ * counterpart to this entry point; it is a deployment convenience.
+ * Same outputs as moe_permute without x / x_perm: counts [E], offsets [E + 1],
+ * perm [T * k].  Its scratch is one static device array of
+ * MOE_STATIC_SCRATCH_BYTES per GPU, held from library load to process exit;
+ * enough for T * k up to 262144 at E = 256.  Dims that need more return
+ * MOE_ERR_UNSUPPORTED_SHAPE, and nothing is launched.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current): make that first call before any stream capture.  Every
+ * call uses the same array, so calls that overlap on the GPU (other streams,
+ * or other host threads) race; serialise them.  An expert id outside [0, E)
+ * is skipped on the device and is not reported by this entry point.  It
+ * calls no cudaMalloc, cudaFree or allocating library routine. */
+moe_status moe_permute_static(const moe_dims_t *dims, const int32_t *topk_idx, int32_t *counts,
+                              int32_t *offsets, int32_t *perm, void *stream);
+
 /* Human-readable name of a status code (static string). */
 const char *moe_status_string(moe_status s);
 

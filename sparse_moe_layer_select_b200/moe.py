@@ -29,7 +29,7 @@ MOE_FLAG_DOWN_F16 = 4
 EXPORTED = ["moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
             "moe_read_device_status", "moe_selftest_bounded_wait", "moe_status_string",
             "moe_last_launch_count", "moe_profile_next_forward", "moe_prepare_down_f16",
-            "moe_logits_offset"]
+            "moe_logits_offset", "moe_permute_static"]
 
 
 class MoeError(RuntimeError):
@@ -93,6 +93,8 @@ def lib():
         L.moe_last_launch_count.argtypes = []
         L.moe_prepare_down_f16.restype = ctypes.c_int
         L.moe_prepare_down_f16.argtypes = [D, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_permute_static.restype = ctypes.c_int
+        L.moe_permute_static.argtypes = [D, P, P, P, P, P]
         L.moe_logits_offset.restype = ctypes.c_size_t
         L.moe_logits_offset.argtypes = [D]
         L.moe_profile_next_forward.restype = ctypes.c_int
