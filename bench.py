@@ -189,7 +189,8 @@ def run_ours(args):
     decode = w.decode_batches > 0
     ring = I.device_decode_ring(w, min(w.decode_batches, 1000)) if decode else None
     layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
-                       max_tokens=w.T)
+                       max_tokens=w.T,
+                       flags=M.MOE_FLAG_GEMM_SINGLE_CTA if args.single_cta else 0)
     x_buf = dev["x"]
     y = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
@@ -338,6 +339,7 @@ def run_ours(args):
                    "num_experts_per_tok": w.k, "moe_intermediate_size": w.F,
                    "shared_intermediate_size": w.Fs, "routed_scaling_factor": w.routed_scaling_factor,
                    "router_bias": "zipf" if w.zipf_s else None, "parallelism": f"replicas x{world}",
+                   "gemm_engine": "single-CTA M=128" if args.single_cta else "CTA-pair M=256",
                    "l2": "L2 flushed between steps" if flush else
                          f"inputs larger than L2 ({working_set / 1e9:.2f} GB resident)"},
         "roofline": roof, "expert_gemm": expert,
@@ -416,6 +418,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--single-cta", action="store_true",
+                    help="expert GEMMs on single CTAs (M=128) instead of CTA pairs (M=256)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -81,6 +81,9 @@ typedef struct {
  * ws_down_f16, made once by moe_prepare_down_f16); without this flag
  * moe_forward converts them into the workspace on every call. */
 #define MOE_FLAG_DOWN_F16         4
+/* Run the expert GEMMs on single CTAs (M = 128 tiles) instead of CTA pairs
+ * (clusters of two SMs, M = 256 tiles); same results, for comparison. */
+#define MOE_FLAG_GEMM_SINGLE_CTA  8
 
 typedef struct {
     const void *w_router;      /* [E, d] bf16 */

@@ -8,15 +8,21 @@
 //   counts[e]  rows of expert e;  offsets = exclusive prefix sum (E + 1)
 //   perm[r]    = t * k + j for the r-th row in expert order, rows of one
 //                expert in ascending (t, j) -- a stable counting sort.
-//   tiles      (expert, first row, rows) blocks of at most 128 rows, in
-//              expert order, followed by the shared expert's token blocks.
+//   tiles      (expert, first row, rows) blocks of at most tile_rows rows
+//              (128 for single-CTA GEMMs, 256 for CTA-pair GEMMs), in expert
+//              order, followed by the shared expert's token blocks.
 //
-// Three launches, all deterministic:
-//   index_hist_kernel     per-chunk expert histogram (chunk = 1024 entries)
-//   index_scan_kernel     one CTA: per-expert running sums over chunks, an
-//                         exclusive scan over experts, tile list
-//   index_scatter_kernel  one warp per chunk: entries in index order, ranks
-//                         among equal experts from __match_any_sync
+// The (t, j) entries are cut into chunks of kIndexChunk = 4096, one CTA of 8
+// warps per chunk, each warp owning 512 consecutive entries:
+//   index_hist_kernel     per-chunk expert histogram
+//   index_scan_kernel     one CTA: per-expert sums over chunks, exclusive
+//                         scan over experts, chunk bases, tile list
+//   index_scatter_kernel  per chunk: per-warp histograms and their scan give
+//                         each warp its first row per expert; each warp then
+//                         places its entries in order, ranks among equal
+//                         experts from __match_any_sync (stable, deterministic)
+// With a single chunk (decode-sized batches) one CTA does all three steps in
+// one launch (index_single_kernel).
 #include "kernels.h"
 #include "status.cuh"
 
@@ -25,29 +31,12 @@ namespace moe {
 namespace {
 
 constexpr int kMaxE = 512;
+constexpr int kIdxWarps = 8;
+constexpr int kSub = kIndexChunk / kIdxWarps;  // 512 entries per warp
+static_assert(kIndexChunk % (kIdxWarps * 32) == 0, "chunk layout");
 
-__global__ void __launch_bounds__(256)
-    index_hist_kernel(const int32_t *__restrict__ topk_idx, int n, int E,
-                      int *__restrict__ chunk_hist, int *status) {
-  __shared__ int h[kMaxE];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
-  __syncthreads();
-  const int base = blockIdx.x * kIndexChunk;
-  const int end = min(n, base + kIndexChunk);
-  for (int i = base + threadIdx.x; i < end; i += blockDim.x) {
-    const int e = topk_idx[i];
-    if (e < 0 || e >= E) {
-      record_status(status, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
-      continue;
-    }
-    atomicAdd(&h[e], 1);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = h[e];
-}
-
-// Block-wide exclusive scan of one value per thread (blockDim.x == 512).
+// Block-wide exclusive scan of one value per thread (blockDim.x a multiple of
+// 32, at most 1024).
 __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -77,62 +66,40 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int *
   return r;
 }
 
-__global__ void __launch_bounds__(512)
-    index_scan_kernel(int *__restrict__ chunk_hist, int nchunks, int E, int T, int with_shared,
-                      int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                      Tile *__restrict__ tiles, int *__restrict__ header) {
-  __shared__ int warp_sums[32];
-  __shared__ int total_rows, total_tiles;
-  const int e = threadIdx.x;
-  int cnt = 0;
-  if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      int *p = chunk_hist + static_cast<size_t>(c) * E + e;
-      const int v = *p;
-      *p = cnt;  // chunk base relative to the expert's first row
-      cnt += v;
+// Per-warp expert histograms of one chunk into h[kIdxWarps][E] (shared).
+__device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk_idx, int n,
+                                                int E, int chunk, int *h, int *status) {
+  for (int i = threadIdx.x; i < kIdxWarps * E; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int base = chunk * kIndexChunk + warp * kSub;
+  int *hw = h + warp * E;
+  for (int r = lane; r < kSub; r += 32) {
+    const int i = base + r;
+    if (i >= n) break;
+    const int e = topk_idx[i];
+    if (e < 0 || e >= E) {
+      if (status) record_status(status, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
+      continue;
     }
+    atomicAdd(&hw[e], 1);
   }
-  const int off = block_exclusive_scan(e < E ? cnt : 0, warp_sums, &total_rows);
-  const int ntile = e < E ? (cnt + kBlockM - 1) / kBlockM : 0;
-  const int toff = block_exclusive_scan(ntile, warp_sums, &total_tiles);
-  if (e < E) {
-    counts[e] = cnt;
-    offsets[e] = off;
-    for (int c = 0; c < nchunks; ++c) chunk_hist[static_cast<size_t>(c) * E + e] += off;
-    for (int i = 0; i < ntile; ++i) {
-      Tile t;
-      t.group = e;
-      t.row0 = off + i * kBlockM;
-      t.nrows = min(kBlockM, cnt - i * kBlockM);
-      t.pad = 0;
-      tiles[toff + i] = t;
-    }
-  }
-  if (e == 0) offsets[E] = total_rows;
-  const int nshared = with_shared ? (T + kBlockM - 1) / kBlockM : 0;
-  for (int i = threadIdx.x; i < nshared; i += blockDim.x) {
-    Tile t;
-    t.group = E;
-    t.row0 = i * kBlockM;
-    t.nrows = min(kBlockM, T - i * kBlockM);
-    t.pad = 0;
-    tiles[total_tiles + i] = t;
-  }
-  if (threadIdx.x == 0) reinterpret_cast<WsHeader *>(header)->n_tiles = total_tiles + nshared;
+  __syncthreads();
 }
 
-__global__ void __launch_bounds__(32)
-    index_scatter_kernel(const int32_t *__restrict__ topk_idx, int n, int E,
-                         const int *__restrict__ chunk_base, int32_t *__restrict__ perm) {
-  __shared__ int fill[kMaxE];
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) fill[e] = chunk_base[static_cast<size_t>(blockIdx.x) * E + e];
-  __syncwarp();
-  const int base = blockIdx.x * kIndexChunk;
+// Each warp places its 512 entries: fill[warp][e] holds its next row of e.
+__device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ topk_idx, int n,
+                                                   int E, int chunk, int *fill,
+                                                   int32_t *__restrict__ perm) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  for (int r = 0; r < kIndexChunk; r += 32) {
+  int *fw = fill + warp * E;
+  const int base = chunk * kIndexChunk + warp * kSub;
+  for (int r = 0; r < kSub; r += 32) {
     const int i = base + r + lane;
+    if (base + r >= n) break;  // warp-uniform
     int e = -1;
     if (i < n) {
       e = topk_idx[i];
@@ -140,28 +107,191 @@ __global__ void __launch_bounds__(32)
     }
     const unsigned m = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(m & lt);
-    if (e >= 0) perm[fill[e] + rank] = i;
+    if (e >= 0) perm[fw[e] + rank] = i;
     __syncwarp();
-    if (e >= 0 && rank == 0) fill[e] += __popc(m);
+    if (e >= 0 && rank == 0) fw[e] += __popc(m);
     __syncwarp();
   }
+}
+
+// Turn the chunk's per-warp histograms h[w][e] into per-warp first rows,
+// starting from the chunk's base row of each expert.
+__device__ __forceinline__ void warp_bases(int E, const int *chunk_base_e, int *h) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = chunk_base_e[e];
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) {
+      const int c = h[w * E + e];
+      h[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kIdxWarps * 32)
+    index_hist_kernel(const int32_t *__restrict__ topk_idx, int n, int E,
+                      int *__restrict__ chunk_hist, int *status) {
+  __shared__ int h[kIdxWarps * kMaxE];
+  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, status);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) s += h[w * E + e];
+    chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = s;
+  }
+}
+
+// Expert sums over chunks, exclusive scan over experts, chunk bases and the
+// tile list.  One CTA of 512 threads (one thread per expert).
+__device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int nchunks, int E,
+                                               int T, int with_shared, int tile_rows,
+                                               int32_t *__restrict__ counts,
+                                               int32_t *__restrict__ offsets,
+                                               Tile *__restrict__ tiles, int *__restrict__ header,
+                                               int *warp_sums, int *totals) {
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < E) {
+    int c = 0;
+    for (; c + 8 <= nchunks; c += 8) {  // eight independent loads in flight
+      int v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = chunk_hist[static_cast<size_t>(c + q) * E + e];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) cnt += v[q];
+    }
+    for (; c < nchunks; ++c) cnt += chunk_hist[static_cast<size_t>(c) * E + e];
+  }
+  const int off = block_exclusive_scan(e < E ? cnt : 0, warp_sums, &totals[0]);
+  const int ntile = e < E ? (cnt + tile_rows - 1) / tile_rows : 0;
+  const int toff = block_exclusive_scan(ntile, warp_sums, &totals[1]);
+  if (e < E) {
+    counts[e] = cnt;
+    offsets[e] = off;
+    int run = off;
+    int c = 0;
+    for (; c + 8 <= nchunks; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = chunk_hist[static_cast<size_t>(c + q) * E + e];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        chunk_hist[static_cast<size_t>(c + q) * E + e] = run;  // chunk base row of expert e
+        run += v[q];
+      }
+    }
+    for (; c < nchunks; ++c) {
+      const int v = chunk_hist[static_cast<size_t>(c) * E + e];
+      chunk_hist[static_cast<size_t>(c) * E + e] = run;
+      run += v;
+    }
+    for (int i = 0; i < ntile; ++i) {
+      Tile t;
+      t.group = e;
+      t.row0 = off + i * tile_rows;
+      t.nrows = min(tile_rows, cnt - i * tile_rows);
+      t.pad = 0;
+      tiles[toff + i] = t;
+    }
+  }
+  if (e == 0) offsets[E] = totals[0];
+  const int nshared = with_shared ? (T + tile_rows - 1) / tile_rows : 0;
+  for (int i = threadIdx.x; i < nshared; i += blockDim.x) {
+    Tile t;
+    t.group = E;
+    t.row0 = i * tile_rows;
+    t.nrows = min(tile_rows, T - i * tile_rows);
+    t.pad = 0;
+    tiles[totals[1] + i] = t;
+  }
+  if (threadIdx.x == 0 && header) reinterpret_cast<WsHeader *>(header)->n_tiles = totals[1] + nshared;
+}
+
+__global__ void __launch_bounds__(512)
+    index_scan_kernel(int *__restrict__ chunk_hist, int nchunks, int E, int T, int with_shared,
+                      int tile_rows, int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                      Tile *__restrict__ tiles, int *__restrict__ header) {
+  __shared__ int warp_sums[32];
+  __shared__ int totals[2];
+  scan_and_tiles(chunk_hist, nchunks, E, T, with_shared, tile_rows, counts, offsets, tiles,
+                 header, warp_sums, totals);
+}
+
+__global__ void __launch_bounds__(kIdxWarps * 32)
+    index_scatter_kernel(const int32_t *__restrict__ topk_idx, int n, int E,
+                         const int *__restrict__ chunk_base, int32_t *__restrict__ perm) {
+  __shared__ int h[kIdxWarps * kMaxE];
+  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, nullptr);
+  warp_bases(E, chunk_base + static_cast<size_t>(blockIdx.x) * E, h);
+  chunk_warp_scatter(topk_idx, n, E, blockIdx.x, h, perm);
+}
+
+// All of the above for a single chunk (n <= kIndexChunk), in one CTA of 512
+// threads: warps 0..7 do the histogram and scatter, all 16 the scan.
+__global__ void __launch_bounds__(512)
+    index_single_kernel(const int32_t *__restrict__ topk_idx, int n, int E, int T,
+                        int with_shared, int tile_rows, int *__restrict__ chunk_hist,
+                        int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                        int32_t *__restrict__ perm, Tile *__restrict__ tiles, int *header) {
+  __shared__ int h[kIdxWarps * kMaxE];
+  __shared__ int warp_sums[32];
+  __shared__ int totals[2];
+  const int warp = threadIdx.x >> 5;
+  // histogram by the first eight warps (the others only clear and wait)
+  for (int i = threadIdx.x; i < kIdxWarps * E; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  if (warp < kIdxWarps) {
+    const int lane = threadIdx.x & 31;
+    int *hw = h + warp * E;
+    for (int r = lane; r < kSub; r += 32) {
+      const int i = warp * kSub + r;
+      if (i >= n) break;
+      const int e = topk_idx[i];
+      if (e < 0 || e >= E) {
+        record_status(header, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
+        continue;
+      }
+      atomicAdd(&hw[e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) s += h[w * E + e];
+    chunk_hist[e] = s;
+  }
+  __syncthreads();
+  scan_and_tiles(chunk_hist, 1, E, T, with_shared, tile_rows, counts, offsets, tiles, header,
+                 warp_sums, totals);
+  __syncthreads();
+  warp_bases(E, chunk_hist, h);
+  if (warp < kIdxWarps) chunk_warp_scatter(topk_idx, n, E, 0, h, perm);
 }
 
 }  // namespace
 
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
-                         int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches) {
+                         int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
+                         int tile_rows) {
   const int n = T * k;
   const int nchunks = (n + kIndexChunk - 1) / kIndexChunk;
-  index_hist_kernel<<<nchunks, 256, 0, s>>>(topk_idx, n, E, chunk_hist, status);
+  if (nchunks == 1) {
+    index_single_kernel<<<1, 512, 0, s>>>(topk_idx, n, E, T, with_shared, tile_rows, chunk_hist,
+                                          counts, offsets, perm, tiles, status);
+    *launches += 1;
+    return cudaGetLastError();
+  }
+  index_hist_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  index_scan_kernel<<<1, 512, 0, s>>>(chunk_hist, nchunks, E, T, with_shared, counts, offsets,
-                                      tiles, status);
+  index_scan_kernel<<<1, 512, 0, s>>>(chunk_hist, nchunks, E, T, with_shared, tile_rows, counts,
+                                      offsets, tiles, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  index_scatter_kernel<<<nchunks, 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm);
+  index_scatter_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm);
   *launches += 3;
   return cudaGetLastError();
 }

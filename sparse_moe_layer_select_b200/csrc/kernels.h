@@ -22,7 +22,7 @@ constexpr int kBlockM = 128;        // rows per tile (tcgen05 M)
 constexpr int kBlockK = 64;         // K elements per pipeline stage (one 128-byte swizzle row)
 constexpr int kStages = 4;          // shared-memory pipeline depth
 constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kIndexChunk = 1024;   // (token, slot) entries per index-builder chunk
+constexpr int kIndexChunk = 4096;   // (token, slot) entries per index-builder chunk
 
 enum GemmMode : int { MODE_ROUTER = 0, MODE_GEMM1 = 1, MODE_GEMM2 = 2 };
 
@@ -56,6 +56,10 @@ struct GemmMaps {
 size_t gemm_smem_bytes();
 cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int grid,
                         cudaStream_t s);
+// CTA-pair (cluster of 2, M = 256) variant of MODE_GEMM1 / MODE_GEMM2; grid even.
+size_t gemm_pair_smem_bytes();
+cudaError_t launch_gemm_pair(int mode, const GemmParams &p, const GemmMaps &m, int grid,
+                             cudaStream_t s);
 
 cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
                              float *logits, int T, int d, int E, cudaStream_t s);
@@ -65,7 +69,8 @@ cudaError_t launch_router_select(const float *logits, const uint16_t *x, const u
 
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
-                         int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches);
+                         int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
+                         int tile_rows = kBlockM);
 cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_rows, int k, int d,
                                uint16_t *x_perm, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *slots, int T, int nslots, int d, uint16_t *y,

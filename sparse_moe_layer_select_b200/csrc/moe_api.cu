@@ -16,6 +16,8 @@
 
 namespace moe {
 cudaError_t gemm_set_attributes();
+cudaError_t gemm_pair_set_attributes();
+cudaError_t gemm_pair_max_clusters(int *clusters);
 }
 
 namespace {
@@ -47,6 +49,7 @@ struct EventMarker {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int g_sms[kMaxDevices] = {0};
+int g_pair_clusters[kMaxDevices] = {0};
 bool g_attrs[kMaxDevices] = {false};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -70,10 +73,20 @@ cudaError_t device_setup(int *sms) {
     if (e != cudaSuccess) return e;
     e = gemm_set_attributes();
     if (e != cudaSuccess) return e;
+    e = gemm_pair_set_attributes();
+    if (e != cudaSuccess) return e;
+    e = gemm_pair_max_clusters(&g_pair_clusters[dev]);
+    if (e != cudaSuccess) return e;
     g_attrs[dev] = true;
   }
   *sms = g_sms[dev];
   return cudaSuccess;
+}
+
+int pair_clusters() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < kMaxDevices) ? g_pair_clusters[dev] : 0;
 }
 
 // 2-D 16-bit tensor [rows, cols] (row-major), 128-byte swizzle, box 64 x box_rows.
@@ -337,11 +350,14 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   st = route_impl(D, x, w->w_router, w->router_bias, routing->topk_idx, routing->topk_w, ws, s,
                   sms, &launches);
   if (st != MOE_OK) return st;
-  // 2. expert order + tile list
+  // 2. expert order + tile list (256-row tiles for the CTA-pair GEMMs)
+  const int pair_grid = 2 * std::min(pair_clusters(), sms / 2);  // all pairs co-resident
+  const bool pair = !(D.flags & MOE_FLAG_GEMM_SINGLE_CTA) && pair_grid >= 2;
   ev.mark();
   if (launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0,
                    reinterpret_cast<int *>(wsp(ws, L.chunk_hist)), tiles, header, routing->counts,
-                   routing->offsets, routing->perm, s, &launches) != cudaSuccess)
+                   routing->offsets, routing->perm, s, &launches,
+                   pair ? 2 * kBlockM : kBlockM) != cudaSuccess)
     return MOE_ERR_CUDA;
 
   // fp16 down projections: caller-prepared, or converted here every call
@@ -409,9 +425,10 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
       m.b0_sh = m.b0;
       m.b1_sh = m.b1;
     }
-    const int grid = sms;
     ev.mark();
-    if (launch_gemm(MODE_GEMM1, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const cudaError_t e = pair ? launch_gemm_pair(MODE_GEMM1, p, m, pair_grid, s)
+                               : launch_gemm(MODE_GEMM1, p, m, sms, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
   }
   // 4. GEMM2: h . W_down^T -> x (routed_scaling_factor * w) -> slot rows
@@ -427,20 +444,22 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     std::memset(&m, 0, sizeof(m));
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (!make_map(&m.a, h, n_rows, D.F, a_rows, f16)) return MOE_ERR_CUDA;
-    if (!make_map(&m.b0, wd16, static_cast<uint64_t>(D.E) * D.d, D.F, n2, f16))
+    const uint32_t b_rows = pair ? n2 / 2 : n2;  // a pair splits B along N
+    if (!make_map(&m.b0, wd16, static_cast<uint64_t>(D.E) * D.d, D.F, b_rows, f16))
       return MOE_ERR_CUDA;
     m.b1 = m.b0;
     if (D.Fs > 0) {
       if (!make_map(&m.a_sh, h_sh, D.T, D.Fs, a_sh_rows, f16)) return MOE_ERR_CUDA;
-      if (!make_map(&m.b0_sh, wsd16, D.d, D.Fs, n2, f16)) return MOE_ERR_CUDA;
+      if (!make_map(&m.b0_sh, wsd16, D.d, D.Fs, b_rows, f16)) return MOE_ERR_CUDA;
     } else {
       m.a_sh = m.a;
       m.b0_sh = m.b0;
     }
     m.b1_sh = m.b0_sh;
-    const int grid = sms;
     ev.mark();
-    if (launch_gemm(MODE_GEMM2, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const cudaError_t e = pair ? launch_gemm_pair(MODE_GEMM2, p, m, pair_grid, s)
+                               : launch_gemm(MODE_GEMM2, p, m, sms, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
   }
   // 5. combine: y = bf16(sum of the scaled routed slots + shared slot)

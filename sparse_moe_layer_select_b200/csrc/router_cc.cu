@@ -84,7 +84,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   }
 }
 
-constexpr int kMaxPerLane = 16;  // E <= 512
 constexpr int kSelectWarps = 8;
 
 // Width of the ambiguous band around the k-th/(k+1)-th boundary, in logit
@@ -146,11 +145,21 @@ __device__ __forceinline__ void warp_argmax(float &bv, int &be) {
   }
 }
 
-// One warp per token: register top-(k+1) of the fp32 logits (ties to the lower
-// expert index), float64 refinement of the experts near the boundary when the
-// k-th and (k+1)-th logits are closer than kRefineBand, then sigmoid scores
-// and post-top-k normalisation (Laguna M.1/XS.2 Technical Report summary, Key
-// claims, report §3.1; Laguna-M.1-base spec sheet, Mixture of experts).
+// (value, expert) order of the selection: larger logit first, equal logits
+// by lower expert id; NaN (empty slot) after everything.
+__device__ __forceinline__ bool sel_before(float va, int ea, float vb, int eb) {
+  return va > vb || (va == vb && ea < eb) || (va == va && vb != vb);
+}
+
+// One warp per token: each lane sorts its NPL = E/32 logits once (odd-even
+// transposition network, registers only); each of the k+1 rounds then takes
+// the warp arg-max of the 32 list heads (ties to the lower expert id) and the
+// winning lane pops its head.  Tokens whose k-th and (k+1)-th logits are
+// within kRefineBand get the experts near that boundary re-decided on
+// float64 logits.  Then sigmoid scores and post-top-k normalisation (Laguna
+// M.1/XS.2 Technical Report summary, Key claims, report §3.1; Laguna-M.1-base
+// spec sheet, Mixture of experts).
+template <int NPL>
 __global__ void __launch_bounds__(kSelectWarps * 32)
     router_select_kernel(const float *__restrict__ logits, const uint16_t *__restrict__ x,
                          const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
@@ -160,32 +169,55 @@ __global__ void __launch_bounds__(kSelectWarps * 32)
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   const float *row = logits + static_cast<size_t>(t) * E;
-  const float kNaN = __int_as_float(0x7fc00000);  // compares false: never selected
-  float v[kMaxPerLane];
+  const float kNaN = __int_as_float(0x7fc00000);
+  float v[NPL];
+  int ev[NPL];
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? row[e] : kNaN;
+  for (int i = 0; i < NPL; ++i) {
+    ev[i] = lane + 32 * i;
+    v[i] = ev[i] < E ? row[ev[i]] : kNaN;
+  }
+  // sort descending (NPL rounds of odd-even transposition)
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+#pragma unroll
+    for (int i = r & 1; i + 1 < NPL; i += 2) {
+      if (sel_before(v[i + 1], ev[i + 1], v[i], ev[i])) {
+        const float tv = v[i];
+        const int te = ev[i];
+        v[i] = v[i + 1];
+        ev[i] = ev[i + 1];
+        v[i + 1] = tv;
+        ev[i + 1] = te;
+      }
+    }
   }
   float my_l = 0.f;  // lane j < k keeps the j-th selected logit and expert
   int my_e = 0;
   float lk = 0.f, lk1 = -INFINITY;
   const int rounds = k < E ? k + 1 : k;
   for (int j = 0; j < rounds; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+    float bv = v[0];
+    int be = ev[0];
+    const int my_head = be;
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-      const int e = lane + 32 * i;
-      if (v[i] > bv || (v[i] == bv && e < be)) {
-        bv = v[i];
-        be = e;
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (sel_before(ov, oe, bv, be)) {
+        bv = ov;
+        be = oe;
       }
     }
-    warp_argmax(bv, be);
+    if (my_head == be) {  // pop the head
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i)
-      if (lane + 32 * i == be) v[i] = kNaN;
+      for (int i = 0; i + 1 < NPL; ++i) {
+        v[i] = v[i + 1];
+        ev[i] = ev[i + 1];
+      }
+      v[NPL - 1] = kNaN;
+      ev[NPL - 1] = 0x7fffffff;
+    }
     if (j < k && lane == j) {
       my_l = bv;
       my_e = be;
@@ -202,7 +234,7 @@ __global__ void __launch_bounds__(kSelectWarps * 32)
     double best_l[16];
     int best_e[16];
     int nbest = 0;
-    for (int i = 0; i < kMaxPerLane; ++i) {
+    for (int i = 0; i < (E + 31) / 32; ++i) {
       const int e_lane = lane + 32 * i;
       const bool cand = e_lane < E && row[e_lane] >= lo;
       unsigned m = __ballot_sync(0xffffffffu, cand);
@@ -281,8 +313,23 @@ cudaError_t launch_router_select(const float *logits, const uint16_t *x, const u
                                  const float *bias, int T, int d, int E, int k, int norm_topk,
                                  int32_t *topk_idx, float *topk_w, cudaStream_t s) {
   const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
-  router_select_kernel<<<blocks, kSelectWarps * 32, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
-                                                           norm_topk, topk_idx, topk_w);
+  const int threads = kSelectWarps * 32;
+  const int npl = (E + 31) / 32;
+  if (npl <= 1)
+    router_select_kernel<1><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
+                                                       norm_topk, topk_idx, topk_w);
+  else if (npl <= 2)
+    router_select_kernel<2><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
+                                                       norm_topk, topk_idx, topk_w);
+  else if (npl <= 4)
+    router_select_kernel<4><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
+                                                       norm_topk, topk_idx, topk_w);
+  else if (npl <= 8)
+    router_select_kernel<8><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
+                                                       norm_topk, topk_idx, topk_w);
+  else
+    router_select_kernel<16><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
+                                                        norm_topk, topk_idx, topk_w);
   return cudaGetLastError();
 }
 

@@ -76,11 +76,15 @@ def test_router_paths_match_oracle(flags, T):
     G.check_routing(idx.cpu().numpy(), wt.cpu().numpy(), ref, w.k)
 
 
-@pytest.mark.parametrize("T", [1, 127, 128, 129, 1000])
-def test_ragged_and_multi_tile_forward(T):
+ENGINES = [0, M.MOE_FLAG_GEMM_SINGLE_CTA]  # CTA-pair (M = 256) and single-CTA (M = 128) GEMMs
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+@pytest.mark.parametrize("T", [1, 127, 128, 129, 255, 256, 257, 1000])
+def test_ragged_and_multi_tile_forward(T, engine):
     w = I.get("c1_tiny").with_(T=T)
     h, dev = _small(w)
-    y, routing, _ = G.run_forward(w, dev)
+    y, routing, _ = G.run_forward(w, dev, flags=engine)
     ref = G.oracle_forward(w, h)
     G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
     G.check_output(G.y_numpy(y), ref["y"], what=f"T={T}")
@@ -159,7 +163,8 @@ def test_zero_shared_weights_isolate_routed_path():
     G.check_output(G.y_numpy(y), 2.5 * ref["R"], what="shared=0")
 
 
-@pytest.mark.parametrize("E,k", [(2, 1), (2, 2), (4, 1), (4, 3), (8, 1), (8, 4), (8, 8), (16, 16)])
+@pytest.mark.parametrize("E,k", [(2, 1), (2, 2), (4, 1), (4, 3), (8, 1), (8, 4), (8, 8), (16, 16),
+                                 (24, 5), (40, 16), (300, 8), (512, 16)])
 def test_small_expert_counts_and_k_extremes(E, k):
     w = I.get("c1_tiny").with_(T=257, num_experts=E, num_experts_per_tok=k)
     h, dev = _small(w)
@@ -243,7 +248,8 @@ def test_fp16_range_violation_is_reported():
     assert code == M.MOE_ERR_DEVICE_BOUNDS and site == 32
 
 
-def test_maximum_skew_all_tokens_on_the_same_experts():
+@pytest.mark.parametrize("engine", ENGINES)
+def test_maximum_skew_all_tokens_on_the_same_experts(engine):
     import torch
     w = I.get("c1_tiny").with_(T=1000)
     h, dev = _small(w)
@@ -251,7 +257,7 @@ def test_maximum_skew_all_tokens_on_the_same_experts():
     bias[[3, 7, 11, 12]] = 100.0   # every token selects experts 3, 7, 11, 12
     h["router_bias"] = bias
     dev["router_bias"] = torch.from_numpy(bias).cuda()
-    y, routing, _ = G.run_forward(w, dev)
+    y, routing, _ = G.run_forward(w, dev, flags=engine)
     counts = routing["counts"].cpu().numpy()
     assert counts[[3, 7, 11, 12]].tolist() == [1000] * 4 and counts.sum() == 4000
     ref = G.oracle_forward(w, h)
@@ -296,11 +302,12 @@ def _device_workload(w):
     return h, dev
 
 
-def test_xs2_dims_multi_tile_full_oracle():
+@pytest.mark.parametrize("engine", ENGINES)
+def test_xs2_dims_multi_tile_full_oracle(engine):
     """XS.2 widths at T=1000: every token through the oracle (ragged tiles everywhere)."""
     w = I.get("c2_xs2_small").with_(T=1000)
     h, dev = _device_workload(w)
-    y, routing, _ = G.run_forward(w, dev)
+    y, routing, _ = G.run_forward(w, dev, flags=engine)
     ref = G.oracle_forward(w, h)
     G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
     same = P.same_selection_mask(routing["topk_idx"].cpu().numpy(), ref["topk_idx"])
