@@ -190,7 +190,8 @@ def run_ours(args):
     ring = I.device_decode_ring(w, min(w.decode_batches, 1000)) if decode else None
     layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
                        max_tokens=w.T,
-                       flags=M.MOE_FLAG_GEMM_SINGLE_CTA if args.single_cta else 0)
+                       flags=(M.MOE_FLAG_GEMM_SINGLE_CTA if args.single_cta else 0)
+                       | (M.MOE_FLAG_GEMM_PAIR if args.pair else 0))
     x_buf = dev["x"]
     y = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
@@ -198,9 +199,14 @@ def run_ours(args):
     flush = working_set < 2 * L2_BYTES
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device="cuda") if flush else None
 
+    graph = None
+
     def step(i, events=None):
         if decode:
             x_buf.copy_(ring[i % ring.shape[0]], non_blocking=True)
+        if graph is not None:
+            graph.replay()
+            return
         if events is not None:
             M.profile_next_forward(events)
         layer.forward(x_buf, y)
@@ -222,6 +228,15 @@ def run_ours(args):
     if code != 0:
         raise RuntimeError(f"device status {M.status_string(code)} at site {site}")
     launches_per_step = M.last_launch_count() + (1 if decode else 0)
+    if decode and not args.no_graph:
+        # decode: the layer is captured once in a CUDA graph and replayed per batch
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer.forward(x_buf, y)
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
 
     n_st = len(M.FORWARD_STAGES)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)] for _ in range(args.steps)]
@@ -261,8 +276,23 @@ def run_ours(args):
         raise RuntimeError(f"device status {M.status_string(code)} at site {site}")
 
     stage_ms = {}
-    for j, name in enumerate(M.FORWARD_STAGES):
-        stage_ms[name] = float(np.mean([ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)]))
+    if graph is not None:
+        # events recorded inside a graph cannot be timed: the stage breakdown of the
+        # decode workload comes from five eager calls after the timed graph replays
+        acc = np.zeros(len(M.FORWARD_STAGES))
+        for i in range(5):
+            x_buf.copy_(ring[i % ring.shape[0]], non_blocking=True)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(M.FORWARD_STAGES) + 1)]
+            M.profile_next_forward(evs)
+            layer.forward(x_buf, y)
+            torch.cuda.synchronize()
+            acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(M.FORWARD_STAGES))]
+        for j, name in enumerate(M.FORWARD_STAGES):
+            stage_ms[name] = float(acc[j] / 5)
+    else:
+        for j, name in enumerate(M.FORWARD_STAGES):
+            stage_ms[name] = float(np.mean([ev[i][j].elapsed_time(ev[i][j + 1])
+                                            for i in range(args.steps)]))
 
     # end to end through the C ABI: pinned host batch in, host output back, every step
     e2e = None
@@ -339,12 +369,14 @@ def run_ours(args):
                    "num_experts_per_tok": w.k, "moe_intermediate_size": w.F,
                    "shared_intermediate_size": w.Fs, "routed_scaling_factor": w.routed_scaling_factor,
                    "router_bias": "zipf" if w.zipf_s else None, "parallelism": f"replicas x{world}",
-                   "gemm_engine": "single-CTA M=128" if args.single_cta else "CTA-pair M=256",
+                   "gemm_engine": ("single-CTA M=128" if args.single_cta else "CTA-pair M=256"
+                                   if args.pair else "auto (CTA pairs when T*k >= 256*E)"),
                    "l2": "L2 flushed between steps" if flush else
                          f"inputs larger than L2 ({working_set / 1e9:.2f} GB resident)"},
         "roofline": roof, "expert_gemm": expert,
         "stages_ms": stage_ms, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+        "cuda_graph": graph is not None,
     }
     if decode:
         byt = sum(work[s]["bytes"] for s in work)
@@ -418,8 +450,12 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="decode: launch each step instead of replaying a CUDA graph")
     ap.add_argument("--single-cta", action="store_true",
-                    help="expert GEMMs on single CTAs (M=128) instead of CTA pairs (M=256)")
+                    help="force the single-CTA (M=128) expert GEMM engine")
+    ap.add_argument("--pair", action="store_true",
+                    help="force the CTA-pair (M=256) expert GEMM engine")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -81,9 +81,12 @@ typedef struct {
  * ws_down_f16, made once by moe_prepare_down_f16); without this flag
  * moe_forward converts them into the workspace on every call. */
 #define MOE_FLAG_DOWN_F16         4
-/* Run the expert GEMMs on single CTAs (M = 128 tiles) instead of CTA pairs
- * (clusters of two SMs, M = 256 tiles); same results, for comparison. */
+/* Engine of the expert GEMMs.  By default CTA pairs (clusters of two SMs,
+ * M = 256 tiles) are used when T * k >= 256 * E (the average expert fills a
+ * 256-row tile) and single CTAs (M = 128 tiles) otherwise; these flags force
+ * one of them.  Both give the same results. */
 #define MOE_FLAG_GEMM_SINGLE_CTA  8
+#define MOE_FLAG_GEMM_PAIR        16
 
 typedef struct {
     const void *w_router;      /* [E, d] bf16 */

@@ -58,11 +58,17 @@ __device__ __forceinline__ Item decode_item(const GemmParams &p, int item) {
   return it;
 }
 
+// Width, in logit units, of the ambiguous band at the k-th/(k+1)-th boundary
+// whose experts the select kernel re-decides on float64 logits (see
+// router_cc.cu); far above twice the fp32 logit error of either logit path.
+constexpr float kRefineBand = 2e-4f;
+
 // Router epilogue: each thread owns one token row and writes its E fp32
 // logits (bias added) as 16-byte vectors; selection happens in the
 // warp-per-token select kernel that follows.
-__device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item &it, uint32_t taddr,
-                                                int row_local, const float *bias_s) {
+__device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item &it,
+                                                       uint32_t taddr, int row_local,
+                                                       const float *bias_s) {
   const bool valid = row_local < it.nrows;
   float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E;
   for (int c = 0; c < p.E; c += 32) {

@@ -63,6 +63,7 @@ cudaError_t launch_gemm_pair(int mode, const GemmParams &p, const GemmMaps &m, i
 
 cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
                              float *logits, int T, int d, int E, cudaStream_t s);
+// Warp-per-token selection over the fp32 logits of every token.
 cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
                                  const float *bias, int T, int d, int E, int k, int norm_topk,
                                  int32_t *topk_idx, float *topk_w, cudaStream_t s);

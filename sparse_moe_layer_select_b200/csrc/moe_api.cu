@@ -210,6 +210,7 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     p.n_tile = D.E;
     p.bias = bias;
     p.logits_out = logits;
+
     const uint32_t a_rows = static_cast<uint32_t>(std::min(D.T, kBlockM));
     p.a_bytes = a_rows * kBlockK * 2;
     GemmMaps m;
@@ -222,11 +223,16 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     m.b1_sh = m.b0;
     const int grid = std::min(sms, p.n_tiles_host);
     if (launch_gemm(MODE_ROUTER, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
-  } else {
-    if (launch_router_cc(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(w_router),
-                         bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
+    if (launch_router_select(logits, static_cast<const uint16_t *>(x),
+                             static_cast<const uint16_t *>(w_router), bias, D.T, D.d, D.E, D.k,
+                             D.norm, topk_idx, topk_w, s) != cudaSuccess)
       return MOE_ERR_CUDA;
+    *launches += 2;
+    return MOE_OK;
   }
+  if (launch_router_cc(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(w_router),
+                       bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (launch_router_select(logits, static_cast<const uint16_t *>(x),
                            static_cast<const uint16_t *>(w_router), bias, D.T, D.d, D.E, D.k,
                            D.norm, topk_idx, topk_w, s) != cudaSuccess)
@@ -351,8 +357,14 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
                   sms, &launches);
   if (st != MOE_OK) return st;
   // 2. expert order + tile list (256-row tiles for the CTA-pair GEMMs)
+  // CTA pairs (M = 256 tiles) when the average expert fills a 256-row tile;
+  // below that, single-CTA M = 128 tiles waste less of the tensor core and
+  // were measured faster (weight-streaming shapes).
   const int pair_grid = 2 * std::min(pair_clusters(), sms / 2);  // all pairs co-resident
-  const bool pair = !(D.flags & MOE_FLAG_GEMM_SINGLE_CTA) && pair_grid >= 2;
+  bool pair = static_cast<int64_t>(D.T) * D.k >= static_cast<int64_t>(2 * kBlockM) * D.E;
+  if (D.flags & MOE_FLAG_GEMM_PAIR) pair = true;
+  if (D.flags & MOE_FLAG_GEMM_SINGLE_CTA) pair = false;
+  if (pair_grid < 2) pair = false;
   ev.mark();
   if (launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0,
                    reinterpret_cast<int *>(wsp(ws, L.chunk_hist)), tiles, header, routing->counts,

@@ -21,9 +21,12 @@
 
 #include <cfloat>
 
+#include "gemm_common.cuh"
 #include "kernels.h"
 
 namespace moe {
+
+using gemm::kRefineBand;
 
 namespace {
 
@@ -86,12 +89,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
 
 constexpr int kSelectWarps = 8;
 
-// Width of the ambiguous band around the k-th/(k+1)-th boundary, in logit
-// units.  It is far above twice the largest fp32 logit error of either logit
-// path at these widths (tensor-core accumulation up to 1.2e-5, CUDA-core FMA
-// below 4e-6), so every expert outside the band is on the right side of the
-// boundary, and the band is decided on float64 logits.
-constexpr float kRefineBand = 2e-4f;
+// kRefineBand (gemm_common.cuh): width of the ambiguous band around the
+// k-th/(k+1)-th boundary, in logit units.  It is far above twice the largest
+// fp32 logit error of either logit path at these widths (tensor-core
+// accumulation up to 1.2e-5, CUDA-core FMA below 4e-6), so every expert
+// outside the band is on the right side of the boundary, and the band is
+// decided on float64 logits.
 
 // float64 logits of up to four experts e[0..n) for one token: exact bf16
 // products, float64 sums (lane-strided, then a butterfly in fixed order), plus
@@ -133,18 +136,6 @@ __device__ __forceinline__ void logits_f64_x4(const uint16_t *__restrict__ x,
   }
 }
 
-__device__ __forceinline__ void warp_argmax(float &bv, int &be) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-    if (ov > bv || (ov == bv && oe < be)) {
-      bv = ov;
-      be = oe;
-    }
-  }
-}
-
 // (value, expert) order of the selection: larger logit first, equal logits
 // by lower expert id; NaN (empty slot) after everything.
 __device__ __forceinline__ bool sel_before(float va, int ea, float vb, int eb) {
@@ -159,15 +150,14 @@ __device__ __forceinline__ bool sel_before(float va, int ea, float vb, int eb) {
 // float64 logits.  Then sigmoid scores and post-top-k normalisation (Laguna
 // M.1/XS.2 Technical Report summary, Key claims, report §3.1; Laguna-M.1-base
 // spec sheet, Mixture of experts).
+
 template <int NPL>
-__global__ void __launch_bounds__(kSelectWarps * 32)
-    router_select_kernel(const float *__restrict__ logits, const uint16_t *__restrict__ x,
-                         const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
-                         int T, int d, int E, int k, int norm_topk,
-                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
-  const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
+__device__ __forceinline__ void select_token(int t, int lane, const float *__restrict__ logits,
+                                             const uint16_t *__restrict__ x,
+                                             const uint16_t *__restrict__ w_router,
+                                             const float *__restrict__ bias, int d, int E, int k,
+                                             int norm_topk, int32_t *__restrict__ topk_idx,
+                                             float *__restrict__ topk_w) {
   const float *row = logits + static_cast<size_t>(t) * E;
   const float kNaN = __int_as_float(0x7fc00000);
   float v[NPL];
@@ -289,6 +279,18 @@ __global__ void __launch_bounds__(kSelectWarps * 32)
   }
 }
 
+template <int NPL>
+__global__ void __launch_bounds__(kSelectWarps * 32)
+    router_select_kernel(const float *__restrict__ logits, const uint16_t *__restrict__ x,
+                         const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
+                         int T, int d, int E, int k, int norm_topk,
+                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
+  if (t < T)
+    select_token<NPL>(t, lane, logits, x, w_router, bias, d, E, k, norm_topk, topk_idx, topk_w);
+}
+
 }  // namespace
 
 cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
@@ -315,21 +317,15 @@ cudaError_t launch_router_select(const float *logits, const uint16_t *x, const u
   const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
   const int threads = kSelectWarps * 32;
   const int npl = (E + 31) / 32;
-  if (npl <= 1)
-    router_select_kernel<1><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
-                                                       norm_topk, topk_idx, topk_w);
-  else if (npl <= 2)
-    router_select_kernel<2><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
-                                                       norm_topk, topk_idx, topk_w);
-  else if (npl <= 4)
-    router_select_kernel<4><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
-                                                       norm_topk, topk_idx, topk_w);
-  else if (npl <= 8)
-    router_select_kernel<8><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
-                                                       norm_topk, topk_idx, topk_w);
-  else
-    router_select_kernel<16><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,
-                                                        norm_topk, topk_idx, topk_w);
+#define MOE_SELECT(N)                                                                          \
+  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,   \
+                                                     norm_topk, topk_idx, topk_w)
+  if (npl <= 1) MOE_SELECT(1);
+  else if (npl <= 2) MOE_SELECT(2);
+  else if (npl <= 4) MOE_SELECT(4);
+  else if (npl <= 8) MOE_SELECT(8);
+  else MOE_SELECT(16);
+#undef MOE_SELECT
   return cudaGetLastError();
 }
 

@@ -25,6 +25,7 @@ MOE_FLAG_ROUTER_CUDA_CORE = 1
 MOE_FLAG_ROUTER_TENSOR = 2
 MOE_FLAG_DOWN_F16 = 4
 MOE_FLAG_GEMM_SINGLE_CTA = 8
+MOE_FLAG_GEMM_PAIR = 16
 
 # Every symbol the header declares (checked by the CPU tests).
 EXPORTED = ["moe_workspace_size", "moe_route", "moe_permute", "moe_forward",

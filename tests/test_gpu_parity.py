@@ -76,7 +76,7 @@ def test_router_paths_match_oracle(flags, T):
     G.check_routing(idx.cpu().numpy(), wt.cpu().numpy(), ref, w.k)
 
 
-ENGINES = [0, M.MOE_FLAG_GEMM_SINGLE_CTA]  # CTA-pair (M = 256) and single-CTA (M = 128) GEMMs
+ENGINES = [M.MOE_FLAG_GEMM_PAIR, M.MOE_FLAG_GEMM_SINGLE_CTA]  # CTA-pair (M = 256), single CTA (M = 128)
 
 
 @pytest.mark.parametrize("engine", ENGINES)
