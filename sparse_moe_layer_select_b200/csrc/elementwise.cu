@@ -3,11 +3,11 @@
 //   gather_rows_kernel  x_perm[r, :] = x[perm[r] / k, :]   (materialised expert-order
 //                       activations; the forward pass fuses this gather into the GEMM
 //                       operand load instead)
-//   combine_kernel      y[t, :] = bf16( sum_j slot[t, j, :] ) in fp32 over the k routed
-//                       fp16 slots (already scaled by routed_scaling_factor * w_t,j)
-//                       and the shared-expert slot: the combine of the routed sum with
-//                       the always-on shared expert (Laguna M.1/XS.2 Technical Report
-//                       summary, Key claims, report §3.1)
+//   combine_kernel      y[t, :] = bf16( sum_j o[inv[t*k + j], :] + s[t, :] ) in fp32 over
+//                       the k routed fp16 rows (already scaled by routed_scaling_factor *
+//                       w_t,j, stored in expert order) and the shared-expert row: the
+//                       combine of the routed sum with the always-on shared expert
+//                       (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1)
 //   bf16_to_f16_kernel  fp16 copy of the down-projection weights (round to nearest
 //                       even; values beyond the fp16 range are reported)
 //   selftest_wait_kernel  a bounded wait on a flag nothing sets (timeout self-test)
@@ -36,18 +36,20 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// One thread per 8 output columns of one token: the k routed rows
+// o[inv[t*k + j]] (already scaled by routed_scaling_factor * w) are added in
+// slot order, then the shared-expert row, all in fp32; one RNE rounding to bf16.
 __global__ void __launch_bounds__(256)
-    combine_kernel(const uint4 *__restrict__ slots, int T, int nslots, int vec_per_row,
+    combine_kernel(const uint4 *__restrict__ o, const uint4 *__restrict__ s_out,
+                   const int32_t *__restrict__ inv, int T, int k, int vec_per_row,
                    uint4 *__restrict__ y) {
   const size_t total = static_cast<size_t>(T) * vec_per_row;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const size_t t = i / vec_per_row;
     const size_t c = i - t * vec_per_row;
-    const uint4 *src = slots + t * nslots * vec_per_row + c;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < nslots; ++j) {
-      const uint4 v = src[static_cast<size_t>(j) * vec_per_row];
+    auto add = [&](const uint4 v) {
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -55,14 +57,19 @@ __global__ void __launch_bounds__(256)
         acc[2 * q] += f.x;
         acc[2 * q + 1] += f.y;
       }
+    };
+    for (int j = 0; j < k; ++j) {
+      const int r = inv[t * k + j];
+      add(o[static_cast<size_t>(r) * vec_per_row + c]);
     }
-    uint32_t o[4];
+    if (s_out) add(s_out[t * vec_per_row + c]);
+    uint32_t out[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-      o[q] = *reinterpret_cast<uint32_t *>(&b);
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+      out[q] = *reinterpret_cast<uint32_t *>(&b2);
     }
-    y[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    y[i] = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 
@@ -129,12 +136,13 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_row
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const uint16_t *slots, int T, int nslots, int d, uint16_t *y,
-                           cudaStream_t s) {
+cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32_t *inv, int T,
+                           int k, int d, uint16_t *y, cudaStream_t s) {
   const int vpr = d / 8;
   const size_t work = static_cast<size_t>(T) * vpr;
-  combine_kernel<<<grid_for(work, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(slots), T,
-                                                     nslots, vpr, reinterpret_cast<uint4 *>(y));
+  combine_kernel<<<grid_for(work, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(o),
+                                                     reinterpret_cast<const uint4 *>(s_out), inv,
+                                                     T, k, vpr, reinterpret_cast<uint4 *>(y));
   return cudaGetLastError();
 }
 

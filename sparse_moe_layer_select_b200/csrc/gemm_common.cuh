@@ -93,81 +93,142 @@ __device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item 
   }
 }
 
-__device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item &it,
-                                                uint32_t taddr, int row_local) {
-  const bool shared = it.group == p.E;
-  const bool valid = row_local < it.nrows;
-  uint16_t *dst = shared ? p.h_shared + static_cast<size_t>(it.row0 + row_local) * p.Fs
-                         : p.h + static_cast<size_t>(it.row0 + row_local) * p.F;
-  dst += it.j * p.n_half;
-  for (int c = 0; c < p.n_half; c += 32) {
-    uint32_t g[32], u[32];
-    tmem_ld_32x32b_x32(taddr + c, g);
-    tmem_ld_32x32b_x32(taddr + p.n_half + c, u);
-    tmem_ld_wait();
-    uint32_t packed[16];
-    float amax = 0.f;
+// Output staging of one epilogue warp: two 4 KB buffers, each one box of 32
+// rows x 64 fp16 columns in the 128-byte-swizzled layout the store tensor
+// maps use.  A box whose 32 rows are all valid is written by one TMA store;
+// a partially valid box (the last rows of a tile) is written row by row, so
+// no store ever reaches rows past the tile.
+struct EpiStage {
+  uint8_t *buf;  // this warp's 8 KB, 1024-byte aligned
+  int cur;
+};
+
+constexpr int kEpiBytesPerWarp = 2 * 32 * 128;
+
+__device__ __forceinline__ void store_box(EpiStage &st, const uint32_t (&packed)[32], int lane,
+                                          bool full_box, bool row_valid, const CUtensorMap *tm,
+                                          int col, int box_row, uint16_t *row_dst) {
+  if (full_box) {
+    uint8_t *b = st.buf + st.cur * (32 * 128);
+    if (lane == 0) bulk_wait_read_le1();  // the store that last used this buffer has read it
+    __syncwarp();
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-      const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-      const float h0 = g0 / (1.f + __expf(-g0)) * u0;
-      const float h1 = g1 / (1.f + __expf(-g1)) * u1;
-      amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
-      packed[i] = pack_f16x2(h0, h1);
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint4 *>(b + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+          make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tm, b, col, box_row);
+      bulk_commit_group();
     }
-    if (valid && amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_H_FP16_RANGE);
-    if (valid) {
-      uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+    st.cur ^= 1;
+  } else if (row_valid) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(row_dst);
 #pragma unroll
-      for (int v = 0; v < 4; ++v)
-        d4[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-    }
+    for (int v = 0; v < 8; ++v)
+      d4[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
   }
 }
 
-__device__ __forceinline__ void slot_epilogue(const GemmParams &p, const Item &it, uint32_t taddr,
-                                              int row_local) {
+// silu(g) * u with a fast reciprocal (the result is rounded to fp16).
+__device__ __forceinline__ float swiglu(float g, float u) {
+  return __fdividef(g, 1.f + __expf(-g)) * u;
+}
+
+// GEMM1 epilogue: h = silu(gate) * up for this thread's row, fp16, 64
+// columns per store box.
+__device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item &it,
+                                                uint32_t taddr, int row_local, EpiStage &st,
+                                                const CUtensorMap *tm_h, const CUtensorMap *tm_hsh) {
   const bool shared = it.group == p.E;
+  const int q = row_local >> 5;
+  const int lane = row_local & 31;
   const bool valid = row_local < it.nrows;
-  float scale = 1.f;
-  size_t dst_row = 0;
-  if (valid) {
-    if (shared) {
-      const size_t t = static_cast<size_t>(it.row0 + row_local);
-      dst_row = t * p.slots + p.k;
-    } else {
-      const int pt = p.perm[it.row0 + row_local];
-      const int t = pt / p.k;
-      const int jslot = pt - t * p.k;
-      scale = p.routed_scale * p.topk_w[pt];
-      dst_row = static_cast<size_t>(t) * p.slots + jslot;
+  const bool full_box = (q + 1) * 32 <= it.nrows;
+  uint16_t *row_dst = shared ? p.h_shared + static_cast<size_t>(it.row0 + row_local) * p.Fs
+                             : p.h + static_cast<size_t>(it.row0 + row_local) * p.F;
+  const int col0 = it.j * p.n_half;
+  float amax = 0.f;
+  for (int cb = 0; cb < p.n_half; cb += 64) {
+    uint32_t packed[32];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t g[32], u[32];
+      tmem_ld_32x32b_x32(taddr + cb + 32 * half, g);
+      tmem_ld_32x32b_x32(taddr + p.n_half + cb + 32 * half, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float h0 = swiglu(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
+        const float h1 = swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
+        amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
+        packed[16 * half + i] = pack_f16x2(h0, h1);
+      }
     }
+    store_box(st, packed, lane, full_box, valid, shared ? tm_hsh : tm_h, col0 + cb,
+              it.row0 + q * 32, row_dst + col0 + cb);
   }
-  uint16_t *dst = p.slot_out + dst_row * p.d + static_cast<size_t>(it.j) * p.n_tile;
-  for (int c = 0; c < p.n_tile; c += 32) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(taddr + c, r);
-    tmem_ld_wait();
-    if (valid) {
-      uint32_t packed[16];
-      float amax = 0.f;
+  if (valid && amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_H_FP16_RANGE);
+}
+
+// GEMM2 epilogue: routed rows -> routed_scale * w * o into o_out (expert-order
+// rows); shared-expert rows -> o into s_out (token rows).  fp16, 64 columns
+// per store box.
+__device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &it, uint32_t taddr,
+                                              int row_local, EpiStage &st,
+                                              const CUtensorMap *tm_o, const CUtensorMap *tm_s) {
+  const bool shared = it.group == p.E;
+  const int q = row_local >> 5;
+  const int lane = row_local & 31;
+  const bool valid = row_local < it.nrows;
+  const bool full_box = (q + 1) * 32 <= it.nrows;
+  float scale = 1.f;
+  if (valid && !shared) scale = p.routed_scale * p.topk_w[p.perm[it.row0 + row_local]];
+  uint16_t *row_dst = (shared ? p.s_out : p.o_out) + static_cast<size_t>(it.row0 + row_local) * p.d;
+  const int col0 = it.j * p.n_tile;
+  float amax = 0.f;
+  for (int cb = 0; cb < p.n_tile; cb += 64) {
+    uint32_t packed[32];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(taddr + cb + 32 * half, r);
+      tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float v0 = __uint_as_float(r[2 * i]) * scale;
         const float v1 = __uint_as_float(r[2 * i + 1]) * scale;
         amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));
-        packed[i] = pack_f16x2(v0, v1);
+        packed[16 * half + i] = pack_f16x2(v0, v1);
       }
-      if (amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_SLOT_FP16_RANGE);
-      uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        d4[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
     }
+    store_box(st, packed, lane, full_box, valid, shared ? tm_s : tm_o, col0 + cb,
+              it.row0 + q * 32, row_dst + col0 + cb);
+  }
+  if (valid && amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_SLOT_FP16_RANGE);
+}
+
+// Row ids of one GEMM1 tile (this CTA's up to 128 rows): lane l reads rows
+// 4l..4l+3.  Issued early (during the previous item), converted to token ids
+// into a shared-memory table when the item starts.
+__device__ __forceinline__ void tile_rows_fetch(const GemmParams &p, const Item &it, int lane,
+                                                int (&v)[4]) {
+  const bool shared = it.group == p.E;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int r = 4 * lane + q;
+    v[q] = r < it.nrows ? (shared ? it.row0 + r : p.perm[it.row0 + r]) : -1;
   }
 }
 
+__device__ __forceinline__ void tile_tokens_store(const GemmParams &p, const Item &it, int lane,
+                                                  const int (&v)[4], int *tok_s) {
+  const bool shared = it.group == p.E;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tok_s[4 * lane + q] = v[q] < 0 ? -1 : (shared ? v[q] : v[q] / p.k);
+  __syncwarp();
+}
 
 // The part of an item that one CTA of a pair owns: rows [128 r, 128 r + 128).
 __device__ __forceinline__ Item pair_half(Item it, int rank) {

@@ -91,7 +91,8 @@ __device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk
 // Each warp places its 512 entries: fill[warp][e] holds its next row of e.
 __device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ topk_idx, int n,
                                                    int E, int chunk, int *fill,
-                                                   int32_t *__restrict__ perm) {
+                                                   int32_t *__restrict__ perm,
+                                                   int32_t *__restrict__ inv) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
@@ -107,7 +108,11 @@ __device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ t
     }
     const unsigned m = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(m & lt);
-    if (e >= 0) perm[fw[e] + rank] = i;
+    if (e >= 0) {
+      const int pos = fw[e] + rank;
+      perm[pos] = i;
+      if (inv) inv[i] = pos;  // expert-order row of entry i = t * k + j
+    }
     __syncwarp();
     if (e >= 0 && rank == 0) fw[e] += __popc(m);
     __syncwarp();
@@ -220,11 +225,12 @@ __global__ void __launch_bounds__(512)
 
 __global__ void __launch_bounds__(kIdxWarps * 32)
     index_scatter_kernel(const int32_t *__restrict__ topk_idx, int n, int E,
-                         const int *__restrict__ chunk_base, int32_t *__restrict__ perm) {
+                         const int *__restrict__ chunk_base, int32_t *__restrict__ perm,
+                         int32_t *__restrict__ inv) {
   __shared__ int h[kIdxWarps * kMaxE];
   chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, nullptr);
   warp_bases(E, chunk_base + static_cast<size_t>(blockIdx.x) * E, h);
-  chunk_warp_scatter(topk_idx, n, E, blockIdx.x, h, perm);
+  chunk_warp_scatter(topk_idx, n, E, blockIdx.x, h, perm, inv);
 }
 
 // All of the above for a single chunk (n <= kIndexChunk), in one CTA of 512
@@ -233,7 +239,8 @@ __global__ void __launch_bounds__(512)
     index_single_kernel(const int32_t *__restrict__ topk_idx, int n, int E, int T,
                         int with_shared, int tile_rows, int *__restrict__ chunk_hist,
                         int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                        int32_t *__restrict__ perm, Tile *__restrict__ tiles, int *header) {
+                        int32_t *__restrict__ perm, int32_t *__restrict__ inv,
+                        Tile *__restrict__ tiles, int *header) {
   __shared__ int h[kIdxWarps * kMaxE];
   __shared__ int warp_sums[32];
   __shared__ int totals[2];
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(512)
                  warp_sums, totals);
   __syncthreads();
   warp_bases(E, chunk_hist, h);
-  if (warp < kIdxWarps) chunk_warp_scatter(topk_idx, n, E, 0, h, perm);
+  if (warp < kIdxWarps) chunk_warp_scatter(topk_idx, n, E, 0, h, perm, inv);
 }
 
 }  // namespace
@@ -275,12 +282,12 @@ __global__ void __launch_bounds__(512)
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
                          int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
-                         int tile_rows) {
+                         int tile_rows, int32_t *inv) {
   const int n = T * k;
   const int nchunks = (n + kIndexChunk - 1) / kIndexChunk;
   if (nchunks == 1) {
     index_single_kernel<<<1, 512, 0, s>>>(topk_idx, n, E, T, with_shared, tile_rows, chunk_hist,
-                                          counts, offsets, perm, tiles, status);
+                                          counts, offsets, perm, inv, tiles, status);
     *launches += 1;
     return cudaGetLastError();
   }
@@ -291,7 +298,7 @@ cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_
                                       offsets, tiles, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  index_scatter_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm);
+  index_scatter_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm, inv);
   *launches += 3;
   return cudaGetLastError();
 }

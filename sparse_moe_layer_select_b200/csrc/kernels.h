@@ -35,7 +35,6 @@ struct GemmParams {
   int T, d, E, k, F, Fs;
   int n_half;               // GEMM1: gate (and up) columns per N tile
   int n_tile;               // MMA N of this launch
-  int slots;                // GEMM2: slots per token (k, plus one if shared)
   uint32_t a_bytes;         // bytes of one A stage (ROUTER, GEMM2 routed rows)
   uint32_t a_sh_bytes;      // bytes of one A stage for shared-expert rows (GEMM2)
   float routed_scale;       // GEMM2: routed_scaling_factor
@@ -46,11 +45,26 @@ struct GemmParams {
   float *logits_out;        // ROUTER out: [T, E] fp32 logits incl. bias
   uint16_t *h;              // GEMM1 out: [T*k, F] fp16 (expert-order rows)
   uint16_t *h_shared;       // GEMM1 out: [T, Fs] fp16
-  uint16_t *slot_out;       // GEMM2 out: [T, slots, d] fp16
+  uint16_t *o_out;          // GEMM2 out: [T*k, d] fp16, routed_scale * w * o (expert-order rows)
+  uint16_t *s_out;          // GEMM2 out: [T, d] fp16 shared-expert output
+  unsigned long long *trace;  // pipeline timestamps (builds with MOE_TRACE only), or null
+};
+
+// Pipeline trace layout (MOE_TRACE builds): trace[(cta * kTraceKinds + kind) * kTraceN + n].
+constexpr int kTraceKinds = 6;
+constexpr int kTraceN = 4096;
+enum TraceKind : int {
+  TR_ISSUE = 0,      // producer issued stage n (after its empty wait)
+  TR_LANDED = 1,     // this CTA's loads of stage n complete (pair relay)
+  TR_FULL = 2,       // MMA thread saw stage n full
+  TR_MMA = 3,        // MMAs of stage n issued
+  TR_EPI_START = 4,  // epilogue saw item n's accumulator
+  TR_EPI_END = 5,    // epilogue released item n's accumulator
 };
 
 struct GemmMaps {
   CUtensorMap a, b0, b1, a_sh, b0_sh, b1_sh;
+  CUtensorMap out, out_sh;  // epilogue TMA stores: 64 columns x 32 rows, 128-byte swizzle
 };
 
 size_t gemm_smem_bytes();
@@ -71,11 +85,12 @@ cudaError_t launch_router_select(const float *logits, const uint16_t *x, const u
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
                          int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
-                         int tile_rows = kBlockM);
+                         int tile_rows = kBlockM, int32_t *inv = nullptr);
 cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_rows, int k, int d,
                                uint16_t *x_perm, cudaStream_t s);
-cudaError_t launch_combine(const uint16_t *slots, int T, int nslots, int d, uint16_t *y,
-                           cudaStream_t s);
+// y[t] = bf16( sum_j o[inv[t*k + j]] + s_out[t] ), fp32 sums in slot order.
+cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32_t *inv, int T,
+                           int k, int d, uint16_t *y, cudaStream_t s);
 cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int *status,
                                cudaStream_t s);
 cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s);

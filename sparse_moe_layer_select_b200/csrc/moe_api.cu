@@ -25,6 +25,10 @@ namespace {
 using namespace moe;
 
 thread_local int32_t g_last_launches = 0;
+#ifdef MOE_TRACE
+unsigned long long *g_trace_gemm1 = nullptr;
+unsigned long long *g_trace_gemm2 = nullptr;
+#endif
 thread_local void **g_prof_events = nullptr;
 thread_local int32_t g_prof_n = 0;
 
@@ -106,12 +110,12 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uin
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Dims {
-  int T, d, E, k, F, Fs, slots, flags, norm;
+  int T, d, E, k, F, Fs, flags, norm;
   float scale;
 };
 
 struct WsLayout {
-  size_t header, chunk_hist, tiles, logits, h, h_sh, slots, down16, down16_sh, total;
+  size_t header, chunk_hist, tiles, logits, inv, h, h_sh, o, s_out, down16, down16_sh, total;
   int max_tiles;
 };
 
@@ -129,12 +133,16 @@ WsLayout ws_layout(const Dims &D) {
   off += align256(static_cast<size_t>(L.max_tiles) * sizeof(Tile));
   L.logits = off;
   off += align256(static_cast<size_t>(D.T) * D.E * 4);
+  L.inv = off;
+  off += align256(n * 4);
   L.h = off;
   off += align256(n * D.F * 2);
   L.h_sh = off;
   off += align256(static_cast<size_t>(D.T) * D.Fs * 2);
-  L.slots = off;
-  off += align256(static_cast<size_t>(D.T) * D.slots * D.d * 2);
+  L.o = off;  // routed contributions, expert-order rows
+  off += align256(n * D.d * 2);
+  L.s_out = off;  // shared-expert output, token rows
+  off += align256(D.Fs > 0 ? static_cast<size_t>(D.T) * D.d * 2 : 0);
   L.down16 = L.down16_sh = off;
   if (!(D.flags & MOE_FLAG_DOWN_F16)) {  // per-call fp16 copy of the down projections
     off += align256(static_cast<size_t>(D.E) * D.d * D.F * 2);
@@ -167,7 +175,6 @@ moe_status check_dims(const moe_dims_t *dims, Dims *D) {
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((dims->flags & MOE_FLAG_ROUTER_TENSOR) && (D->E % 16 != 0 || D->E > 256))
     return MOE_ERR_UNSUPPORTED_SHAPE;
-  D->slots = D->k + (D->Fs > 0 ? 1 : 0);
   return MOE_OK;
 }
 
@@ -347,7 +354,9 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   Tile *tiles = reinterpret_cast<Tile *>(wsp(ws, L.tiles));
   uint16_t *h = reinterpret_cast<uint16_t *>(wsp(ws, L.h));
   uint16_t *h_sh = reinterpret_cast<uint16_t *>(wsp(ws, L.h_sh));
-  uint16_t *slots = reinterpret_cast<uint16_t *>(wsp(ws, L.slots));
+  uint16_t *o_out = reinterpret_cast<uint16_t *>(wsp(ws, L.o));
+  uint16_t *s_out = D.Fs > 0 ? reinterpret_cast<uint16_t *>(wsp(ws, L.s_out)) : nullptr;
+  int32_t *inv = reinterpret_cast<int32_t *>(wsp(ws, L.inv));
   int launches = 0;
   EventMarker ev(s);
 
@@ -369,7 +378,7 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   if (launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0,
                    reinterpret_cast<int *>(wsp(ws, L.chunk_hist)), tiles, header, routing->counts,
                    routing->offsets, routing->perm, s, &launches,
-                   pair ? 2 * kBlockM : kBlockM) != cudaSuccess)
+                   pair ? 2 * kBlockM : kBlockM, inv) != cudaSuccess)
     return MOE_ERR_CUDA;
 
   // fp16 down projections: caller-prepared, or converted here every call
@@ -407,13 +416,13 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   base.k = D.k;
   base.F = D.F;
   base.Fs = D.Fs;
-  base.slots = D.slots;
   base.routed_scale = D.scale;
   base.perm = routing->perm;
   base.topk_w = routing->topk_w;
   base.h = h;
   base.h_shared = h_sh;
-  base.slot_out = slots;
+  base.o_out = o_out;
+  base.s_out = s_out;
 
   // 3. GEMM1: gathered x rows . [W_gate | W_up]^T -> SwiGLU -> h (bf16)
   {
@@ -422,6 +431,9 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     p.n_tile = 2 * n_half;
     p.n_ntiles = std::max(D.F, D.Fs) / n_half;
     p.x = static_cast<const uint16_t *>(x);
+#ifdef MOE_TRACE
+    p.trace = g_trace_gemm1;
+#endif
     p.a_bytes = kBlockM * kBlockK * 2;
     p.a_sh_bytes = p.a_bytes;
     GemmMaps m;
@@ -430,12 +442,16 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     if (!make_map(&m.b0, w->w_gate, static_cast<uint64_t>(D.E) * D.F, D.d, n_half)) return MOE_ERR_CUDA;
     if (!make_map(&m.b1, w->w_up, static_cast<uint64_t>(D.E) * D.F, D.d, n_half)) return MOE_ERR_CUDA;
     m.a_sh = m.a;
+    const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&m.out, h, n_rows, D.F, std::min(32, n_rows), f16)) return MOE_ERR_CUDA;
     if (D.Fs > 0) {
       if (!make_map(&m.b0_sh, w->ws_gate, D.Fs, D.d, n_half)) return MOE_ERR_CUDA;
       if (!make_map(&m.b1_sh, w->ws_up, D.Fs, D.d, n_half)) return MOE_ERR_CUDA;
+      if (!make_map(&m.out_sh, h_sh, D.T, D.Fs, std::min(32, D.T), f16)) return MOE_ERR_CUDA;
     } else {
       m.b0_sh = m.b0;
       m.b1_sh = m.b1;
+      m.out_sh = m.out;
     }
     ev.mark();
     const cudaError_t e = pair ? launch_gemm_pair(MODE_GEMM1, p, m, pair_grid, s)
@@ -443,11 +459,14 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
   }
-  // 4. GEMM2: h . W_down^T -> x (routed_scaling_factor * w) -> slot rows
+  // 4. GEMM2: h . W_down^T -> x (routed_scaling_factor * w) -> expert-order rows
   {
     GemmParams p = base;
     p.n_tile = n2;
     p.n_ntiles = D.d / n2;
+#ifdef MOE_TRACE
+    p.trace = g_trace_gemm2;
+#endif
     const uint32_t a_rows = static_cast<uint32_t>(std::min(n_rows, kBlockM));
     const uint32_t a_sh_rows = static_cast<uint32_t>(std::min(D.T, kBlockM));
     p.a_bytes = a_rows * kBlockK * 2;
@@ -460,9 +479,12 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     if (!make_map(&m.b0, wd16, static_cast<uint64_t>(D.E) * D.d, D.F, b_rows, f16))
       return MOE_ERR_CUDA;
     m.b1 = m.b0;
+    if (!make_map(&m.out, o_out, n_rows, D.d, std::min(32, n_rows), f16)) return MOE_ERR_CUDA;
+    m.out_sh = m.out;
     if (D.Fs > 0) {
       if (!make_map(&m.a_sh, h_sh, D.T, D.Fs, a_sh_rows, f16)) return MOE_ERR_CUDA;
       if (!make_map(&m.b0_sh, wsd16, D.d, D.Fs, b_rows, f16)) return MOE_ERR_CUDA;
+      if (!make_map(&m.out_sh, s_out, D.T, D.d, std::min(32, D.T), f16)) return MOE_ERR_CUDA;
     } else {
       m.a_sh = m.a;
       m.b0_sh = m.b0;
@@ -474,9 +496,10 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
   }
-  // 5. combine: y = bf16(sum of the scaled routed slots + shared slot)
+  // 5. combine: y = bf16(sum of the scaled routed rows + shared row)
   ev.mark();
-  if (launch_combine(slots, D.T, D.slots, D.d, static_cast<uint16_t *>(y), s) != cudaSuccess)
+  if (launch_combine(o_out, s_out, inv, D.T, D.k, D.d, static_cast<uint16_t *>(y), s) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   launches += 1;
   ev.mark();
@@ -562,6 +585,15 @@ const char *moe_status_string(moe_status s) {
 }
 
 int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+#ifdef MOE_TRACE
+// Trace builds only: device buffers receiving the pipeline timestamps of the
+// next forward calls' GEMMs (layout in kernels.h).
+void moe_debug_set_trace(void *gemm1, void *gemm2) {
+  g_trace_gemm1 = static_cast<unsigned long long *>(gemm1);
+  g_trace_gemm2 = static_cast<unsigned long long *>(gemm2);
+}
+#endif
 
 moe_status moe_profile_next_forward(void **events, int32_t n_events) {
   if (events != nullptr && n_events < 1) return MOE_ERR_INVALID_ARG;

@@ -56,13 +56,16 @@ constexpr int kAccStride = 256;
 struct SmemLayout {
   static constexpr int a_off = 0;
   static constexpr int b_off = a_off + kStages * kABytes;
-  static constexpr int bar_off = b_off + kStages * kBBytesMax;
+  // epilogue output staging (4 warps x 8 KB); the router's bias table reuses it
+  static constexpr int epi_off = b_off + kStages * kBBytesMax;
+  static constexpr int bias_off = epi_off;
+  static constexpr int bar_off = epi_off + 4 * kEpiBytesPerWarp;
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
   static constexpr int n_bars = 2 * kStages + 5;
   static constexpr int tmem_slot_off = bar_off + n_bars * 8;
-  static constexpr int bias_off = (tmem_slot_off + 16 + 15) / 16 * 16;
-  static constexpr int total = bias_off + 512 * 4;
+  static constexpr int total = tmem_slot_off + 16;
 };
+static_assert(SmemLayout::total + 1024 <= 232448, "shared memory budget");
 
 }  // namespace
 
@@ -73,7 +76,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const __grid_constant__ CUtensorMap tm_b1,
                     const __grid_constant__ CUtensorMap tm_a_sh,
                     const __grid_constant__ CUtensorMap tm_b0_sh,
-                    const __grid_constant__ CUtensorMap tm_b1_sh) {
+                    const __grid_constant__ CUtensorMap tm_b1_sh,
+                    const __grid_constant__ CUtensorMap tm_out,
+                    const __grid_constant__ CUtensorMap tm_out_sh) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -171,6 +176,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ok = false;
           break;
         }
+        if (lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
         uint8_t *a_dst = sA + s * kABytes;
         uint8_t *b_dst = sB + s * kBBytesMax;
         const int kc = kb * kBlockK;
@@ -225,6 +231,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t aph = 0;
       bool ok = true;
+      int consumed = 0;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         const Item it = decode_item<MODE>(p, item);
         if (it.skip) continue;
@@ -237,6 +244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
+          MOE_TRACE_AT(p, TR_FULL, consumed);
           if (MODE == MODE_GEMM1) fence_proxy_async_smem();  // A was written by cp.async
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kABytes);
@@ -247,6 +255,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                          idesc, (kb | kk) != 0);
           }
           umma_commit(&empty[s]);
+          MOE_TRACE_AT(p, TR_MMA, consumed);
+          ++consumed;
           if (++s == kStages) {
             s = 0;
             ph ^= 1;
@@ -268,29 +278,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row_local = q * 32 + lane;
+    EpiStage st{smem + SmemLayout::epi_off + (warp - 2) * kEpiBytesPerWarp, 0};
     int acc = 0;
     uint32_t aph = 0;
+    int done = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item it = decode_item<MODE>(p, item);
       if (it.skip) continue;
       if (status_is_set(status)) break;
       if (!mbar_wait(&acc_full[acc], aph, status, SITE_GEMM_EPI_ACC_FULL)) break;
+      if (warp == 2 && lane == 0) MOE_TRACE_AT(p, TR_EPI_START, done);
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccStride;
       if (MODE == MODE_ROUTER) {
         router_epilogue(p, it, taddr, row_local, bias_s);
       } else if (MODE == MODE_GEMM1) {
-        swiglu_epilogue(p, it, taddr, row_local);
+        swiglu_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       } else {
-        slot_epilogue(p, it, taddr, row_local);
+        down_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
+      if (warp == 2 && lane == 0) MOE_TRACE_AT(p, TR_EPI_END, done);
+      ++done;
       if (++acc == 2) {
         acc = 0;
         aph ^= 1;
       }
     }
+    if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
   }
 
   tc_fence_before();
@@ -316,13 +332,13 @@ cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int gr
   switch (mode) {
     case MODE_ROUTER:
       return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_ROUTER>, p, m.a, m.b0, m.b1, m.a_sh,
-                                m.b0_sh, m.b1_sh);
+                                m.b0_sh, m.b1_sh, m.out, m.out_sh);
     case MODE_GEMM1:
       return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM1>, p, m.a, m.b0, m.b1, m.a_sh,
-                                m.b0_sh, m.b1_sh);
+                                m.b0_sh, m.b1_sh, m.out, m.out_sh);
     default:
       return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM2>, p, m.a, m.b0, m.b1, m.a_sh,
-                                m.b0_sh, m.b1_sh);
+                                m.b0_sh, m.b1_sh, m.out, m.out_sh);
   }
 }
 

@@ -45,12 +45,14 @@ constexpr int kPAccStride = 256;
 struct PairSmem {
   static constexpr int a_off = 0;
   static constexpr int b_off = a_off + kPairStages * kPABytes;
-  static constexpr int bar_off = b_off + kPairStages * kPBBytes;
+  static constexpr int epi_off = b_off + kPairStages * kPBBytes;  // 4 warps x 8 KB staging
+  static constexpr int bar_off = epi_off + 4 * kEpiBytesPerWarp;
   // full[S], lfull[S], empty[S], acc_full[2], acc_empty[2], drain
   static constexpr int n_bars = 3 * kPairStages + 5;
   static constexpr int tmem_slot_off = bar_off + n_bars * 8;
   static constexpr int total = tmem_slot_off + 16;
 };
+static_assert(PairSmem::total + 1024 <= 232448, "shared memory budget");
 
 }  // namespace
 
@@ -62,7 +64,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                          const __grid_constant__ CUtensorMap tm_b1,
                          const __grid_constant__ CUtensorMap tm_a_sh,
                          const __grid_constant__ CUtensorMap tm_b0_sh,
-                         const __grid_constant__ CUtensorMap tm_b1_sh) {
+                         const __grid_constant__ CUtensorMap tm_b1_sh,
+                         const __grid_constant__ CUtensorMap tm_out,
+                         const __grid_constant__ CUtensorMap tm_out_sh) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -152,6 +156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           ok = false;
           break;
         }
+        if (lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
         uint8_t *a_dst = sA + s * kPABytes;
         uint8_t *b_dst = sB + s * kPBBytes;
         const int kc = kb * kBlockK;
@@ -199,6 +204,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      int relayed = 0;
       for (int item = cluster_id; item < n_items && ok; item += n_clusters) {
         const Item whole = decode_item<MODE>(p, item);
         if (whole.skip) continue;
@@ -208,6 +214,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ok = false;
             break;
           }
+          MOE_TRACE_AT(p, TR_LANDED, relayed);
+          ++relayed;
           if (MODE == MODE_GEMM1) fence_proxy_async_smem();  // rows written by cp.async
           mbar_arrive_cluster(leader_full0 + s * 8);
           if (++s == kPairStages) {
@@ -228,6 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       int acc = 0;
       uint32_t aph = 0;
       bool ok = true;
+      int consumed = 0;
       for (int item = cluster_id; item < n_items && ok; item += n_clusters) {
         const Item it = decode_item<MODE>(p, item);
         if (it.skip) continue;
@@ -240,6 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ok = false;
             break;
           }
+          MOE_TRACE_AT(p, TR_FULL, consumed);
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kPABytes);
           const uint32_t b0 = smem_u32(sB + s * kPBBytes);
@@ -248,6 +258,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             umma_f16_ss_pair(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
                              idesc, (kb | kk) != 0);
           umma_commit_pair_multicast(&empty[s], 0x3);
+          MOE_TRACE_AT(p, TR_MMA, consumed);
+          ++consumed;
           if (++s == kPairStages) {
             s = 0;
             ph ^= 1;
@@ -269,26 +281,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
     const uint32_t leader_acc_empty0 = map_shared_rank(smem_u32(&acc_empty[0]), 0);
+    EpiStage st{smem + PairSmem::epi_off + (warp - 2) * kEpiBytesPerWarp, 0};
     int acc = 0;
     uint32_t aph = 0;
+    int done = 0;
     for (int item = cluster_id; item < n_items; item += n_clusters) {
       const Item whole = decode_item<MODE>(p, item);
       if (whole.skip) continue;
       if (status_is_set(status)) break;
       if (!mbar_wait(&acc_full[acc], aph, status, SITE_GEMM_EPI_ACC_FULL)) break;
+      if (warp == 2 && lane == 0) MOE_TRACE_AT(p, TR_EPI_START, done);
       tc_fence_after();
       const Item it = pair_half(whole, rank);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kPAccStride;
-      if (MODE == MODE_GEMM1) swiglu_epilogue(p, it, taddr, row_local);
-      else slot_epilogue(p, it, taddr, row_local);
+      if (MODE == MODE_GEMM1) swiglu_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+      else down_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + acc * 8);
+      if (warp == 2 && lane == 0) MOE_TRACE_AT(p, TR_EPI_END, done);
+      ++done;
       if (++acc == 2) {
         acc = 0;
         aph ^= 1;
       }
     }
+    if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
   }
 
   tc_fence_before();
@@ -311,9 +329,9 @@ cudaError_t launch_gemm_pair(int mode, const GemmParams &p, const GemmMaps &m, i
   cfg.stream = s;
   if (mode == MODE_GEMM1)
     return cudaLaunchKernelEx(&cfg, moe_gemm_pair_kernel<MODE_GEMM1>, p, m.a, m.b0, m.b1, m.a_sh,
-                              m.b0_sh, m.b1_sh);
+                              m.b0_sh, m.b1_sh, m.out, m.out_sh);
   return cudaLaunchKernelEx(&cfg, moe_gemm_pair_kernel<MODE_GEMM2>, p, m.a, m.b0, m.b1, m.a_sh,
-                            m.b0_sh, m.b1_sh);
+                            m.b0_sh, m.b1_sh, m.out, m.out_sh);
 }
 
 cudaError_t gemm_pair_set_attributes() {

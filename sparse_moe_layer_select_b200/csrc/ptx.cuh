@@ -84,6 +84,30 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
       : "memory");
 }
 
+// 2-D tiled store of a shared-memory box to global memory at (c0, c1), in a
+// bulk async-group of this thread.
+__device__ __forceinline__ void tma_store_2d(const void *tmap, const void *smem_src, int32_t c0,
+                                             int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most one of this thread's bulk groups still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Wait until all of this thread's bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Row gather: four rows (r0..r3) of one column box, written as four
 // consecutive box rows.  The tensor map's box is one row high.
 __device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, uint64_t *bar,
@@ -282,6 +306,25 @@ __device__ __forceinline__ void umma_commit_pair_multicast(uint64_t *bar, uint16
       "h"(mask)
       : "memory");
 }
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+#ifdef MOE_TRACE
+#define MOE_TRACE_AT(p, kind, n)                                                             \
+  do {                                                                                        \
+    if ((p).trace != nullptr && (n) < kTraceN)                                                \
+      (p).trace[(static_cast<size_t>(blockIdx.x) * kTraceKinds + (kind)) * kTraceN + (n)] =  \
+          global_timer_ns();                                                                  \
+  } while (0)
+#else
+#define MOE_TRACE_AT(p, kind, n) \
+  do {                           \
+  } while (0)
+#endif
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
