@@ -28,8 +28,17 @@ struct Item {
   bool skip;   // no work (N tile beyond this group's width)
 };
 
+// The tile record an item reads (zero for router items and past the end).
+// Roles load the record of their next item one item ahead, so that the gap
+// between two items holds no global-load round trip.
 template <int MODE>
-__device__ __forceinline__ Item decode_item(const GemmParams &p, int item) {
+__device__ __forceinline__ int4 load_tile_rec(const GemmParams &p, int item, int n_items) {
+  if (MODE == MODE_ROUTER || item >= n_items) return make_int4(0, 0, 0, 0);
+  return *reinterpret_cast<const int4 *>(&p.tiles[item / p.n_ntiles]);
+}
+
+template <int MODE>
+__device__ __forceinline__ Item decode_tile(const GemmParams &p, int item, int4 t) {
   Item it;
   if (MODE == MODE_ROUTER) {
     it.group = -1;
@@ -42,7 +51,6 @@ __device__ __forceinline__ Item decode_item(const GemmParams &p, int item) {
   }
   const int ti = item / p.n_ntiles;
   it.j = item - ti * p.n_ntiles;
-  const int4 t = *reinterpret_cast<const int4 *>(&p.tiles[ti]);
   it.group = t.x;
   it.row0 = t.y;
   it.nrows = t.z;
@@ -56,6 +64,111 @@ __device__ __forceinline__ Item decode_item(const GemmParams &p, int item) {
     it.nk = (shared ? p.Fs : p.F) / kBlockK;
   }
   return it;
+}
+
+// Walks one role's items (item, item + step, ...) with a one-item look-ahead:
+// current() decodes the role's next non-empty item from the tile record that
+// was loaded while the previous item ran; prefetch() starts the loads of the
+// record (and the status word) for the item after it; next() steps on.  A
+// status word raised by any role is seen at most one item late (every wait
+// in the pipeline is bounded on its own).
+template <int MODE>
+struct ItemWalk {
+  int item, step, n_items;
+  int4 rec;
+  int stop;
+
+  __device__ __forceinline__ ItemWalk(const GemmParams &p, int first, int step_, int n)
+      : item(first), step(step_), n_items(n), stop(0) {
+    rec = load_tile_rec<MODE>(p, item, n_items);
+  }
+  // false when this role has no item left (or an error was raised).
+  __device__ __forceinline__ bool current(const GemmParams &p, Item &it) {
+    for (;;) {
+      if (item >= n_items || stop) return false;
+      it = decode_tile<MODE>(p, item, rec);
+      if (!it.skip) return true;
+      item += step;
+      rec = load_tile_rec<MODE>(p, item, n_items);
+    }
+  }
+  // Issue the loads for the item after the current one (results consumed by
+  // the next current()).
+  __device__ __forceinline__ void prefetch(const GemmParams &p) {
+    rec = load_tile_rec<MODE>(p, item + step, n_items);
+    stop = *reinterpret_cast<const volatile int *>(p.status);
+  }
+  __device__ __forceinline__ void next() { item += step; }
+};
+
+// A 128-row GEMM1 operand part is gathered by kGatherWarps warps, each
+// copying kGatherRows consecutive rows with 16-byte cp.async (one warp
+// instruction moves 4 whole 128-byte rows).  One warp issues such copies at
+// about one instruction per 15 ns, slower than the tensor cores consume a
+// stage, so the rows are split across warps on all four SM sub-partitions.
+// (TMA tile::gather4 moves the same 4 rows per instruction; measured in
+// place of, and beside, cp.async it was slower: one, the other or any split
+// of the rows between them took 2.34 to 2.99 ms for the gate/up GEMM of the
+// skewed T=32768 prefill with one gathering warp.)
+#ifndef MOE_GATHER_WARPS
+#define MOE_GATHER_WARPS 8
+#endif
+// Whether the TMA-issuing warp also gathers a share (1) or only issues TMA (0).
+#ifndef MOE_TMA_WARP_GATHERS
+#define MOE_TMA_WARP_GATHERS 0
+#endif
+constexpr int kGatherWarps = MOE_GATHER_WARPS;
+constexpr bool kTmaWarpGathers = MOE_TMA_WARP_GATHERS != 0;
+constexpr int kExtraGatherWarps = kGatherWarps - (kTmaWarpGathers ? 1 : 0);
+constexpr int kGatherRows = kBlockM / kGatherWarps;
+constexpr int kGatherGroups = kGatherRows / 4;  // cp.async instructions per lane per stage
+static_assert(kBlockM % (4 * kGatherWarps) == 0 && kExtraGatherWarps >= 0, "gather split");
+
+// Row ids (expert-order row -> token * k + slot, or the token itself for a
+// shared-expert tile) of the rows lane `lane` of gather warp gw copies:
+// rows gw * kGatherRows + (lane >> 3) + 4 i, i < kGatherGroups; -1 past the
+// valid rows.  Issued during the previous item (plain loads whose results
+// are first used when the item starts), so that no load, shuffle or
+// shared-memory access sits between two items: on a gathering warp those
+// would queue behind the in-flight copy instructions.
+__device__ __forceinline__ void gather_rows_fetch(const GemmParams &p, const Item &it, int lane,
+                                                  int gw, int (&raw)[kGatherGroups]) {
+  const bool shared = it.group == p.E;
+#pragma unroll
+  for (int i = 0; i < kGatherGroups; ++i) {
+    const int r = gw * kGatherRows + (lane >> 3) + 4 * i;
+    raw[i] = r < it.nrows ? (shared ? it.row0 + r : p.perm[it.row0 + r]) : -1;
+  }
+}
+
+// Token ids from row ids (arithmetic only).
+__device__ __forceinline__ void gather_tokens(const GemmParams &p, const Item &it,
+                                              const int (&raw)[kGatherGroups],
+                                              int (&tok)[kGatherGroups]) {
+  const bool shared = it.group == p.E;
+#pragma unroll
+  for (int i = 0; i < kGatherGroups; ++i)
+    tok[i] = (raw[i] < 0 || shared) ? raw[i] : raw[i] / p.k;
+}
+
+// Issue this warp's share of one stage's A gather (GEMM1): the k-block
+// starting at column kc, into the 128B-swizzled A buffer at a_dst; the
+// lanes' completions arrive on bar (one arrival per lane).
+__device__ __forceinline__ void gather_a_stage(const GemmParams &p, const int (&tok)[kGatherGroups],
+                                               int lane, int gw, uint8_t *a_dst, uint64_t *bar,
+                                               int kc) {
+  // 128-byte swizzle: chunk c of row r sits at chunk (c ^ (r & 7)).
+  const int c = lane & 7;
+  const uint32_t a_base = smem_u32(a_dst);
+  const char *xsrc = reinterpret_cast<const char *>(p.x) + kc * 2 + c * 16;
+#pragma unroll
+  for (int i = 0; i < kGatherGroups; ++i) {
+    const int r = gw * kGatherRows + (lane >> 3) + 4 * i;
+    if (tok[i] >= 0)
+      cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4),
+                  xsrc + static_cast<size_t>(tok[i]) * p.d * 2);
+  }
+  cp_async_arrive_noinc(bar);
 }
 
 // Width, in logit units, of the ambiguous band at the k-th/(k+1)-th boundary
@@ -207,27 +320,6 @@ __device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &i
               it.row0 + q * 32, row_dst + col0 + cb);
   }
   if (valid && amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_SLOT_FP16_RANGE);
-}
-
-// Row ids of one GEMM1 tile (this CTA's up to 128 rows): lane l reads rows
-// 4l..4l+3.  Issued early (during the previous item), converted to token ids
-// into a shared-memory table when the item starts.
-__device__ __forceinline__ void tile_rows_fetch(const GemmParams &p, const Item &it, int lane,
-                                                int (&v)[4]) {
-  const bool shared = it.group == p.E;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int r = 4 * lane + q;
-    v[q] = r < it.nrows ? (shared ? it.row0 + r : p.perm[it.row0 + r]) : -1;
-  }
-}
-
-__device__ __forceinline__ void tile_tokens_store(const GemmParams &p, const Item &it, int lane,
-                                                  const int (&v)[4], int *tok_s) {
-  const bool shared = it.group == p.E;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) tok_s[4 * lane + q] = v[q] < 0 ? -1 : (shared ? v[q] : v[q] / p.k);
-  __syncwarp();
 }
 
 // The part of an item that one CTA of a pair owns: rows [128 r, 128 r + 128).

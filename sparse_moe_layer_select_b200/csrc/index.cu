@@ -147,14 +147,44 @@ __global__ void __launch_bounds__(kIdxWarps * 32)
   }
 }
 
+// One tile list: blocks of at most tile_rows rows of each expert in expert
+// order, then the shared-expert blocks (token rows); returns the count.
+__device__ __forceinline__ int write_tiles(int e, int cnt, int off, int E, int T, int with_shared,
+                                           int tile_rows, Tile *__restrict__ tiles,
+                                           int *warp_sums, int *total) {
+  const int ntile = e < E ? (cnt + tile_rows - 1) / tile_rows : 0;
+  const int toff = block_exclusive_scan(ntile, warp_sums, total);
+  for (int i = 0; i < ntile; ++i) {
+    Tile t;
+    t.group = e;
+    t.row0 = off + i * tile_rows;
+    t.nrows = min(tile_rows, cnt - i * tile_rows);
+    t.pad = 0;
+    tiles[toff + i] = t;
+  }
+  const int nshared = with_shared ? (T + tile_rows - 1) / tile_rows : 0;
+  for (int i = threadIdx.x; i < nshared; i += blockDim.x) {
+    Tile t;
+    t.group = E;
+    t.row0 = i * tile_rows;
+    t.nrows = min(tile_rows, T - i * tile_rows);
+    t.pad = 0;
+    tiles[*total + i] = t;
+  }
+  return *total + nshared;
+}
+
 // Expert sums over chunks, exclusive scan over experts, chunk bases and the
-// tile list.  One CTA of 512 threads (one thread per expert).
+// tile lists (128-row tiles; 256-row tiles too when tiles_pair is given).
+// One CTA of 512 threads (one thread per expert).
 __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int nchunks, int E,
-                                               int T, int with_shared, int tile_rows,
+                                               int T, int with_shared,
                                                int32_t *__restrict__ counts,
                                                int32_t *__restrict__ offsets,
-                                               Tile *__restrict__ tiles, int *__restrict__ header,
-                                               int *warp_sums, int *totals) {
+                                               Tile *__restrict__ tiles,
+                                               Tile *__restrict__ tiles_pair,
+                                               int *__restrict__ header, int *warp_sums,
+                                               int *totals) {
   const int e = threadIdx.x;
   int cnt = 0;
   if (e < E) {
@@ -169,8 +199,6 @@ __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int
     for (; c < nchunks; ++c) cnt += chunk_hist[static_cast<size_t>(c) * E + e];
   }
   const int off = block_exclusive_scan(e < E ? cnt : 0, warp_sums, &totals[0]);
-  const int ntile = e < E ? (cnt + tile_rows - 1) / tile_rows : 0;
-  const int toff = block_exclusive_scan(ntile, warp_sums, &totals[1]);
   if (e < E) {
     counts[e] = cnt;
     offsets[e] = off;
@@ -191,35 +219,27 @@ __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int
       chunk_hist[static_cast<size_t>(c) * E + e] = run;
       run += v;
     }
-    for (int i = 0; i < ntile; ++i) {
-      Tile t;
-      t.group = e;
-      t.row0 = off + i * tile_rows;
-      t.nrows = min(tile_rows, cnt - i * tile_rows);
-      t.pad = 0;
-      tiles[toff + i] = t;
-    }
   }
   if (e == 0) offsets[E] = totals[0];
-  const int nshared = with_shared ? (T + tile_rows - 1) / tile_rows : 0;
-  for (int i = threadIdx.x; i < nshared; i += blockDim.x) {
-    Tile t;
-    t.group = E;
-    t.row0 = i * tile_rows;
-    t.nrows = min(tile_rows, T - i * tile_rows);
-    t.pad = 0;
-    tiles[totals[1] + i] = t;
+  const int n1 = write_tiles(e, cnt, off, E, T, with_shared, kBlockM, tiles, warp_sums, &totals[1]);
+  int n2 = 0;
+  if (tiles_pair != nullptr)
+    n2 = write_tiles(e, cnt, off, E, T, with_shared, 2 * kBlockM, tiles_pair, warp_sums,
+                     &totals[2]);
+  if (threadIdx.x == 0 && header) {
+    reinterpret_cast<WsHeader *>(header)->n_tiles = n1;
+    reinterpret_cast<WsHeader *>(header)->n_tiles_pair = n2;
   }
-  if (threadIdx.x == 0 && header) reinterpret_cast<WsHeader *>(header)->n_tiles = totals[1] + nshared;
 }
 
 __global__ void __launch_bounds__(512)
     index_scan_kernel(int *__restrict__ chunk_hist, int nchunks, int E, int T, int with_shared,
-                      int tile_rows, int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                      Tile *__restrict__ tiles, int *__restrict__ header) {
+                      int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                      Tile *__restrict__ tiles, Tile *__restrict__ tiles_pair,
+                      int *__restrict__ header) {
   __shared__ int warp_sums[32];
-  __shared__ int totals[2];
-  scan_and_tiles(chunk_hist, nchunks, E, T, with_shared, tile_rows, counts, offsets, tiles,
+  __shared__ int totals[3];
+  scan_and_tiles(chunk_hist, nchunks, E, T, with_shared, counts, offsets, tiles, tiles_pair,
                  header, warp_sums, totals);
 }
 
@@ -237,13 +257,13 @@ __global__ void __launch_bounds__(kIdxWarps * 32)
 // threads: warps 0..7 do the histogram and scatter, all 16 the scan.
 __global__ void __launch_bounds__(512)
     index_single_kernel(const int32_t *__restrict__ topk_idx, int n, int E, int T,
-                        int with_shared, int tile_rows, int *__restrict__ chunk_hist,
+                        int with_shared, int *__restrict__ chunk_hist,
                         int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                         int32_t *__restrict__ perm, int32_t *__restrict__ inv,
-                        Tile *__restrict__ tiles, int *header) {
+                        Tile *__restrict__ tiles, Tile *__restrict__ tiles_pair, int *header) {
   __shared__ int h[kIdxWarps * kMaxE];
   __shared__ int warp_sums[32];
-  __shared__ int totals[2];
+  __shared__ int totals[3];
   const int warp = threadIdx.x >> 5;
   // histogram by the first eight warps (the others only clear and wait)
   for (int i = threadIdx.x; i < kIdxWarps * E; i += blockDim.x) h[i] = 0;
@@ -270,7 +290,7 @@ __global__ void __launch_bounds__(512)
     chunk_hist[e] = s;
   }
   __syncthreads();
-  scan_and_tiles(chunk_hist, 1, E, T, with_shared, tile_rows, counts, offsets, tiles, header,
+  scan_and_tiles(chunk_hist, 1, E, T, with_shared, counts, offsets, tiles, tiles_pair, header,
                  warp_sums, totals);
   __syncthreads();
   warp_bases(E, chunk_hist, h);
@@ -282,20 +302,20 @@ __global__ void __launch_bounds__(512)
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
                          int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
-                         int tile_rows, int32_t *inv) {
+                         Tile *tiles_pair, int32_t *inv) {
   const int n = T * k;
   const int nchunks = (n + kIndexChunk - 1) / kIndexChunk;
   if (nchunks == 1) {
-    index_single_kernel<<<1, 512, 0, s>>>(topk_idx, n, E, T, with_shared, tile_rows, chunk_hist,
-                                          counts, offsets, perm, inv, tiles, status);
+    index_single_kernel<<<1, 512, 0, s>>>(topk_idx, n, E, T, with_shared, chunk_hist, counts,
+                                          offsets, perm, inv, tiles, tiles_pair, status);
     *launches += 1;
     return cudaGetLastError();
   }
   index_hist_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  index_scan_kernel<<<1, 512, 0, s>>>(chunk_hist, nchunks, E, T, with_shared, tile_rows, counts,
-                                      offsets, tiles, status);
+  index_scan_kernel<<<1, 512, 0, s>>>(chunk_hist, nchunks, E, T, with_shared, counts, offsets,
+                                      tiles, tiles_pair, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   index_scatter_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm, inv);

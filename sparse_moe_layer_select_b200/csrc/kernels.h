@@ -21,7 +21,6 @@ struct Tile {
 constexpr int kBlockM = 128;        // rows per tile (tcgen05 M)
 constexpr int kBlockK = 64;         // K elements per pipeline stage (one 128-byte swizzle row)
 constexpr int kStages = 4;          // shared-memory pipeline depth
-constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kIndexChunk = 4096;   // (token, slot) entries per index-builder chunk
 
 enum GemmMode : int { MODE_ROUTER = 0, MODE_GEMM1 = 1, MODE_GEMM2 = 2 };
@@ -51,7 +50,7 @@ struct GemmParams {
 };
 
 // Pipeline trace layout (MOE_TRACE builds): trace[(cta * kTraceKinds + kind) * kTraceN + n].
-constexpr int kTraceKinds = 6;
+constexpr int kTraceKinds = 8;
 constexpr int kTraceN = 4096;
 enum TraceKind : int {
   TR_ISSUE = 0,      // producer issued stage n (after its empty wait)
@@ -60,6 +59,8 @@ enum TraceKind : int {
   TR_MMA = 3,        // MMAs of stage n issued
   TR_EPI_START = 4,  // epilogue saw item n's accumulator
   TR_EPI_END = 5,    // epilogue released item n's accumulator
+  TR_PWAIT = 6,      // producer starts waiting for stage n's buffer
+  TR_PDONE = 7,      // producer finished issuing stage n
 };
 
 struct GemmMaps {
@@ -85,7 +86,7 @@ cudaError_t launch_router_select(const float *logits, const uint16_t *x, const u
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
                          int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
-                         int tile_rows = kBlockM, int32_t *inv = nullptr);
+                         Tile *tiles_pair = nullptr, int32_t *inv = nullptr);
 cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_rows, int k, int d,
                                uint16_t *x_perm, cudaStream_t s);
 // y[t] = bf16( sum_j o[inv[t*k + j]] + s_out[t] ), fp32 sums in slot order.

@@ -115,7 +115,8 @@ struct Dims {
 };
 
 struct WsLayout {
-  size_t header, chunk_hist, tiles, logits, inv, h, h_sh, o, s_out, down16, down16_sh, total;
+  size_t header, chunk_hist, tiles, tiles_pair, logits, inv, h, h_sh, o, s_out, down16, down16_sh,
+      total;
   int max_tiles;
 };
 
@@ -129,7 +130,9 @@ WsLayout ws_layout(const Dims &D) {
   off += align256(sizeof(WsHeader));
   L.chunk_hist = off;
   off += align256(std::max<size_t>(nchunks, 1) * D.E * 4);
-  L.tiles = off;
+  L.tiles = off;  // 128-row tiles (single-CTA GEMMs)
+  off += align256(static_cast<size_t>(L.max_tiles) * sizeof(Tile));
+  L.tiles_pair = off;  // 256-row tiles (CTA-pair GEMMs); fewer than the 128-row ones
   off += align256(static_cast<size_t>(L.max_tiles) * sizeof(Tile));
   L.logits = off;
   off += align256(static_cast<size_t>(D.T) * D.E * 4);
@@ -365,20 +368,24 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   st = route_impl(D, x, w->w_router, w->router_bias, routing->topk_idx, routing->topk_w, ws, s,
                   sms, &launches);
   if (st != MOE_OK) return st;
-  // 2. expert order + tile list (256-row tiles for the CTA-pair GEMMs)
-  // CTA pairs (M = 256 tiles) when the average expert fills a 256-row tile;
-  // below that, single-CTA M = 128 tiles waste less of the tensor core and
-  // were measured faster (weight-streaming shapes).
+  // 2. expert order + tile lists.  Engines, as measured on B200: the gate/up
+  // GEMM runs on single CTAs (128-row tiles; with its A rows gathered by
+  // cp.async, the CTA-pair engine lost 12-14% to it at the large prefill
+  // shapes); the down GEMM runs on CTA pairs (256-row tiles, half of B per
+  // SM) when the average expert fills a 256-row tile, below that single CTAs
+  // waste less of the tensor core.  The flags force one engine for both.
   const int pair_grid = 2 * std::min(pair_clusters(), sms / 2);  // all pairs co-resident
-  bool pair = static_cast<int64_t>(D.T) * D.k >= static_cast<int64_t>(2 * kBlockM) * D.E;
-  if (D.flags & MOE_FLAG_GEMM_PAIR) pair = true;
-  if (D.flags & MOE_FLAG_GEMM_SINGLE_CTA) pair = false;
-  if (pair_grid < 2) pair = false;
+  bool pair1 = false;
+  bool pair2 = static_cast<int64_t>(D.T) * D.k >= static_cast<int64_t>(2 * kBlockM) * D.E;
+  if (D.flags & MOE_FLAG_GEMM_PAIR) pair1 = pair2 = true;
+  if (D.flags & MOE_FLAG_GEMM_SINGLE_CTA) pair1 = pair2 = false;
+  if (pair_grid < 2) pair1 = pair2 = false;
+  Tile *tiles_pair = reinterpret_cast<Tile *>(wsp(ws, L.tiles_pair));
   ev.mark();
   if (launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0,
                    reinterpret_cast<int *>(wsp(ws, L.chunk_hist)), tiles, header, routing->counts,
                    routing->offsets, routing->perm, s, &launches,
-                   pair ? 2 * kBlockM : kBlockM, inv) != cudaSuccess)
+                   (pair1 || pair2) ? tiles_pair : nullptr, inv) != cudaSuccess)
     return MOE_ERR_CUDA;
 
   // fp16 down projections: caller-prepared, or converted here every call
@@ -408,8 +415,8 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   GemmParams base;
   std::memset(&base, 0, sizeof(base));
   base.status = header;
-  base.tiles = tiles;
-  base.n_tiles_dev = header + offsetof(WsHeader, n_tiles) / sizeof(int);
+  int *n_tiles = header + offsetof(WsHeader, n_tiles) / sizeof(int);
+  int *n_tiles_pair = header + offsetof(WsHeader, n_tiles_pair) / sizeof(int);
   base.T = D.T;
   base.d = D.d;
   base.E = D.E;
@@ -427,6 +434,8 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   // 3. GEMM1: gathered x rows . [W_gate | W_up]^T -> SwiGLU -> h (bf16)
   {
     GemmParams p = base;
+    p.tiles = pair1 ? tiles_pair : tiles;
+    p.n_tiles_dev = pair1 ? n_tiles_pair : n_tiles;
     p.n_half = n_half;
     p.n_tile = 2 * n_half;
     p.n_ntiles = std::max(D.F, D.Fs) / n_half;
@@ -454,7 +463,7 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
       m.out_sh = m.out;
     }
     ev.mark();
-    const cudaError_t e = pair ? launch_gemm_pair(MODE_GEMM1, p, m, pair_grid, s)
+    const cudaError_t e = pair1 ? launch_gemm_pair(MODE_GEMM1, p, m, pair_grid, s)
                                : launch_gemm(MODE_GEMM1, p, m, sms, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
@@ -462,6 +471,8 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
   // 4. GEMM2: h . W_down^T -> x (routed_scaling_factor * w) -> expert-order rows
   {
     GemmParams p = base;
+    p.tiles = pair2 ? tiles_pair : tiles;
+    p.n_tiles_dev = pair2 ? n_tiles_pair : n_tiles;
     p.n_tile = n2;
     p.n_ntiles = D.d / n2;
 #ifdef MOE_TRACE
@@ -475,7 +486,7 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     std::memset(&m, 0, sizeof(m));
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (!make_map(&m.a, h, n_rows, D.F, a_rows, f16)) return MOE_ERR_CUDA;
-    const uint32_t b_rows = pair ? n2 / 2 : n2;  // a pair splits B along N
+    const uint32_t b_rows = pair2 ? n2 / 2 : n2;  // a pair splits B along N
     if (!make_map(&m.b0, wd16, static_cast<uint64_t>(D.E) * D.d, D.F, b_rows, f16))
       return MOE_ERR_CUDA;
     m.b1 = m.b0;
@@ -491,7 +502,7 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
     }
     m.b1_sh = m.b0_sh;
     ev.mark();
-    const cudaError_t e = pair ? launch_gemm_pair(MODE_GEMM2, p, m, pair_grid, s)
+    const cudaError_t e = pair2 ? launch_gemm_pair(MODE_GEMM2, p, m, pair_grid, s)
                                : launch_gemm(MODE_GEMM2, p, m, sms, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;

@@ -21,9 +21,11 @@
 //                (token, slot)'s row of the slot buffer; shared-expert rows go
 //                to the last slot with scale 1.
 //
-// Roles inside a CTA (192 threads, one CTA per SM, persistent over items):
-//   warp 0      producer: fills a kStages-deep ring of (A, B) stages (TMA
-//               tiles; for GEMM1 the A rows by cp.async from all 32 lanes).
+// Roles inside a CTA (one CTA per SM, persistent over items):
+//   warp 0      producer: fills a kStages-deep ring of (A, B) stages with
+//               TMA tiles (GEMM1: the B tiles only).
+//   warps 6..   GEMM1: gather the A rows by cp.async through the expert-order
+//               permutation, a share of the 128 rows each (gemm_common.cuh).
 //   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma
 //               (M=128, N<=256, K=16 per instruction) into one of two
 //               accumulator buffers and commits stage releases.
@@ -52,6 +54,9 @@ constexpr int kABytes = kBlockM * kBlockK * 2;  // 16 KB: 128 rows x 128 bytes
 constexpr int kBBytesMax = 256 * kBlockK * 2;   // 32 KB: up to 256 rows
 constexpr int kTmemCols = 512;                  // two accumulators of up to 256 columns
 constexpr int kAccStride = 256;
+// warps: 0 TMA loads, 1 MMA, 2-5 epilogue, 6.. gather (GEMM1)
+constexpr int kGather2Warp = 6;
+constexpr int kSingleThreads = 192 + 32 * kExtraGatherWarps;
 
 struct SmemLayout {
   static constexpr int a_off = 0;
@@ -70,7 +75,7 @@ static_assert(SmemLayout::total + 1024 <= 232448, "shared memory budget");
 }  // namespace
 
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kSingleThreads, 1)
     moe_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_b0,
                     const __grid_constant__ CUtensorMap tm_b1,
@@ -99,8 +104,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       // GEMM1: one expect_tx arrival for the B tiles plus one cp.async
-      // completion arrival from each lane of the gathering warp.
-      mbar_init(&full[s], MODE == MODE_GEMM1 ? 1 + 32 : 1);
+      // completion arrival from each lane of the gathering warps.
+      mbar_init(&full[s], MODE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -134,94 +139,98 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       MODE == MODE_GEMM2 ? idesc_f16_f32(kBlockM, p.n_tile) : idesc_bf16_f32(kBlockM, p.n_tile);
   int *status = p.status;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int s = 0;
-    uint32_t ph = 0;
-    long long issued = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const Item it = decode_item<MODE>(p, item);
-      if (it.skip) continue;
-      if (status_is_set(status)) break;
-      const bool shared = it.group == p.E;
-      // GEMM1: lane l copies 16-byte chunk (l & 7) of rows (l >> 3) + 4 i,
-      // i = 0..31, so one warp instruction moves four whole 128-byte rows.
-      // Rows past the tile's valid count are not loaded (their accumulator
-      // rows are discarded by the epilogue).
-      int tok[32];
-      if (MODE == MODE_GEMM1) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int r = (lane >> 3) + 4 * i;
-          tok[i] = -1;
-          if (r < it.nrows) tok[i] = shared ? it.row0 + r : p.perm[it.row0 + r] / p.k;
+  if (warp == 0 || warp >= kGather2Warp) {
+    // ------------------------------------------------------------ loads
+    // Warp 0 issues the TMA loads (and arms each stage's barrier); the
+    // gathering warps (warp 0 too when kTmaWarpGathers) copy GEMM1's A rows,
+    // kGatherRows each.
+    const bool tma_warp = warp == 0;
+    const int gw = tma_warp ? (kTmaWarpGathers ? 0 : -1)
+                            : (kTmaWarpGathers ? 1 : 0) + (warp - kGather2Warp);
+    const bool gathers = MODE == MODE_GEMM1 && gw >= 0;
+    if (tma_warp || gathers) {
+      int s = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
+      bool ok = true;
+      ItemWalk<MODE> walk(p, blockIdx.x, gridDim.x, n_items);
+      Item it;
+      // GEMM1: row ids of this warp's rows of item raw_item (loaded one item ahead).
+      int raw[kGatherGroups];
+      int raw_item = -1;
+      while (ok && walk.current(p, it)) {
+        const bool shared = it.group == p.E;
+        int tok[kGatherGroups];
+        if (gathers) {
+          if (raw_item != walk.item) gather_rows_fetch(p, it, lane, gw, raw);
+          gather_tokens(p, it, raw, tok);
         }
-      }
-      // A boxes shorter than 128 rows (tensors with fewer rows) fill only
-      // their rows; the rest of the stage feeds accumulator rows that the
-      // epilogue discards.
-      uint32_t bytes;
-      if (MODE == MODE_ROUTER) bytes = p.a_bytes + p.E * 128;
-      else if (MODE == MODE_GEMM1) bytes = 2 * p.n_half * 128;  // A arrives by cp.async
-      else bytes = (shared ? p.a_sh_bytes : p.a_bytes) + p.n_tile * 128;
-      for (int kb = 0; kb < it.nk; ++kb) {
-        int good = 1;
-        if (lane == 0) {
-          good = mbar_wait(&empty[s], ph ^ 1, status, SITE_GEMM_PRODUCER_EMPTY);
-          if (good) mbar_arrive_expect_tx(&full[s], bytes);
-        }
-        good = __shfl_sync(0xffffffffu, good, 0);
-        if (!good) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
-        uint8_t *a_dst = sA + s * kABytes;
-        uint8_t *b_dst = sB + s * kBBytesMax;
-        const int kc = kb * kBlockK;
-        if (MODE == MODE_GEMM1) {
+        walk.prefetch(p);
+        // A boxes shorter than 128 rows (tensors with fewer rows) fill only
+        // their rows; the rest of the stage feeds accumulator rows that the
+        // epilogue discards.
+        uint32_t bytes;
+        if (MODE == MODE_ROUTER) bytes = p.a_bytes + p.E * 128;
+        else if (MODE == MODE_GEMM1) bytes = 2 * p.n_half * 128;  // A arrives by cp.async
+        else bytes = (shared ? p.a_sh_bytes : p.a_bytes) + p.n_tile * 128;
+        for (int kb = 0; kb < it.nk; ++kb) {
+          int good = 1;
+          if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_PWAIT, issued);
           if (lane == 0) {
-            const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
-            tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
-            tma_load_2d(b_dst + p.n_half * 128, shared ? &tm_b1_sh : &tm_b1, &full[s], kc, brow);
+            good = mbar_wait(&empty[s], ph ^ 1, status, SITE_GEMM_PRODUCER_EMPTY);
+            if (good && tma_warp) mbar_arrive_expect_tx(&full[s], bytes);
           }
-          // 128-byte swizzle: chunk c of row r sits at chunk (c ^ (r & 7)).
-          const int c = lane & 7;
-          const uint32_t a_base = smem_u32(a_dst);
-          const char *xsrc = reinterpret_cast<const char *>(p.x) + kc * 2 + c * 16;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int r = (lane >> 3) + 4 * i;
-            if (tok[i] >= 0)
-              cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4),
-                          xsrc + static_cast<size_t>(tok[i]) * p.d * 2);
+          good = __shfl_sync(0xffffffffu, good, 0);
+          if (!good) {
+            ok = false;
+            break;
           }
-          cp_async_arrive_noinc(&full[s]);
-        } else if (lane == 0) {
-          if (MODE == MODE_ROUTER) {
-            tma_load_2d(a_dst, &tm_a, &full[s], kc, it.row0);
-            tma_load_2d(b_dst, &tm_b0, &full[s], kc, 0);
-          } else {
-            tma_load_2d(a_dst, shared ? &tm_a_sh : &tm_a, &full[s], kc, it.row0);
-            const int brow = (shared ? 0 : it.group * p.d) + it.j * p.n_tile;
-            tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
+          if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
+          uint8_t *a_dst = sA + s * kABytes;
+          uint8_t *b_dst = sB + s * kBBytesMax;
+          const int kc = kb * kBlockK;
+          if (tma_warp && lane == 0) {
+            if (MODE == MODE_GEMM1) {
+              const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
+              tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
+              tma_load_2d(b_dst + p.n_half * 128, shared ? &tm_b1_sh : &tm_b1, &full[s], kc, brow);
+            } else if (MODE == MODE_ROUTER) {
+              tma_load_2d(a_dst, &tm_a, &full[s], kc, it.row0);
+              tma_load_2d(b_dst, &tm_b0, &full[s], kc, 0);
+            } else {
+              tma_load_2d(a_dst, shared ? &tm_a_sh : &tm_a, &full[s], kc, it.row0);
+              const int brow = (shared ? 0 : it.group * p.d) + it.j * p.n_tile;
+              tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
+            }
+          }
+          if (gathers) gather_a_stage(p, tok, lane, gw, a_dst, &full[s], kc);
+          if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_PDONE, issued);
+          ++issued;
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+          if (gathers && kb == 0) {
+            // Row ids of the next item; its tile record was loaded at this
+            // item's start.  Skipped items are fetched when reached.
+            const Item nx = decode_tile<MODE>(p, walk.item + walk.step, walk.rec);
+            raw_item = -1;
+            if (walk.item + walk.step < n_items && !nx.skip) {
+              gather_rows_fetch(p, nx, lane, gw, raw);
+              raw_item = walk.item + walk.step;
+            }
           }
         }
-        ++issued;
-        if (++s == kStages) {
-          s = 0;
-          ph ^= 1;
-        }
+        walk.next();
       }
-    }
-    // Drain: every stage this warp filled must have landed before the CTA exits.
-    if (MODE == MODE_GEMM1) cp_async_wait_all();
-    if (lane == 0) {
-      for (long long n = (issued > kStages ? issued - kStages : 0); n < issued; ++n)
-        if (!mbar_wait(&full[n % kStages], static_cast<uint32_t>((n / kStages) & 1), status,
-                       SITE_GEMM_DRAIN))
-          break;
+      // Every stage filled must have landed before the CTA exits.
+      if (gathers) cp_async_wait_all();
+      if (tma_warp && lane == 0) {
+        for (long long n = (issued > kStages ? issued - kStages : 0); n < issued; ++n)
+          if (!mbar_wait(&full[n % kStages], static_cast<uint32_t>((n / kStages) & 1), status,
+                         SITE_GEMM_DRAIN))
+            break;
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -232,10 +241,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t aph = 0;
       bool ok = true;
       int consumed = 0;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const Item it = decode_item<MODE>(p, item);
-        if (it.skip) continue;
-        if (status_is_set(status)) break;
+      ItemWalk<MODE> walk(p, blockIdx.x, gridDim.x, n_items);
+      Item it;
+      while (ok && walk.current(p, it)) {
+        walk.prefetch(p);
+        walk.next();
         if (!mbar_wait(&acc_empty[acc], aph ^ 1, status, SITE_GEMM_MMA_ACC_EMPTY)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccStride;
@@ -282,10 +292,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t aph = 0;
     int done = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item<MODE>(p, item);
-      if (it.skip) continue;
-      if (status_is_set(status)) break;
+    ItemWalk<MODE> walk(p, blockIdx.x, gridDim.x, n_items);
+    Item it;
+    while (walk.current(p, it)) {
+      walk.prefetch(p);
+      walk.next();
       if (!mbar_wait(&acc_full[acc], aph, status, SITE_GEMM_EPI_ACC_FULL)) break;
       if (warp == 2 && lane == 0) MOE_TRACE_AT(p, TR_EPI_START, done);
       tc_fence_after();
@@ -324,7 +335,7 @@ cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int gr
   const size_t smem = gemm_smem_bytes();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(kSingleThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = nullptr;

@@ -12,6 +12,8 @@
 // Synchronisation (all waits bounded, as in moe_gemm.cu):
 //   lfull[s]   per CTA: its own loads of stage s have landed (TMA bytes and
 //              cp.async arrivals)
+//   gather     GEMM1's A rows are copied by warps 7.. (each a share of the
+//              128 rows, gemm_common.cuh); warp 0 issues the TMA loads
 //   relay      warp 6 of each CTA forwards each completed stage to the
 //              leader's full[s] (two arrivals per phase), after a proxy fence
 //              for the cp.async-written rows; each CTA can therefore always
@@ -36,7 +38,9 @@ using namespace gemm;
 namespace {
 
 constexpr int kPairStages = 6;
-constexpr int kPairThreads = 224;                // warps: 0 load, 1 MMA, 2-5 epilogue, 6 relay
+// warps: 0 TMA loads, 1 MMA, 2-5 epilogue, 6 relay, 7.. gather (GEMM1)
+constexpr int kPairGather2Warp = 7;
+constexpr int kPairThreads = 224 + 32 * kExtraGatherWarps;
 constexpr int kPABytes = kBlockM * kBlockK * 2;  // 16 KB: this CTA's 128 rows of A
 constexpr int kPBBytes = 128 * kBlockK * 2;      // 16 KB: this CTA's half of B (<= 128 rows)
 constexpr int kPTmemCols = 512;
@@ -89,8 +93,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&full[s], 2);
-      // own loads: one expect_tx arrival (+ 32 cp.async arrivals for the gathered rows)
-      mbar_init(&lfull[s], MODE == MODE_GEMM1 ? 1 + 32 : 1);
+      // own loads: one expect_tx arrival (+ one cp.async arrival per gathering lane)
+      mbar_init(&lfull[s], MODE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -103,7 +107,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_b0);
     prefetch_tmap(&tm_b1);
-    if (MODE == MODE_GEMM2) prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_a);  // GEMM1: the gather4 map of x (one-row boxes)
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kPTmemCols);
@@ -121,81 +125,94 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   int *status = p.status;
   const int half_b_rows = MODE == MODE_GEMM1 ? p.n_half : p.n_tile / 2;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ loads (both CTAs)
-    int s = 0;
-    uint32_t ph = 0;
-    long long issued = 0;
-    bool ok = true;
-    for (int item = cluster_id; item < n_items && ok; item += n_clusters) {
-      const Item whole = decode_item<MODE>(p, item);
-      if (whole.skip) continue;
-      if (status_is_set(status)) break;
-      const Item it = pair_half(whole, rank);
-      const bool shared = it.group == p.E;
-      int tok[32];
-      if (MODE == MODE_GEMM1) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int r = (lane >> 3) + 4 * i;
-          tok[i] = -1;
-          if (r < it.nrows) tok[i] = shared ? it.row0 + r : p.perm[it.row0 + r] / p.k;
+  if (warp == 0 || warp >= kPairGather2Warp) {
+    // ------------------------------------------------------------ loads
+    // Warp 0 issues the TMA loads (and arms each stage's barrier); the
+    // gathering warps (warp 0 too when kTmaWarpGathers) copy GEMM1's A rows,
+    // kGatherRows each.
+    const bool tma_warp = warp == 0;
+    const int gw = tma_warp ? (kTmaWarpGathers ? 0 : -1)
+                            : (kTmaWarpGathers ? 1 : 0) + (warp - kPairGather2Warp);
+    const bool gathers = MODE == MODE_GEMM1 && gw >= 0;
+    if (tma_warp || gathers) {
+      int s = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
+      bool ok = true;
+      ItemWalk<MODE> walk(p, cluster_id, n_clusters, n_items);
+      Item whole;
+      // GEMM1: row ids of this warp's rows of item raw_item (loaded one item ahead).
+      int raw[kGatherGroups];
+      int raw_item = -1;
+      while (ok && walk.current(p, whole)) {
+        const Item it = pair_half(whole, rank);
+        const bool shared = it.group == p.E;
+        int tok[kGatherGroups];
+        if (gathers) {
+          if (raw_item != walk.item) gather_rows_fetch(p, it, lane, gw, raw);
+          gather_tokens(p, it, raw, tok);
         }
-      }
-      const uint32_t bytes = MODE == MODE_GEMM1
-                                 ? static_cast<uint32_t>(half_b_rows * 128)
-                                 : (shared ? p.a_sh_bytes : p.a_bytes) + half_b_rows * 128;
-      for (int kb = 0; kb < whole.nk; ++kb) {
-        int good = 1;
-        if (lane == 0) {
-          good = mbar_wait(&empty[s], ph ^ 1, status, SITE_GEMM_PRODUCER_EMPTY);
-          if (good) mbar_arrive_expect_tx(&lfull[s], bytes);
-        }
-        good = __shfl_sync(0xffffffffu, good, 0);
-        if (!good) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
-        uint8_t *a_dst = sA + s * kPABytes;
-        uint8_t *b_dst = sB + s * kPBBytes;
-        const int kc = kb * kBlockK;
-        if (MODE == MODE_GEMM1) {
+        walk.prefetch(p);
+        const uint32_t bytes = MODE == MODE_GEMM1
+                                   ? static_cast<uint32_t>(half_b_rows * 128)
+                                   : (shared ? p.a_sh_bytes : p.a_bytes) + half_b_rows * 128;
+        for (int kb = 0; kb < whole.nk; ++kb) {
+          int good = 1;
+          if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_PWAIT, issued);
           if (lane == 0) {
-            // leader: gate rows; peer: up rows of the same column block
-            const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
-            const CUtensorMap *tm = leader ? (shared ? &tm_b0_sh : &tm_b0) : (shared ? &tm_b1_sh : &tm_b1);
-            tma_load_2d(b_dst, tm, &lfull[s], kc, brow);
+            good = mbar_wait(&empty[s], ph ^ 1, status, SITE_GEMM_PRODUCER_EMPTY);
+            if (good && tma_warp) mbar_arrive_expect_tx(&lfull[s], bytes);
           }
-          const int c = lane & 7;
-          const uint32_t a_base = smem_u32(a_dst);
-          const char *xsrc = reinterpret_cast<const char *>(p.x) + kc * 2 + c * 16;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int r = (lane >> 3) + 4 * i;
-            if (tok[i] >= 0)
-              cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4),
-                          xsrc + static_cast<size_t>(tok[i]) * p.d * 2);
+          good = __shfl_sync(0xffffffffu, good, 0);
+          if (!good) {
+            ok = false;
+            break;
           }
-          cp_async_arrive_noinc(&lfull[s]);
-        } else if (lane == 0) {
-          tma_load_2d(a_dst, shared ? &tm_a_sh : &tm_a, &lfull[s], kc, it.row0);
-          const int brow = (shared ? 0 : it.group * p.d) + it.j * p.n_tile + rank * half_b_rows;
-          tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &lfull[s], kc, brow);
+          if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
+          uint8_t *a_dst = sA + s * kPABytes;
+          uint8_t *b_dst = sB + s * kPBBytes;
+          const int kc = kb * kBlockK;
+          if (tma_warp && lane == 0) {
+            if (MODE == MODE_GEMM1) {
+              // leader: gate rows; peer: up rows of the same column block
+              const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
+              const CUtensorMap *tm =
+                  leader ? (shared ? &tm_b0_sh : &tm_b0) : (shared ? &tm_b1_sh : &tm_b1);
+              tma_load_2d(b_dst, tm, &lfull[s], kc, brow);
+            } else {
+              tma_load_2d(a_dst, shared ? &tm_a_sh : &tm_a, &lfull[s], kc, it.row0);
+              const int brow = (shared ? 0 : it.group * p.d) + it.j * p.n_tile + rank * half_b_rows;
+              tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &lfull[s], kc, brow);
+            }
+          }
+          if (gathers) gather_a_stage(p, tok, lane, gw, a_dst, &lfull[s], kc);
+          if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_PDONE, issued);
+          ++issued;
+          if (++s == kPairStages) {
+            s = 0;
+            ph ^= 1;
+          }
+          if (gathers && kb == 0) {
+            // Row ids of the next item; its tile record was loaded at this
+            // item's start.  Skipped items are fetched when reached.
+            const Item nx = decode_tile<MODE>(p, walk.item + walk.step, walk.rec);
+            raw_item = -1;
+            if (walk.item + walk.step < n_items && !nx.skip) {
+              gather_rows_fetch(p, pair_half(nx, rank), lane, gw, raw);
+              raw_item = walk.item + walk.step;
+            }
+          }
         }
-        ++issued;
-        if (++s == kPairStages) {
-          s = 0;
-          ph ^= 1;
-        }
+        walk.next();
       }
-    }
-    if (MODE == MODE_GEMM1) cp_async_wait_all();
-    if (lane == 0) {
-      for (long long n = (issued > kPairStages ? issued - kPairStages : 0); n < issued; ++n)
-        if (!mbar_wait(&lfull[n % kPairStages], static_cast<uint32_t>((n / kPairStages) & 1), status,
-                       SITE_GEMM_DRAIN))
-          break;
+      // Every stage filled must have landed before the CTA exits.
+      if (gathers) cp_async_wait_all();
+      if (tma_warp && lane == 0) {
+        for (long long n = (issued > kPairStages ? issued - kPairStages : 0); n < issued; ++n)
+          if (!mbar_wait(&lfull[n % kPairStages], static_cast<uint32_t>((n / kPairStages) & 1), status,
+                         SITE_GEMM_DRAIN))
+            break;
+      }
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------ relay (both CTAs)
@@ -205,10 +222,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t ph = 0;
       bool ok = true;
       int relayed = 0;
-      for (int item = cluster_id; item < n_items && ok; item += n_clusters) {
-        const Item whole = decode_item<MODE>(p, item);
-        if (whole.skip) continue;
-        if (status_is_set(status)) break;
+      ItemWalk<MODE> walk(p, cluster_id, n_clusters, n_items);
+      Item whole;
+      while (ok && walk.current(p, whole)) {
+        walk.prefetch(p);
+        walk.next();
         for (int kb = 0; kb < whole.nk; ++kb) {
           if (!mbar_wait(&lfull[s], ph, status, SITE_GEMM_MMA_FULL)) {
             ok = false;
@@ -237,10 +255,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t aph = 0;
       bool ok = true;
       int consumed = 0;
-      for (int item = cluster_id; item < n_items && ok; item += n_clusters) {
-        const Item it = decode_item<MODE>(p, item);
-        if (it.skip) continue;
-        if (status_is_set(status)) break;
+      ItemWalk<MODE> walk(p, cluster_id, n_clusters, n_items);
+      Item it;
+      while (ok && walk.current(p, it)) {
+        walk.prefetch(p);
+        walk.next();
         if (!mbar_wait(&acc_empty[acc], aph ^ 1, status, SITE_GEMM_MMA_ACC_EMPTY)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kPAccStride;
@@ -285,10 +304,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     int acc = 0;
     uint32_t aph = 0;
     int done = 0;
-    for (int item = cluster_id; item < n_items; item += n_clusters) {
-      const Item whole = decode_item<MODE>(p, item);
-      if (whole.skip) continue;
-      if (status_is_set(status)) break;
+    ItemWalk<MODE> walk(p, cluster_id, n_clusters, n_items);
+    Item whole;
+    while (walk.current(p, whole)) {
+      walk.prefetch(p);
+      walk.next();
       if (!mbar_wait(&acc_full[acc], aph, status, SITE_GEMM_EPI_ACC_FULL)) break;
       if (warp == 2 && lane == 0) MOE_TRACE_AT(p, TR_EPI_START, done);
       tc_fence_after();

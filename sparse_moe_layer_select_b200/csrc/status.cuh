@@ -28,8 +28,9 @@ enum Site : int {
 struct WsHeader {
   int status;     // first error code (0 = none)
   int site;       // Site of that error
-  int n_tiles;    // row tiles in the expert tile list (written by the index builder)
-  int pad[61];
+  int n_tiles;    // 128-row tiles in the expert tile list (written by the index builder)
+  int n_tiles_pair;  // 256-row tiles in the second list, when one is built
+  int pad[60];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 

@@ -90,6 +90,25 @@ def test_ragged_and_multi_tile_forward(T, engine):
     G.check_output(G.y_numpy(y), ref["y"], what=f"T={T}")
 
 
+@pytest.mark.parametrize("T", [1024, 1500])
+def test_auto_engines_mixed_and_equal_to_forced(T):
+    """T*k >= 256*E: by default the gate/up GEMM runs on single CTAs (128-row tile list) and the
+    down GEMM on CTA pairs (256-row tile list).  Checked against the oracle, and against both
+    forced engines bit for bit: every engine runs the same K order of fp32 MMA accumulation."""
+    w = I.get("c1_tiny").with_(T=T)
+    assert w.T * w.k >= 256 * w.E
+    h, dev = _small(w)
+    y, routing, _ = G.run_forward(w, dev, flags=0)
+    ref = G.oracle_forward(w, h)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
+    G.check_output(G.y_numpy(y), ref["y"], what=f"auto T={T}")
+    import torch
+    bits = y.view(torch.int16).cpu().numpy()
+    for engine in ENGINES:
+        y2, _, _ = G.run_forward(w, dev, flags=engine)
+        assert np.array_equal(y2.view(torch.int16).cpu().numpy(), bits), engine
+
+
 def test_permute_materialised_gather_and_counts():
     import torch
     w = I.get("c1_tiny").with_(T=1000)
