@@ -237,9 +237,7 @@ def run_ours(args):
             M.profile_next_forward(events)
         layer.forward(x_buf, y)
 
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                          if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
-                          else f"/tmp/clocks_rank{rank}.csv")
+    clocks = ClockSampler(local, os.environ.get("MOE_CLOCKS_CSV", f"/tmp/clocks_rank{rank}.csv"))
     clocks.wait_first_sample()
     # warm-up: at least W steps and at least 0.3 s, so clocks settle under load
     t_w = time.time()

@@ -76,15 +76,16 @@ typedef struct {
 /* flags: force one of the two router implementations (both compute the same
  * selection rule; the choice only changes speed). */
 #define MOE_FLAG_ROUTER_CUDA_CORE 1   /* fp32 FMA logits + warp-per-token top-k */
-#define MOE_FLAG_ROUTER_TENSOR    2   /* tcgen05 logits with the top-k in the epilogue */
+#define MOE_FLAG_ROUTER_TENSOR    2   /* tcgen05 logits + the same warp-per-token top-k */
 /* The caller passes fp16 copies of the down projections (w_down_f16,
  * ws_down_f16, made once by moe_prepare_down_f16); without this flag
  * moe_forward converts them into the workspace on every call. */
 #define MOE_FLAG_DOWN_F16         4
-/* Engine of the expert GEMMs.  By default CTA pairs (clusters of two SMs,
- * M = 256 tiles) are used when T * k >= 256 * E (the average expert fills a
- * 256-row tile) and single CTAs (M = 128 tiles) otherwise; these flags force
- * one of them.  Both give the same results. */
+/* Engine of the expert GEMMs.  By default the gate/up GEMM runs on single
+ * CTAs (M = 128 tiles) and the down GEMM on CTA pairs (clusters of two SMs,
+ * M = 256 tiles) when T * k >= 256 * E (the average expert fills a 256-row
+ * tile), on single CTAs otherwise; these flags force one engine for both.
+ * All choices give the same results. */
 #define MOE_FLAG_GEMM_SINGLE_CTA  8
 #define MOE_FLAG_GEMM_PAIR        16
 
@@ -127,14 +128,29 @@ moe_status moe_route(const moe_dims_t *dims, const void *x, const void *w_router
                      const float *router_bias, int32_t *topk_idx, float *topk_w,
                      void *ws, size_t ws_bytes, void *stream);
 
+/* Expert id of a (token, slot) pair that is not routed. */
+#define MOE_NOT_ROUTED (-1)
+
+/* moe_route with a padding mask: token_mask [T] uint8 device array, 0 marks a
+ * padding token, which is not routed (the Laguna training notes: padding
+ * tokens are best neither routed nor load-balanced).  Its k slots get
+ * topk_idx = MOE_NOT_ROUTED and topk_w = 0.  token_mask = NULL routes every
+ * token (same as moe_route).  Other tokens are routed exactly as by moe_route. */
+moe_status moe_route_masked(const moe_dims_t *dims, const void *x, const void *w_router,
+                            const float *router_bias, const uint8_t *token_mask,
+                            int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes,
+                            void *stream);
+
 /* Expert order of the (token, slot) pairs, the layout in which tokens are
  * handed to the grouped expert GEMM (Laguna M.1/XS.2 Technical Report
  * summary, Key claims, report §3.1.2, Fig. 2: tokens copied "in expert
  * order").  counts[e] = rows of expert e; offsets = exclusive prefix sum
  * ([E + 1]); perm[r] = t * k + j, rows of one expert in ascending (t, j).
  * If x and x_perm are both non-NULL the gathered rows are also materialised:
- * x_perm[r, :] = x[perm[r] / k, :] ([T * k, d] bf16).  An expert id outside
- * [0, E) sets MOE_ERR_DEVICE_BOUNDS in the status word. */
+ * x_perm[r, :] = x[perm[r] / k, :] ([T * k, d] bf16).  Pairs with expert id
+ * MOE_NOT_ROUTED are left out (counts and offsets[E] cover the routed pairs;
+ * perm and x_perm rows past offsets[E] are not written).  Any other expert id
+ * outside [0, E) sets MOE_ERR_DEVICE_BOUNDS in the status word. */
 moe_status moe_permute(const moe_dims_t *dims, const int32_t *topk_idx, int32_t *counts,
                        int32_t *offsets, int32_t *perm, const void *x, void *x_perm,
                        void *ws, size_t ws_bytes, void *stream);
@@ -152,6 +168,16 @@ moe_status moe_permute(const moe_dims_t *dims, const int32_t *topk_idx, int32_t 
 moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *weights, const void *x,
                        void *y, const moe_routing_t *routing, void *ws, size_t ws_bytes,
                        void *stream);
+
+/* moe_forward with a padding mask (token_mask as in moe_route_masked, NULL =
+ * none).  A padding token is not routed: it adds no rows to any expert and its
+ * routed contribution is zero, so y_t = shared expert(x_t) (the shared expert
+ * involves no routing and is applied to every token; zero if Fs = 0).  Other
+ * tokens' outputs are those of moe_forward. */
+moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *weights,
+                              const void *x, const uint8_t *token_mask, void *y,
+                              const moe_routing_t *routing, void *ws, size_t ws_bytes,
+                              void *stream);
 
 /* One-time preparation of the down projections for moe_forward: fp16 copies
  * w_down_f16 [E, d, F] and ws_down_f16 [d, Fs] (NULL if Fs = 0) of the bf16

@@ -25,7 +25,7 @@ What the layer computes, and where the pages say so:
   (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1.2,
   Fig. 2: tokens are copied "in expert order").
 
-Readings where the pages are silent (each one listed in the design doc):
+Readings where the pages are silent:
 
 * SwiGLU(x) = W_down (silu(W_gate x) * (W_up x)), silu(z) = z * sigmoid(z).
 * One shared expert of the same SwiGLU form, ungated, added after the 2.5.
@@ -35,6 +35,8 @@ Readings where the pages are silent (each one listed in the design doc):
   is the same as taking it on the logits.  Exact ties go to the lower expert
   index.  The selected list is ordered by descending score.
 * Normalisation runs over the k selected experts only, with no epsilon.
+* A padding token (token mask 0) is not routed: no expert, weight 0, no row
+  in the expert order; the shared expert still applies to it.
 
 Every function is a direct transcription of these definitions; numpy's
 matmul is the only library step.
@@ -99,8 +101,16 @@ def normalise(selected_scores, norm_topk_prob=True):
     return s / s.sum(axis=1, keepdims=True)
 
 
-def route(x, w_router, bias, k, norm_topk_prob=True):
+# Expert id of a (token, slot) pair that is not routed (a padding token).
+NOT_ROUTED = -1
+
+
+def route(x, w_router, bias, k, norm_topk_prob=True, token_mask=None):
     """Sigmoid router with post-top-k normalisation.
+
+    token_mask ([T], 0 = padding token) leaves padding tokens unrouted: their
+    k slots get expert id NOT_ROUTED and weight 0 (Laguna training notes:
+    padding tokens are best neither routed nor load-balanced).
 
     Returns (topk_idx [T,k] int64, topk_w [T,k] f64, scores [T,E] f64, logits [T,E] f64).
     """
@@ -108,7 +118,12 @@ def route(x, w_router, bias, k, norm_topk_prob=True):
     scores = sigmoid(logits)
     idx = select_topk(logits, k)
     sel = np.take_along_axis(scores, idx, axis=1)
-    return idx, normalise(sel, norm_topk_prob), scores, logits
+    w = normalise(sel, norm_topk_prob)
+    if token_mask is not None:
+        pad = np.asarray(token_mask) == 0
+        idx[pad, :] = NOT_ROUTED
+        w[pad, :] = 0.0
+    return idx, w, scores, logits
 
 
 def swiglu_ffn(x, w_gate, w_up, w_down):
@@ -130,19 +145,23 @@ def expert_order(topk_idx, E):
     offsets    = exclusive prefix sum of counts, length E + 1;
     perm[r]    = t * k + j for the r-th row in expert order, where rows of
                  one expert are sorted by token t, then by slot j.
+    Pairs with expert id NOT_ROUTED are left out: perm has offsets[E] rows.
     """
     idx = np.asarray(topk_idx, dtype=np.int64)
     T, k = idx.shape
     counts = np.zeros(E, dtype=np.int64)
     for e in idx.reshape(-1):
-        counts[e] += 1
+        if e != NOT_ROUTED:
+            counts[e] += 1
     offsets = np.zeros(E + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(counts)
-    perm = np.empty(T * k, dtype=np.int64)
+    perm = np.empty(offsets[E], dtype=np.int64)
     fill = offsets[:-1].copy()
     for t in range(T):
         for j in range(k):
             e = idx[t, j]
+            if e == NOT_ROUTED:
+                continue
             perm[fill[e]] = t * k + j
             fill[e] += 1
     return counts, offsets, perm
@@ -150,12 +169,16 @@ def expert_order(topk_idx, E):
 
 def moe_forward(x, w_router, w_gate, w_up, w_down, k, *, router_bias=None,
                 ws_gate=None, ws_up=None, ws_down=None,
-                routed_scaling_factor=2.5, norm_topk_prob=True, routing=None):
+                routed_scaling_factor=2.5, norm_topk_prob=True, routing=None,
+                token_mask=None):
     """y_t = S(x_t) + scale * sum_j w_{t,j} * E_{e_{t,j}}(x_t), in float64.
 
     x: [T, d]; w_router: [E, d]; w_gate, w_up: [E, F, d]; w_down: [E, d, F];
     ws_gate, ws_up: [Fs, d]; ws_down: [d, Fs] (None: no shared expert).
     ``routing`` may pass a precomputed (topk_idx, topk_w) pair from ``route``.
+    ``token_mask`` ([T], 0 = padding): a padding token is not routed, so its
+    routed sum is empty and y_t = S(x_t); the shared expert, which involves no
+    routing, still applies.
 
     Returns a dict with y, the routed sum R (before the scale), the shared
     output Sh, and the routing (topk_idx, topk_w, scores, logits).
@@ -163,7 +186,7 @@ def moe_forward(x, w_router, w_gate, w_up, w_down, k, *, router_bias=None,
     X = bf16_to_f64(x)
     T, d = X.shape
     if routing is None:
-        idx, w, scores, logits = route(x, w_router, router_bias, k, norm_topk_prob)
+        idx, w, scores, logits = route(x, w_router, router_bias, k, norm_topk_prob, token_mask)
     else:
         idx, w = routing
         scores = logits = None

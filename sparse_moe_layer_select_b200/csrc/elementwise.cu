@@ -4,7 +4,8 @@
 //                       activations; the forward pass fuses this gather into the GEMM
 //                       operand load instead)
 //   combine_kernel      y[t, :] = bf16( sum_j o[inv[t*k + j], :] + s[t, :] ) in fp32 over
-//                       the k routed fp16 rows (already scaled by routed_scaling_factor *
+//                       the k routed fp16 rows (a padding token's slots have inv = -1
+//                       and add nothing) (already scaled by routed_scaling_factor *
 //                       w_t,j, stored in expert order) and the shared-expert row: the
 //                       combine of the routed sum with the always-on shared expert
 //                       (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1)
@@ -24,9 +25,10 @@ namespace moe {
 namespace {
 
 __global__ void __launch_bounds__(256)
-    gather_rows_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ perm, int n_rows,
-                       int k, int vec_per_row, uint4 *__restrict__ x_perm) {
-  const size_t total = static_cast<size_t>(n_rows) * vec_per_row;
+    gather_rows_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ perm,
+                       const int32_t *__restrict__ n_valid, int n_rows, int k, int vec_per_row,
+                       uint4 *__restrict__ x_perm) {
+  const size_t total = static_cast<size_t>(min(*n_valid, n_rows)) * vec_per_row;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int r = static_cast<int>(i / vec_per_row);
@@ -60,7 +62,7 @@ __global__ void __launch_bounds__(256)
     };
     for (int j = 0; j < k; ++j) {
       const int r = inv[t * k + j];
-      add(o[static_cast<size_t>(r) * vec_per_row + c]);
+      if (r >= 0) add(o[static_cast<size_t>(r) * vec_per_row + c]);
     }
     if (s_out) add(s_out[t * vec_per_row + c]);
     uint32_t out[4];
@@ -126,12 +128,12 @@ int grid_for(size_t work, int threads) {
 
 }  // namespace
 
-cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_rows, int k, int d,
-                               uint16_t *x_perm, cudaStream_t s) {
+cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, const int32_t *n_valid,
+                               int n_rows, int k, int d, uint16_t *x_perm, cudaStream_t s) {
   const int vpr = d / 8;
   const size_t work = static_cast<size_t>(n_rows) * vpr;
   gather_rows_kernel<<<grid_for(work, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(x), perm,
-                                                         n_rows, k, vpr,
+                                                         n_valid, n_rows, k, vpr,
                                                          reinterpret_cast<uint4 *>(x_perm));
   return cudaGetLastError();
 }

@@ -7,7 +7,9 @@
 //
 //   counts[e]  rows of expert e;  offsets = exclusive prefix sum (E + 1)
 //   perm[r]    = t * k + j for the r-th row in expert order, rows of one
-//                expert in ascending (t, j) -- a stable counting sort.
+//                expert in ascending (t, j) -- a stable counting sort.  Pairs
+//                with expert id kNotRouted (-1: padding tokens) are left out:
+//                offsets[E] counts the routed pairs only.
 //   tiles      (expert, first row, rows) blocks of at most tile_rows rows
 //              (128 for single-CTA GEMMs, 256 for CTA-pair GEMMs), in expert
 //              order, followed by the shared expert's token blocks.
@@ -79,6 +81,7 @@ __device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk
     const int i = base + r;
     if (i >= n) break;
     const int e = topk_idx[i];
+    if (e == kNotRouted) continue;
     if (e < 0 || e >= E) {
       if (status) record_status(status, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
       continue;
@@ -112,6 +115,8 @@ __device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ t
       const int pos = fw[e] + rank;
       perm[pos] = i;
       if (inv) inv[i] = pos;  // expert-order row of entry i = t * k + j
+    } else if (inv && i < n) {
+      inv[i] = -1;  // not routed
     }
     __syncwarp();
     if (e >= 0 && rank == 0) fw[e] += __popc(m);
@@ -275,6 +280,7 @@ __global__ void __launch_bounds__(512)
       const int i = warp * kSub + r;
       if (i >= n) break;
       const int e = topk_idx[i];
+      if (e == kNotRouted) continue;
       if (e < 0 || e >= E) {
         record_status(header, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
         continue;

@@ -79,17 +79,25 @@ cudaError_t launch_gemm_pair(int mode, const GemmParams &p, const GemmMaps &m, i
 cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
                              float *logits, int T, int d, int E, cudaStream_t s);
 // Warp-per-token selection over the fp32 logits of every token.
+// Expert id of a (token, slot) pair that is not routed (a padding token).
+constexpr int kNotRouted = -1;
+
+// token_mask (optional, [T]): 0 = padding token, which gets kNotRouted ids
+// and zero weights.
 cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
-                                 const float *bias, int T, int d, int E, int k, int norm_topk,
-                                 int32_t *topk_idx, float *topk_w, cudaStream_t s);
+                                 const float *bias, const uint8_t *token_mask, int T, int d, int E,
+                                 int k, int norm_topk, int32_t *topk_idx, float *topk_w,
+                                 cudaStream_t s);
 
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
                          int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
                          Tile *tiles_pair = nullptr, int32_t *inv = nullptr);
-cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, int n_rows, int k, int d,
-                               uint16_t *x_perm, cudaStream_t s);
-// y[t] = bf16( sum_j o[inv[t*k + j]] + s_out[t] ), fp32 sums in slot order.
+// x_perm[r] = x[perm[r] / k] for r < *n_valid (the routed rows, offsets[E]).
+cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, const int32_t *n_valid,
+                               int n_rows, int k, int d, uint16_t *x_perm, cudaStream_t s);
+// y[t] = bf16( sum_j o[inv[t*k + j]] + s_out[t] ), fp32 sums in slot order; slots
+// with inv < 0 (not routed) are skipped.
 cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32_t *inv, int T,
                            int k, int d, uint16_t *y, cudaStream_t s);
 cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int *status,

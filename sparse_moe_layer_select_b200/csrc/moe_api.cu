@@ -201,8 +201,8 @@ bool use_tensor_router(const Dims &D) {
 // Router: fp32 logits (tcgen05 GEMM or CUDA-core FMA) into the workspace,
 // then the warp-per-token selection kernel.
 moe_status route_impl(const Dims &D, const void *x, const void *w_router, const float *bias,
-                      int32_t *topk_idx, float *topk_w, void *ws, cudaStream_t s, int sms,
-                      int *launches) {
+                      const uint8_t *token_mask, int32_t *topk_idx, float *topk_w, void *ws,
+                      cudaStream_t s, int sms, int *launches) {
   const WsLayout L = ws_layout(D);
   float *logits = reinterpret_cast<float *>(wsp(ws, L.logits));
   if (use_tensor_router(D)) {
@@ -234,8 +234,8 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     const int grid = std::min(sms, p.n_tiles_host);
     if (launch_gemm(MODE_ROUTER, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (launch_router_select(logits, static_cast<const uint16_t *>(x),
-                             static_cast<const uint16_t *>(w_router), bias, D.T, D.d, D.E, D.k,
-                             D.norm, topk_idx, topk_w, s) != cudaSuccess)
+                             static_cast<const uint16_t *>(w_router), bias, token_mask, D.T, D.d,
+                             D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
       return MOE_ERR_CUDA;
     *launches += 2;
     return MOE_OK;
@@ -244,8 +244,8 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
                        bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (launch_router_select(logits, static_cast<const uint16_t *>(x),
-                           static_cast<const uint16_t *>(w_router), bias, D.T, D.d, D.E, D.k,
-                           D.norm, topk_idx, topk_w, s) != cudaSuccess)
+                           static_cast<const uint16_t *>(w_router), bias, token_mask, D.T, D.d,
+                           D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   *launches += 2;
   return MOE_OK;
@@ -268,6 +268,14 @@ size_t moe_workspace_size(const moe_dims_t *dims) {
 moe_status moe_route(const moe_dims_t *dims, const void *x, const void *w_router,
                      const float *router_bias, int32_t *topk_idx, float *topk_w, void *ws,
                      size_t ws_bytes, void *stream) {
+  return moe_route_masked(dims, x, w_router, router_bias, nullptr, topk_idx, topk_w, ws, ws_bytes,
+                          stream);
+}
+
+moe_status moe_route_masked(const moe_dims_t *dims, const void *x, const void *w_router,
+                            const float *router_bias, const uint8_t *token_mask,
+                            int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes,
+                            void *stream) {
   Dims D;
   moe_status st = check_dims(dims, &D);
   if (st != MOE_OK) return st;
@@ -283,7 +291,8 @@ moe_status moe_route(const moe_dims_t *dims, const void *x, const void *w_router
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = clear_header(ws, s)) != MOE_OK) return st;
   int launches = 0;
-  st = route_impl(D, x, w_router, router_bias, topk_idx, topk_w, ws, s, sms, &launches);
+  st = route_impl(D, x, w_router, router_bias, token_mask, topk_idx, topk_w, ws, s, sms,
+                  &launches);
   g_last_launches = launches;
   return st;
 }
@@ -314,8 +323,8 @@ moe_status moe_permute(const moe_dims_t *dims, const int32_t *topk_idx, int32_t 
                    &launches) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (x) {
-    if (launch_gather_rows(static_cast<const uint16_t *>(x), perm, D.T * D.k, D.k, D.d,
-                           static_cast<uint16_t *>(x_perm), s) != cudaSuccess)
+    if (launch_gather_rows(static_cast<const uint16_t *>(x), perm, offsets + D.E, D.T * D.k, D.k,
+                           D.d, static_cast<uint16_t *>(x_perm), s) != cudaSuccess)
       return MOE_ERR_CUDA;
     launches += 1;
   }
@@ -325,6 +334,12 @@ moe_status moe_permute(const moe_dims_t *dims, const int32_t *topk_idx, int32_t 
 
 moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const void *x, void *y,
                        const moe_routing_t *routing, void *ws, size_t ws_bytes, void *stream) {
+  return moe_forward_masked(dims, w, x, nullptr, y, routing, ws, ws_bytes, stream);
+}
+
+moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, const void *x,
+                              const uint8_t *token_mask, void *y, const moe_routing_t *routing,
+                              void *ws, size_t ws_bytes, void *stream) {
   Dims D;
   moe_status st = check_dims(dims, &D);
   if (st != MOE_OK) return st;
@@ -365,8 +380,8 @@ moe_status moe_forward(const moe_dims_t *dims, const moe_weights_t *w, const voi
 
   // 1. router
   ev.mark();
-  st = route_impl(D, x, w->w_router, w->router_bias, routing->topk_idx, routing->topk_w, ws, s,
-                  sms, &launches);
+  st = route_impl(D, x, w->w_router, w->router_bias, token_mask, routing->topk_idx,
+                  routing->topk_w, ws, s, sms, &launches);
   if (st != MOE_OK) return st;
   // 2. expert order + tile lists.  Engines, as measured on B200: the gate/up
   // GEMM runs on single CTAs (128-row tiles; with its A rows gathered by

@@ -283,12 +283,21 @@ template <int NPL>
 __global__ void __launch_bounds__(kSelectWarps * 32)
     router_select_kernel(const float *__restrict__ logits, const uint16_t *__restrict__ x,
                          const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
-                         int T, int d, int E, int k, int norm_topk,
+                         const uint8_t *__restrict__ token_mask, int T, int d, int E, int k,
+                         int norm_topk,
                          int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
-  if (t < T)
-    select_token<NPL>(t, lane, logits, x, w_router, bias, d, E, k, norm_topk, topk_idx, topk_w);
+  if (t >= T) return;
+  if (token_mask != nullptr && token_mask[t] == 0) {
+    // padding token: not routed (no experts, zero weights)
+    if (lane < k) {
+      topk_idx[static_cast<size_t>(t) * k + lane] = kNotRouted;
+      topk_w[static_cast<size_t>(t) * k + lane] = 0.f;
+    }
+    return;
+  }
+  select_token<NPL>(t, lane, logits, x, w_router, bias, d, E, k, norm_topk, topk_idx, topk_w);
 }
 
 }  // namespace
@@ -312,14 +321,15 @@ cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const 
 }
 
 cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
-                                 const float *bias, int T, int d, int E, int k, int norm_topk,
-                                 int32_t *topk_idx, float *topk_w, cudaStream_t s) {
+                                 const float *bias, const uint8_t *token_mask, int T, int d, int E,
+                                 int k, int norm_topk, int32_t *topk_idx, float *topk_w,
+                                 cudaStream_t s) {
   const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
   const int threads = kSelectWarps * 32;
   const int npl = (E + 31) / 32;
 #define MOE_SELECT(N)                                                                          \
-  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, T, d, E, k,   \
-                                                     norm_topk, topk_idx, topk_w)
+  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, token_mask, T, \
+                                                     d, E, k, norm_topk, topk_idx, topk_w)
   if (npl <= 1) MOE_SELECT(1);
   else if (npl <= 2) MOE_SELECT(2);
   else if (npl <= 4) MOE_SELECT(4);

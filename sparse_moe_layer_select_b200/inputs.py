@@ -124,6 +124,14 @@ WORKLOADS = {
                             shared_intermediate_size=1024, sigma_x=1.0, sigma_w=0.015,
                             sigma_router=0.02,
                             note="M.1-width layer, T=16384, d=4096, F=Fs=1024"),
+    # M.1 as its spec sheet configures the layer (Mixture of experts: 16 experts
+    # per token, routed scaling factor 1), at the M.1 widths of c4_m1_width.
+    "c6_m1_top16": Workload("c6_m1_top16", T=16384, d_model=4096, num_experts=256,
+                            num_experts_per_tok=16, moe_intermediate_size=1024,
+                            shared_intermediate_size=1024, sigma_x=1.0, sigma_w=0.015,
+                            sigma_router=0.02, routed_scaling_factor=1.0,
+                            note="M.1-faithful layer: top-16 of 256, routed scale 1.0, "
+                                 "T=16384, d=4096, F=Fs=1024"),
     "c5_decode": Workload("c5_decode", T=64, d_model=2048, num_experts=256,
                           num_experts_per_tok=8, moe_intermediate_size=512,
                           shared_intermediate_size=512, sigma_x=1.0, sigma_w=0.02,

@@ -31,7 +31,11 @@ MOE_FLAG_GEMM_PAIR = 16
 EXPORTED = ["moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
             "moe_read_device_status", "moe_selftest_bounded_wait", "moe_status_string",
             "moe_last_launch_count", "moe_profile_next_forward", "moe_prepare_down_f16",
-            "moe_logits_offset", "moe_permute_static"]
+            "moe_logits_offset", "moe_permute_static", "moe_route_masked",
+            "moe_forward_masked"]
+
+# Expert id of a (token, slot) pair that is not routed (a padding token).
+MOE_NOT_ROUTED = -1
 
 
 class MoeError(RuntimeError):
@@ -85,6 +89,11 @@ def lib():
         L.moe_forward.restype = ctypes.c_int
         L.moe_forward.argtypes = [D, ctypes.POINTER(moe_weights_t), P, P,
                                   ctypes.POINTER(moe_routing_t), P, ctypes.c_size_t, P]
+        L.moe_route_masked.restype = ctypes.c_int
+        L.moe_route_masked.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_forward_masked.restype = ctypes.c_int
+        L.moe_forward_masked.argtypes = [D, ctypes.POINTER(moe_weights_t), P, P, P,
+                                         ctypes.POINTER(moe_routing_t), P, ctypes.c_size_t, P]
         L.moe_read_device_status.restype = ctypes.c_int
         L.moe_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.moe_selftest_bounded_wait.restype = ctypes.c_int
@@ -149,9 +158,15 @@ def alloc_workspace(dims, device="cuda"):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def route(dims, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
-    _check(lib().moe_route(ctypes.byref(dims), _p(x), _p(w_router), _p(bias), _p(topk_idx),
-                           _p(topk_w), _p(ws), ws.numel(), _stream(stream)), "moe_route")
+def route(dims, x, w_router, bias, topk_idx, topk_w, ws, stream=None, token_mask=None):
+    """moe_route, or moe_route_masked when a [T] uint8 token_mask (0 = padding) is given."""
+    if token_mask is None:
+        _check(lib().moe_route(ctypes.byref(dims), _p(x), _p(w_router), _p(bias), _p(topk_idx),
+                               _p(topk_w), _p(ws), ws.numel(), _stream(stream)), "moe_route")
+    else:
+        _check(lib().moe_route_masked(ctypes.byref(dims), _p(x), _p(w_router), _p(bias),
+                                      _p(token_mask), _p(topk_idx), _p(topk_w), _p(ws),
+                                      ws.numel(), _stream(stream)), "moe_route_masked")
 
 
 def permute(dims, topk_idx, counts, offsets, perm, ws, x=None, x_perm=None, stream=None):
@@ -190,13 +205,19 @@ def routing_struct(R):
                                                      "perm")])
 
 
-def forward(dims, weights, x, y, routing, ws, stream=None):
-    """moe_forward on torch tensors; weights/routing are dicts of tensors (or prebuilt structs)."""
+def forward(dims, weights, x, y, routing, ws, stream=None, token_mask=None):
+    """moe_forward on torch tensors; weights/routing are dicts of tensors (or prebuilt structs).
+    With a [T] uint8 token_mask (0 = padding token) it calls moe_forward_masked."""
     ws_s = weights if isinstance(weights, moe_weights_t) else weights_struct(weights)
     r_s = routing if isinstance(routing, moe_routing_t) else routing_struct(routing)
-    _check(lib().moe_forward(ctypes.byref(dims), ctypes.byref(ws_s), _p(x), _p(y),
-                             ctypes.byref(r_s), _p(ws), ws.numel(), _stream(stream)),
-           "moe_forward")
+    if token_mask is None:
+        _check(lib().moe_forward(ctypes.byref(dims), ctypes.byref(ws_s), _p(x), _p(y),
+                                 ctypes.byref(r_s), _p(ws), ws.numel(), _stream(stream)),
+               "moe_forward")
+    else:
+        _check(lib().moe_forward_masked(ctypes.byref(dims), ctypes.byref(ws_s), _p(x),
+                                        _p(token_mask), _p(y), ctypes.byref(r_s), _p(ws),
+                                        ws.numel(), _stream(stream)), "moe_forward_masked")
 
 
 def alloc_routing(dims, device="cuda"):
@@ -278,7 +299,7 @@ class MoeLayer:
         self.routing = alloc_routing(d, self.device)
         self._r_struct = routing_struct(self.routing)
 
-    def forward(self, x, y=None, stream=None):
+    def forward(self, x, y=None, stream=None, token_mask=None):
         import torch
         T = x.shape[0]
         if T > self.max_tokens:
@@ -286,5 +307,5 @@ class MoeLayer:
         if y is None:
             y = torch.empty_like(x)
         d = self.dims(T)
-        forward(d, self._ws_struct, x, y, self._r_struct, self.ws, stream)
+        forward(d, self._ws_struct, x, y, self._r_struct, self.ws, stream, token_mask=token_mask)
         return y

@@ -109,6 +109,73 @@ def test_auto_engines_mixed_and_equal_to_forced(T):
         assert np.array_equal(y2.view(torch.int16).cpu().numpy(), bits), engine
 
 
+def _mask_run(w, h, dev, mask, flags=0):
+    import torch
+    dims = M.dims_for(w, flags=flags)
+    ws = M.alloc_workspace(dims)
+    ws.fill_(0xFF)
+    routing = M.alloc_routing(dims)
+    y = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
+    M.forward(dims, dev, dev["x"], y, routing, ws, token_mask=torch.from_numpy(mask).cuda())
+    torch.cuda.synchronize()
+    assert M.read_device_status(ws)[0] == 0
+    return y, routing
+
+
+@pytest.mark.parametrize("engine", [0] + ENGINES)
+@pytest.mark.parametrize("T,frac", [(300, 0.3), (1500, 0.5), (257, 1.0), (129, 0.0)])
+def test_padding_mask_forward(T, frac, engine):
+    """Padding tokens (mask 0) are not routed: MOE_NOT_ROUTED ids, zero weights, no expert
+    rows, y = shared expert only; the other tokens match the oracle as without a mask."""
+    w = I.get("c1_tiny").with_(T=T)
+    h, dev = _small(w)
+    rng = np.random.default_rng(T)
+    mask = (rng.random(T) >= frac).astype(np.uint8)
+    y, routing = _mask_run(w, h, dev, mask, engine)
+    ref = O.moe_forward(h["x"], h["w_router"], h["w_gate"], h["w_up"], h["w_down"], w.k,
+                        ws_gate=h["ws_gate"], ws_up=h["ws_up"], ws_down=h["ws_down"],
+                        routed_scaling_factor=w.routed_scaling_factor, token_mask=mask)
+    gidx = routing["topk_idx"].cpu().numpy()
+    gw = routing["topk_w"].cpu().numpy()
+    pad = mask == 0
+    assert np.all(gidx[pad] == M.MOE_NOT_ROUTED) and np.all(gw[pad] == 0.0)
+    keep = ~pad
+    if keep.any():
+        G.check_routing(gidx[keep], gw[keep], {"topk_idx": ref["topk_idx"][keep],
+                                               "topk_w": ref["topk_w"][keep],
+                                               "scores": ref["scores"][keep]}, w.k)
+    c, o, p = O.expert_order(gidx, w.E)
+    assert np.array_equal(routing["counts"].cpu().numpy(), c)
+    assert np.array_equal(routing["offsets"].cpu().numpy(), o)
+    assert np.array_equal(routing["perm"].cpu().numpy()[:o[-1]], p)
+    G.check_output(G.y_numpy(y), ref["y"], what=f"mask T={T} frac={frac}")
+
+
+def test_padding_mask_permute_and_gather():
+    import torch
+    w = I.get("c1_tiny").with_(T=500)
+    h, dev = _small(w)
+    ridx = O.route(h["x"], h["w_router"], None, w.k)[0]
+    ridx[::3] = M.MOE_NOT_ROUTED
+    dims = M.dims_for(w)
+    ws = M.alloc_workspace(dims)
+    idx = torch.from_numpy(ridx.astype(np.int32)).cuda()
+    counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((w.T * w.k,), -7, dtype=torch.int32, device="cuda")
+    xp = torch.zeros((w.T * w.k, w.d_model), dtype=torch.bfloat16, device="cuda")
+    M.permute(dims, idx, counts, offsets, perm, ws, x=dev["x"], x_perm=xp)
+    torch.cuda.synchronize()
+    assert M.read_device_status(ws)[0] == 0
+    c, o, p = O.expert_order(ridx, w.E)
+    n = int(o[-1])
+    assert np.array_equal(counts.cpu().numpy(), c) and np.array_equal(offsets.cpu().numpy(), o)
+    got = perm.cpu().numpy()
+    assert np.array_equal(got[:n], p) and np.all(got[n:] == -7)   # rows past offsets[E] untouched
+    xpn = P.to_numpy_bf16(xp)
+    assert np.array_equal(xpn[:n], h["x"][p // w.k]) and np.all(xpn[n:] == 0)
+
+
 def test_permute_materialised_gather_and_counts():
     import torch
     w = I.get("c1_tiny").with_(T=1000)
@@ -191,6 +258,18 @@ def test_small_expert_counts_and_k_extremes(E, k):
     ref = G.oracle_forward(w, h)
     G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, k)
     G.check_output(G.y_numpy(y), ref["y"], what=f"E={E},k={k}")
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+def test_m1_top16_unit_scale(engine):
+    """The M.1 configuration of the layer: top-16, routed scale 1.0 (ragged tiles, full oracle)."""
+    w = I.get("c1_tiny").with_(T=700, num_experts=64, num_experts_per_tok=16,
+                               routed_scaling_factor=1.0)
+    h, dev = _small(w)
+    y, routing, _ = G.run_forward(w, dev, flags=engine)
+    ref = G.oracle_forward(w, h)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
+    G.check_output(G.y_numpy(y), ref["y"], what="top-16, scale 1")
 
 
 @pytest.mark.parametrize("flags", [M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR])
@@ -334,7 +413,7 @@ def test_xs2_dims_multi_tile_full_oracle(engine):
 
 
 @pytest.mark.parametrize("name,n_sample", [("c2_xs2_small", 1024), ("c3_xs2_prefill_zipf", 1024),
-                                           ("c4_m1_width", 256)])
+                                           ("c4_m1_width", 256), ("c6_m1_top16", 256)])
 def test_full_size_workloads(name, n_sample):
     """Routing and counts on every token; y on a seeded sample of tokens."""
     w = I.get(name)

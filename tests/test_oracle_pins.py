@@ -301,6 +301,64 @@ def test_expert_order_against_brute_force():
             assert counts[e] == len(want)
 
 
+# ---------------------------------------------------------------- padding mask
+
+def test_padding_token_gets_shared_expert_only():
+    """A masked token is not routed: y_t equals the shared expert alone, evaluated in plain
+    Python; its slots carry the not-routed id and zero weight."""
+    rng = np.random.default_rng(21)
+    T, d, E, k, F, Fs = 9, 6, 5, 2, 3, 4
+    L = _rand_layer(rng, T, d, E, F, Fs, scale=0.6)
+    mask = np.array([1, 0, 1, 1, 0, 0, 1, 0, 1], dtype=np.uint8)
+    out = _fwd(L, k, token_mask=mask)
+    for t in np.nonzero(mask == 0)[0]:
+        s = _py_swiglu(L["x"][t].tolist(), L["ws_gate"].tolist(), L["ws_up"].tolist(),
+                       L["ws_down"].tolist())
+        assert np.allclose(out["y"][t], s, rtol=1e-12, atol=1e-14)
+        assert np.all(out["R"][t] == 0.0)
+        assert np.all(out["topk_idx"][t] == O.NOT_ROUTED) and np.all(out["topk_w"][t] == 0.0)
+    # the pin is sensitive: routing the masked tokens would change their outputs
+    full = _fwd(L, k)
+    assert not np.allclose(full["y"][mask == 0], out["y"][mask == 0])
+    # the same layer without a shared expert gives exact zeros for masked tokens
+    L0 = dict(L, ws_gate=None, ws_up=None, ws_down=None)
+    out0 = _fwd(L0, k, token_mask=mask)
+    assert np.all(out0["y"][mask == 0] == 0.0)
+
+
+def test_mask_leaves_other_tokens_unchanged():
+    """Tokens are independent, so masking some changes nothing for the others."""
+    rng = np.random.default_rng(22)
+    L = _rand_layer(rng, 40, 16, 8, 4, 4)
+    mask = (rng.random(40) < 0.6).astype(np.uint8)
+    a = _fwd(L, 3)
+    b = _fwd(L, 3, token_mask=mask)
+    keep = mask == 1
+    assert np.array_equal(b["y"][keep], a["y"][keep])
+    assert np.array_equal(b["topk_idx"][keep], a["topk_idx"][keep])
+    assert np.array_equal(b["topk_w"][keep], a["topk_w"][keep])
+    ones = _fwd(L, 3, token_mask=np.ones(40, np.uint8))
+    assert np.array_equal(ones["y"], a["y"])
+
+
+def test_expert_order_skips_unrouted_pairs():
+    """Counts cover the routed pairs only; perm is a bijection onto them, in (t, j) order."""
+    rng = np.random.default_rng(23)
+    T, E, k = 50, 8, 3
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    pad = rng.random(T) < 0.3
+    idx[pad] = O.NOT_ROUTED
+    counts, offsets, perm = O.expert_order(idx, E)
+    routed = [t * k + j for t in range(T) for j in range(k) if not pad[t]]
+    assert counts.sum() == len(routed) == k * int((~pad).sum()) and offsets[-1] == len(routed)
+    assert sorted(perm.tolist()) == routed
+    for e in range(E):
+        want = [t * k + j for t in range(T) for j in range(k) if idx[t, j] == e]
+        assert perm[offsets[e]:offsets[e + 1]].tolist() == want
+    none, noff, nperm = O.expert_order(np.full((4, 2), O.NOT_ROUTED), E)
+    assert none.sum() == 0 and noff[-1] == 0 and nperm.size == 0
+
+
 def test_bf16_widening_is_exact():
     bits = np.array([0x3F80, 0xBF80, 0x0000, 0x8000, 0x3E80, 0x4049, 0x7F7F, 0x0080], np.uint16)
     want = [1.0, -1.0, 0.0, -0.0, 0.25, 3.140625, 3.3895313892515355e38, 2.0 ** -126]
