@@ -79,20 +79,24 @@ def dist_env():
 
 # ----------------------------------------------------------------- work model
 
-def stage_work(w, counts):
-    """Algorithmic FLOPs and bytes per launch of each stage (no padding, no re-reads)."""
+def stage_work(w, counts, fp8=False):
+    """Algorithmic FLOPs and bytes per launch of each stage (no padding, no re-reads).
+    fp8: expert weights of one byte per element (plus one float32 scale per row)."""
     T, d, E, k, F, Fs = w.T, w.d_model, w.E, w.k, w.F, w.Fs
     touched = int((np.asarray(counts) > 0).sum())
     bf = 2
+    wb = 1 if fp8 else 2
     rows = T * k
     h_bytes = (rows * F + T * Fs) * bf
+    scales = 4 * (touched * (2 * F + d) + 2 * Fs + d) if fp8 else 0
     return {
         "router": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * bf + T * k * 8},
         "index": {"flops": 0, "bytes": T * k * 4 * 3 + E * 8},
         "gemm1_swiglu": {"flops": 4 * d * F * rows + 4 * d * Fs * T,
-                         "bytes": touched * 2 * F * d * bf + 2 * Fs * d * bf + T * d * bf + h_bytes},
+                         "bytes": touched * 2 * F * d * wb + 2 * Fs * d * wb + T * d * bf + h_bytes
+                         + scales},
         "gemm2_down_scale": {"flops": 2 * d * F * rows + 2 * d * Fs * T,
-                             "bytes": touched * d * F * bf + d * Fs * bf + h_bytes
+                             "bytes": touched * d * F * wb + d * Fs * wb + h_bytes
                              + T * (k + (1 if Fs else 0)) * d * bf},
         "combine": {"flops": 0, "bytes": T * (k + (1 if Fs else 0)) * d * bf + T * d * bf},
     }
@@ -170,8 +174,9 @@ def blas_threads():
         return 1
 
 
-def oracle_sample(w, h_small, n_tokens, seed=7):
-    """Time the oracle on n_tokens tokens of the workload (its x rows are regenerated on the host)."""
+def oracle_sample(w, h_small, n_tokens, seed=7, fp8=None):
+    """Time the oracle on n_tokens tokens of the workload (its x rows are regenerated on the host).
+    fp8: the oracle's FP8 expert weights (the FP8 forward is timed then)."""
     from oracle import moe_oracle as O
     from sparse_moe_layer_select_b200 import inputs as I
     rng = np.random.default_rng(seed)
@@ -179,10 +184,14 @@ def oracle_sample(w, h_small, n_tokens, seed=7):
     x = np.stack([I.generate_numpy((w.d_model,), w.seed, I.TID_X, w.sigma_x, start=int(r) * w.d_model)
                   for r in rows])
     t0 = time.perf_counter()
-    O.moe_forward(x, h_small["w_router"], h_small["w_gate"], h_small["w_up"], h_small["w_down"],
-                  w.k, router_bias=h_small.get("router_bias"), ws_gate=h_small.get("ws_gate"),
-                  ws_up=h_small.get("ws_up"), ws_down=h_small.get("ws_down"),
-                  routed_scaling_factor=w.routed_scaling_factor)
+    if fp8 is not None:
+        O.moe_forward_fp8(x, h_small["w_router"], fp8, w.k, router_bias=h_small.get("router_bias"),
+                          routed_scaling_factor=w.routed_scaling_factor)
+    else:
+        O.moe_forward(x, h_small["w_router"], h_small["w_gate"], h_small["w_up"], h_small["w_down"],
+                      w.k, router_bias=h_small.get("router_bias"), ws_gate=h_small.get("ws_gate"),
+                      ws_up=h_small.get("ws_up"), ws_down=h_small.get("ws_down"),
+                      routed_scaling_factor=w.routed_scaling_factor)
     return time.perf_counter() - t0, len(rows)
 
 
@@ -217,7 +226,7 @@ def run_ours(args):
     layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
                        max_tokens=w.T,
                        flags=(M.MOE_FLAG_GEMM_SINGLE_CTA if args.single_cta else 0)
-                       | (M.MOE_FLAG_GEMM_PAIR if args.pair else 0))
+                       | (M.MOE_FLAG_GEMM_PAIR if args.pair else 0), fp8=args.fp8)
     x_buf = dev["x"]
     y = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
@@ -351,7 +360,7 @@ def run_ours(args):
 
     peaks = load_peaks()
     counts = layer.routing["counts"].cpu().numpy()
-    work = stage_work(w, counts)
+    work = stage_work(w, counts, fp8=args.fp8)
     gemm_stages = ("gemm1_swiglu", "gemm2_down_scale")
     dom = max(gemm_stages, key=lambda s: stage_ms[s])
     t_dom = stage_ms[dom] / 1e3
@@ -385,7 +394,13 @@ def run_ours(args):
                        (None if v is None else v.cpu().numpy()))
                    for k, v in dev.items() if k != "x"}
         n = cpu_sample_size(w) if args.cpu_tokens <= 0 else args.cpu_tokens
-        secs, n = oracle_sample(w, h_small, n)
+        fp8 = None
+        if args.fp8:  # the oracle's own e4m3 weights (made once, not timed)
+            from oracle import moe_oracle as O
+            fp8 = O.quantize_experts_fp8(h_small["w_gate"], h_small["w_up"], h_small["w_down"],
+                                         h_small.get("ws_gate"), h_small.get("ws_up"),
+                                         h_small.get("ws_down"))
+        secs, n = oracle_sample(w, h_small, n, fp8=fp8)
         cpu = {"value": n / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{n} seeded tokens of the same workload through the float64 oracle "
                          f"({secs:.1f} s)"}
@@ -394,13 +409,17 @@ def run_ours(args):
         "metric": METRIC, "value": w.T * args.steps * world / elapsed, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox normal, bf16)",
+        "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16",
+        "data": "synthetic (seeded Philox normal, bf16)",
         "config": {"workload": w.name, "T": w.T, "d_model": w.d_model, "num_experts": w.E,
                    "num_experts_per_tok": w.k, "moe_intermediate_size": w.F,
                    "shared_intermediate_size": w.Fs, "routed_scaling_factor": w.routed_scaling_factor,
                    "router_bias": "zipf" if w.zipf_s else None, "parallelism": f"replicas x{world}",
-                   "gemm_engine": ("single-CTA M=128" if args.single_cta else "CTA-pair M=256"
-                                   if args.pair else "auto (CTA pairs when T*k >= 256*E)"),
+                   "gemm_engine": ("single-CTA M=128" if args.single_cta or args.fp8 else
+                                   "CTA-pair M=256" if args.pair else
+                                   "auto (gate/up single-CTA; down on CTA pairs when T*k >= 256*E)"),
+                   "experts": ("e4m3 weights, x and h with per-row fp32 scales" if args.fp8 else
+                               "bf16 weights (fp16 copy of W_down), fp16 h"),
                    "l2": "L2 flushed between steps" if flush else
                          f"inputs larger than L2 ({working_set / 1e9:.2f} GB resident)"},
         "roofline": roof, "expert_gemm": expert,
@@ -486,6 +505,8 @@ def main():
                     help="force the single-CTA (M=128) expert GEMM engine")
     ap.add_argument("--pair", action="store_true",
                     help="force the CTA-pair (M=256) expert GEMM engine")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 (e4m3) expert weights: moe_prepare_fp8 + moe_forward_fp8")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -88,6 +88,16 @@ typedef struct {
  * All choices give the same results. */
 #define MOE_FLAG_GEMM_SINGLE_CTA  8
 #define MOE_FLAG_GEMM_PAIR        16
+/* router_bias is a selection-only score bias (auxiliary-loss-free load
+ * balancing, Laguna-M.1-base spec sheet, Mixture of experts, "Load balancing"):
+ * the k experts are those with the largest sigmoid(logit) + bias, the weights
+ * are the unbiased sigmoid scores normalised over them.  Without the flag the
+ * bias is added to the logits (it then changes selection and weights alike).
+ * The per-expert loads (routing counts) are what a caller's bias update uses. */
+#define MOE_FLAG_BIAS_SELECTION_ONLY 32
+/* Size the workspace for moe_forward_fp8 (required by it; F and Fs must be
+ * multiples of 128). */
+#define MOE_FLAG_FP8_EXPERTS 64
 
 typedef struct {
     const void *w_router;      /* [E, d] bf16 */
@@ -101,6 +111,25 @@ typedef struct {
     const void *w_down_f16;    /* [E, d, F] fp16 copy of w_down (with MOE_FLAG_DOWN_F16) */
     const void *ws_down_f16;   /* [d, Fs] fp16 copy of ws_down (with MOE_FLAG_DOWN_F16) */
 } moe_weights_t;
+
+/* FP8 copies of the expert weights (moe_prepare_fp8 writes them; caller-owned
+ * device memory).  Every row of every expert matrix (one output channel) is
+ * stored as e4m3 codes with one float32 scale: s = amax(|row|) / 448 (1 for
+ * an all-zero row), code = e4m3(w / s), round to nearest even, saturating. */
+typedef struct {
+    void *w_gate;     /* [E, F, d] e4m3 */
+    void *w_up;       /* [E, F, d] e4m3 */
+    void *w_down;     /* [E, d, F] e4m3 */
+    float *s_gate;    /* [E * F] scale of each row of w_gate */
+    float *s_up;      /* [E * F] */
+    float *s_down;    /* [E * d] */
+    void *ws_gate;    /* [Fs, d] e4m3, NULL if Fs = 0 */
+    void *ws_up;      /* [Fs, d] */
+    void *ws_down;    /* [d, Fs] */
+    float *ss_gate;   /* [Fs] */
+    float *ss_up;     /* [Fs] */
+    float *ss_down;   /* [d] */
+} moe_fp8_weights_t;
 
 /* Routing outputs of moe_forward (caller-owned device memory, all required). */
 typedef struct {
@@ -178,6 +207,25 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *weigh
                               const void *x, const uint8_t *token_mask, void *y,
                               const moe_routing_t *routing, void *ws, size_t ws_bytes,
                               void *stream);
+
+/* One-time FP8 copies of the expert weights (bf16 `weights` in, `fp8` out;
+ * every pointer of `fp8` required, shared ones only if Fs > 0; scale arrays
+ * 16-byte aligned).  ws needs only 256 bytes (status header). */
+moe_status moe_prepare_fp8(const moe_dims_t *dims, const moe_weights_t *weights,
+                           const moe_fp8_weights_t *fp8, void *ws, size_t ws_bytes, void *stream);
+
+/* The layer with FP8 expert weights, for weight-bandwidth-bound (decode-sized)
+ * batches: routing as moe_forward (bf16 router); x is quantized per token
+ * (e4m3 codes, one float32 scale per row, as the weights); both expert GEMMs
+ * run on e4m3 operands (tcgen05 kind::f8f6f4, fp32 accumulation) with the
+ * row and column scales applied to the accumulator; h is held in fp16 and
+ * quantized per row before the down projection; the combine is moe_forward's.
+ * `weights` supplies the router (w_router, router_bias); dims->flags must
+ * include MOE_FLAG_FP8_EXPERTS (workspace size).  The expert GEMMs always run
+ * on single CTAs. */
+moe_status moe_forward_fp8(const moe_dims_t *dims, const moe_weights_t *weights,
+                           const moe_fp8_weights_t *fp8, const void *x, void *y,
+                           const moe_routing_t *routing, void *ws, size_t ws_bytes, void *stream);
 
 /* One-time preparation of the down projections for moe_forward: fp16 copies
  * w_down_f16 [E, d, F] and ws_down_f16 [d, Fs] (NULL if Fs = 0) of the bf16

@@ -37,6 +37,9 @@ Readings where the pages are silent:
 * Normalisation runs over the k selected experts only, with no epsilon.
 * A padding token (token mask 0) is not routed: no expert, weight 0, no row
   in the expert order; the shared expert still applies to it.
+* Auxiliary-loss-free balancing: a per-expert bias is added to the sigmoid
+  scores for the choice of the experts only; the weights stay the
+  normalised unbiased scores.
 
 Every function is a direct transcription of these definitions; numpy's
 matmul is the only library step.
@@ -105,19 +108,32 @@ def normalise(selected_scores, norm_topk_prob=True):
 NOT_ROUTED = -1
 
 
-def route(x, w_router, bias, k, norm_topk_prob=True, token_mask=None):
+def route(x, w_router, bias, k, norm_topk_prob=True, token_mask=None, selection_bias=None):
     """Sigmoid router with post-top-k normalisation.
 
     token_mask ([T], 0 = padding token) leaves padding tokens unrouted: their
     k slots get expert id NOT_ROUTED and weight 0 (Laguna training notes:
     padding tokens are best neither routed nor load-balanced).
 
+    selection_bias ([E]): the auxiliary-loss-free balancing variant (Laguna-
+    M.1-base spec sheet, Mixture of experts, "Load balancing: auxiliary-loss-
+    free").  The bias is added to the sigmoid scores for the choice of the k
+    experts only; the weights are the normalised unbiased scores.  (``bias``
+    and ``selection_bias`` are not combined: pass one of them.)
+
     Returns (topk_idx [T,k] int64, topk_w [T,k] f64, scores [T,E] f64, logits [T,E] f64).
+    For selection_bias, ``scores`` are the selection keys sigmoid(l) + b.
     """
     logits = router_logits(x, w_router, bias)
     scores = sigmoid(logits)
-    idx = select_topk(logits, k)
+    if selection_bias is None:
+        idx = select_topk(logits, k)
+    else:
+        keys = scores + np.asarray(selection_bias, dtype=np.float64)[None, :]
+        idx = select_topk(keys, k)
     sel = np.take_along_axis(scores, idx, axis=1)
+    if selection_bias is not None:
+        scores = keys
     w = normalise(sel, norm_topk_prob)
     if token_mask is not None:
         pad = np.asarray(token_mask) == 0
@@ -170,7 +186,7 @@ def expert_order(topk_idx, E):
 def moe_forward(x, w_router, w_gate, w_up, w_down, k, *, router_bias=None,
                 ws_gate=None, ws_up=None, ws_down=None,
                 routed_scaling_factor=2.5, norm_topk_prob=True, routing=None,
-                token_mask=None):
+                token_mask=None, selection_bias=None):
     """y_t = S(x_t) + scale * sum_j w_{t,j} * E_{e_{t,j}}(x_t), in float64.
 
     x: [T, d]; w_router: [E, d]; w_gate, w_up: [E, F, d]; w_down: [E, d, F];
@@ -186,7 +202,8 @@ def moe_forward(x, w_router, w_gate, w_up, w_down, k, *, router_bias=None,
     X = bf16_to_f64(x)
     T, d = X.shape
     if routing is None:
-        idx, w, scores, logits = route(x, w_router, router_bias, k, norm_topk_prob, token_mask)
+        idx, w, scores, logits = route(x, w_router, router_bias, k, norm_topk_prob, token_mask,
+                                       selection_bias)
     else:
         idx, w = routing
         scores = logits = None
@@ -207,3 +224,120 @@ def moe_forward(x, w_router, w_gate, w_up, w_down, k, *, router_bias=None,
     y = routed_scaling_factor * R + Sh
     return {"y": y, "R": R, "Sh": Sh, "topk_idx": idx, "topk_w": w,
             "scores": scores, "logits": logits}
+
+
+# ---------------------------------------------------------------- FP8 experts
+# FP8 expert weights for decode (the pages name FP8 deployment of the weights
+# but no scale layout; this build defines one): every row of every expert
+# matrix (an output channel), every token row of x and every row of h gets
+# its own float32 scale, s = amax(|row|) / 448 (s = 1 for an all-zero row),
+# and the row is stored as e4m3 codes q = e4m3(row / s), the division in
+# float32.  Products of codes are exact; the GEMMs accumulate in float32 and
+# apply the row and column scales to the accumulator.  h is held in fp16
+# before it is quantized, as in the 16-bit path.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code):
+    """Value of e4m3 codes (1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+    bits; exponent 0 is subnormal, 2^-6 * m/8; code S.1111.111 is NaN; no
+    infinities)."""
+    c = np.asarray(code, dtype=np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    v = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    v = np.where((e == 15) & (m == 7), np.nan, v)
+    return s * v
+
+
+def e4m3_round(v):
+    """Round float32 values to e4m3 codes: nearest representable value, ties to
+    the even code, magnitudes beyond 448 saturate to 448, NaN to the NaN code.
+
+    Returns uint8 codes.
+    """
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    neg = np.signbit(v)
+    a = np.abs(v)
+    nan = np.isnan(a)
+    a = np.where(nan, 0.0, a)
+    _, ex = np.frexp(a)                  # a = f * 2^ex, f in [0.5, 1): floor(log2 a) = ex - 1
+    e = np.maximum(ex - 1, -6)           # binade; below 2^-6 the subnormal quantum applies
+    q = np.ldexp(1.0, e - 3)             # spacing of the 3-bit mantissa in that binade
+    r = np.rint(a / q) * q               # round half to even (exact in float64)
+    r = np.minimum(r, E4M3_MAX)
+    # encode the (representable) magnitude
+    _, rx = np.frexp(r)
+    re = np.maximum(rx - 1, -6)
+    sub = r < 2.0 ** -6
+    mant = np.where(sub, np.rint(r / 2.0 ** -9), np.rint((r / np.ldexp(1.0, re) - 1.0) * 8.0))
+    code = np.where(sub, mant, ((re + 7) << 3) + mant).astype(np.int64)
+    code = np.where(nan, 0x7F, code) | np.where(neg, 0x80, 0)
+    return code.astype(np.uint8)
+
+
+def quantize_rows_e4m3(a):
+    """Per-row e4m3 quantization of a float32 matrix [..., K] (last axis = row).
+
+    Returns (codes uint8 [..., K], scales float32 [...]): s = amax / 448 in
+    float32 (1 for an all-zero row), codes = e4m3_round(float32(a / s)).
+    """
+    a = np.asarray(a, dtype=np.float32)
+    amax = np.max(np.abs(a), axis=-1)
+    s = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32), np.float32(1.0))
+    s = s.astype(np.float32)
+    codes = e4m3_round((a / s[..., None]).astype(np.float32))
+    return codes, s
+
+
+def dequantize_rows_e4m3(codes, scales):
+    return e4m3_value(codes) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def quantize_experts_fp8(w_gate, w_up, w_down, ws_gate=None, ws_up=None, ws_down=None):
+    """FP8 copies of the expert weights (bf16 bit patterns or floats in), one
+    scale per output row: gate/up [E, F] (rows of [E, F, d]), down [E, d]."""
+    f = lambda w: None if w is None else quantize_rows_e4m3(bf16_to_f64(w).astype(np.float32))
+    return {"gate": f(w_gate), "up": f(w_up), "down": f(w_down),
+            "s_gate": f(ws_gate), "s_up": f(ws_up), "s_down": f(ws_down)}
+
+
+def moe_forward_fp8(x, w_router, fp8, k, *, router_bias=None, routed_scaling_factor=2.5,
+                    norm_topk_prob=True):
+    """The layer with FP8 expert weights: routing as in ``route`` (bf16 router),
+    x quantized per token, h = SwiGLU(x_q W_g,q^T, x_q W_u,q^T) rounded to fp16 and
+    quantized per row, o = h_q W_d,q^T; combine as in ``moe_forward``.  Every
+    product of dequantized values is evaluated in float64."""
+    X = bf16_to_f64(x)
+    T, d = X.shape
+    idx, w, scores, logits = route(x, w_router, router_bias, k, norm_topk_prob)
+    xq = dequantize_rows_e4m3(*quantize_rows_e4m3(X.astype(np.float32)))
+
+    def expert(xrows, g, u, dn):
+        G = xrows @ dequantize_rows_e4m3(*g).T
+        U = xrows @ dequantize_rows_e4m3(*u).T
+        h = (silu(G) * U).astype(np.float16).astype(np.float32)
+        hq = dequantize_rows_e4m3(*quantize_rows_e4m3(h))
+        return hq @ dequantize_rows_e4m3(*dn).T
+
+    gq, gs = fp8["gate"]
+    uq, us = fp8["up"]
+    dq, ds = fp8["down"]
+    E = gq.shape[0]
+    contrib = np.zeros((T, k, d), dtype=np.float64)
+    for e in range(E):
+        tt, jj = np.nonzero(idx == e)
+        if tt.size == 0:
+            continue
+        o = expert(xq[tt], (gq[e], gs[e]), (uq[e], us[e]), (dq[e], ds[e]))
+        contrib[tt, jj, :] = w[tt, jj][:, None] * o
+    R = contrib.sum(axis=1)
+    if fp8["s_gate"] is not None:
+        Sh = expert(xq, fp8["s_gate"], fp8["s_up"], fp8["s_down"])
+    else:
+        Sh = np.zeros((T, d), dtype=np.float64)
+    y = routed_scaling_factor * R + Sh
+    return {"y": y, "R": R, "Sh": Sh, "topk_idx": idx, "topk_w": w, "scores": scores,
+            "logits": logits}

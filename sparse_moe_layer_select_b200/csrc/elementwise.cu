@@ -16,6 +16,7 @@
 // All three move 16-byte vectors with one thread per vector, grid-stride.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "kernels.h"
 #include "status.cuh"
@@ -38,40 +39,107 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// One thread per 8 output columns of one token: the k routed rows
-// o[inv[t*k + j]] (already scaled by routed_scaling_factor * w) are added in
-// slot order, then the shared-expert row, all in fp32; one RNE rounding to bf16.
-__global__ void __launch_bounds__(256)
+// One CTA per token row at a time (grid-stride over tokens), one thread per
+// 8 output columns: the k routed rows o[inv[t*k + j]] (already scaled by
+// routed_scaling_factor * w) are added in slot order, then the shared-expert
+// row, all in fp32; one RNE rounding to bf16.  The token's k row indices are
+// staged in shared memory one token ahead, so a thread's row loads never
+// wait on an index load.
+constexpr int kCombineThreads = 256;
+
+template <int KMAX>  // k <= KMAX
+__global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint4 *__restrict__ o, const uint4 *__restrict__ s_out,
                    const int32_t *__restrict__ inv, int T, int k, int vec_per_row,
                    uint4 *__restrict__ y) {
-  const size_t total = static_cast<size_t>(T) * vec_per_row;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t t = i / vec_per_row;
-    const size_t c = i - t * vec_per_row;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    auto add = [&](const uint4 v) {
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  __shared__ int rows[2][16];
+  int t = blockIdx.x;
+  if (threadIdx.x < k && t < T) rows[0][threadIdx.x] = inv[static_cast<size_t>(t) * k + threadIdx.x];
+  __syncthreads();
+  int buf = 0;
+  for (; t < T; t += gridDim.x) {
+    const int tn = t + gridDim.x;
+    if (threadIdx.x < k && tn < T)
+      rows[buf ^ 1][threadIdx.x] = inv[static_cast<size_t>(tn) * k + threadIdx.x];
+    for (int c = threadIdx.x; c < vec_per_row; c += kCombineThreads) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      auto add = [&](const uint4 v) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[q]));
+          acc[2 * q] += f.x;
+          acc[2 * q + 1] += f.y;
+        }
+      };
+      uint4 v[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {  // all row loads first (independent)
+        const int r = j < k ? rows[buf][j] : -1;
+        v[j] = r >= 0 ? o[static_cast<size_t>(r) * vec_per_row + c] : make_uint4(0, 0, 0, 0);
+      }
+      const uint4 sv = s_out ? s_out[static_cast<size_t>(t) * vec_per_row + c] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && rows[buf][j] >= 0) add(v[j]);
+      if (s_out) add(sv);
+      uint32_t out[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[q]));
-        acc[2 * q] += f.x;
-        acc[2 * q + 1] += f.y;
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+        out[q] = *reinterpret_cast<uint32_t *>(&b2);
       }
-    };
-    for (int j = 0; j < k; ++j) {
-      const int r = inv[t * k + j];
-      if (r >= 0) add(o[static_cast<size_t>(r) * vec_per_row + c]);
+      y[static_cast<size_t>(t) * vec_per_row + c] = make_uint4(out[0], out[1], out[2], out[3]);
     }
-    if (s_out) add(s_out[t * vec_per_row + c]);
-    uint32_t out[4];
+    __syncthreads();  // next token's indices staged; this token's reads done
+    buf ^= 1;
+  }
+}
+
+// Per-row e4m3 quantization (FP8 experts): one warp per row of K 16-bit
+// values (bf16 or fp16 by `is_f16`), s = amax / 448 (1 for an all-zero
+// row), codes = e4m3(v / s) with round to nearest even and saturation to
+// +-448; the division is the IEEE float32 one.  Rows from *n_valid on (if
+// given) are skipped.
+__global__ void __launch_bounds__(256)
+    quant_rows_e4m3_kernel(const uint16_t *__restrict__ src, int is_f16, int rows,
+                           const int32_t *__restrict__ n_valid, int K,
+                           uint8_t *__restrict__ codes, float *__restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int nrows = n_valid ? min(rows, *n_valid) : rows;
+  auto to_f32 = [&](uint16_t b) -> float {
+    return is_f16 ? __half2float(__ushort_as_half(b)) : __uint_as_float(static_cast<uint32_t>(b) << 16);
+  };
+  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < nrows; r += warps) {
+    const uint4 *row = reinterpret_cast<const uint4 *>(src + static_cast<size_t>(r) * K);
+    float amax = 0.f;
+    for (int c = lane; c < K / 8; c += 32) {
+      const uint4 v = row[c];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-      out[q] = *reinterpret_cast<uint32_t *>(&b2);
+      for (int q = 0; q < 4; ++q)
+        amax = fmaxf(amax, fmaxf(fabsf(to_f32(w[q] & 0xffffu)), fabsf(to_f32(w[q] >> 16))));
     }
-    y[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    // amax >= 0: its bits order as unsigned integers
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    uint2 *out = reinterpret_cast<uint2 *>(codes + static_cast<size_t>(r) * K);
+    for (int c = lane; c < K / 8; c += 32) {
+      const uint4 v = row[c];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = __nv_cvt_float_to_fp8(__fdiv_rn(to_f32(w[q] & 0xffffu), scale),
+                                                  __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float_to_fp8(__fdiv_rn(to_f32(w[q] >> 16), scale),
+                                                  __NV_SATFINITE, __NV_E4M3);
+        packed[q >> 1] |= (lo | (hi << 8)) << (16 * (q & 1));
+      }
+      out[c] = make_uint2(packed[0], packed[1]);
+    }
+    if (lane == 0) scales[r] = scale;
   }
 }
 
@@ -141,10 +209,17 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, const int
 cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32_t *inv, int T,
                            int k, int d, uint16_t *y, cudaStream_t s) {
   const int vpr = d / 8;
-  const size_t work = static_cast<size_t>(T) * vpr;
-  combine_kernel<<<grid_for(work, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(o),
-                                                     reinterpret_cast<const uint4 *>(s_out), inv,
-                                                     T, k, vpr, reinterpret_cast<uint4 *>(y));
+  const size_t work = static_cast<size_t>(T) * kCombineThreads;  // one CTA per token
+  const int grid = grid_for(work, kCombineThreads);
+  const uint4 *o4 = reinterpret_cast<const uint4 *>(o);
+  const uint4 *s4 = reinterpret_cast<const uint4 *>(s_out);
+  uint4 *y4 = reinterpret_cast<uint4 *>(y);
+  if (k <= 4)
+    combine_kernel<4><<<grid, kCombineThreads, 0, s>>>(o4, s4, inv, T, k, vpr, y4);
+  else if (k <= 8)
+    combine_kernel<8><<<grid, kCombineThreads, 0, s>>>(o4, s4, inv, T, k, vpr, y4);
+  else
+    combine_kernel<16><<<grid, kCombineThreads, 0, s>>>(o4, s4, inv, T, k, vpr, y4);
   return cudaGetLastError();
 }
 
@@ -159,6 +234,16 @@ cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int
 
 cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s) {
   selftest_wait_kernel<<<1, 32, 0, s>>>(status, limit_cycles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows_e4m3(const uint16_t *src, bool is_f16, int rows,
+                                  const int32_t *n_valid, int K, uint8_t *codes, float *scales,
+                                  cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const size_t threads = static_cast<size_t>(rows) * 32;
+  quant_rows_e4m3_kernel<<<grid_for(threads, 256), 256, 0, s>>>(src, is_f16 ? 1 : 0, rows, n_valid,
+                                                               K, codes, scales);
   return cudaGetLastError();
 }
 

@@ -33,19 +33,22 @@ struct Item {
 // between two items holds no global-load round trip.
 template <int MODE>
 __device__ __forceinline__ int4 load_tile_rec(const GemmParams &p, int item, int n_items) {
-  if (MODE == MODE_ROUTER || item >= n_items) return make_int4(0, 0, 0, 0);
+  if ((MODE & 3) == MODE_ROUTER || item >= n_items) return make_int4(0, 0, 0, 0);
   return *reinterpret_cast<const int4 *>(&p.tiles[item / p.n_ntiles]);
 }
 
 template <int MODE>
 __device__ __forceinline__ Item decode_tile(const GemmParams &p, int item, int4 t) {
+  constexpr int BASE = MODE & 3;
+  constexpr int KB = stage_k(MODE);
   Item it;
-  if (MODE == MODE_ROUTER) {
+  if (BASE == MODE_ROUTER) {  // item = (128-token tile, block of n_tile experts)
+    const int ti = item / p.n_ntiles;
     it.group = -1;
-    it.row0 = item * kBlockM;
+    it.row0 = ti * kBlockM;
     it.nrows = min(kBlockM, p.T - it.row0);
-    it.j = 0;
-    it.nk = p.d / kBlockK;
+    it.j = item - ti * p.n_ntiles;
+    it.nk = p.d / KB;
     it.skip = false;
     return it;
   }
@@ -55,13 +58,13 @@ __device__ __forceinline__ Item decode_tile(const GemmParams &p, int item, int4 
   it.row0 = t.y;
   it.nrows = t.z;
   const bool shared = it.group == p.E;
-  if (MODE == MODE_GEMM1) {
+  if (BASE == MODE_GEMM1) {
     const int width = shared ? p.Fs : p.F;
     it.skip = it.j * p.n_half >= width;
-    it.nk = p.d / kBlockK;
+    it.nk = p.d / KB;
   } else {
     it.skip = false;
-    it.nk = (shared ? p.Fs : p.F) / kBlockK;
+    it.nk = (shared ? p.Fs : p.F) / KB;
   }
   return it;
 }
@@ -153,20 +156,25 @@ __device__ __forceinline__ void gather_tokens(const GemmParams &p, const Item &i
 
 // Issue this warp's share of one stage's A gather (GEMM1): the k-block
 // starting at column kc, into the 128B-swizzled A buffer at a_dst; the
-// lanes' completions arrive on bar (one arrival per lane).
+// lanes' completions arrive on bar (one arrival per lane).  Rows are bf16 x,
+// or e4m3 xq for MODE_F8 (128 bytes of a row either way).
+template <int MODE>
 __device__ __forceinline__ void gather_a_stage(const GemmParams &p, const int (&tok)[kGatherGroups],
                                                int lane, int gw, uint8_t *a_dst, uint64_t *bar,
                                                int kc) {
+  constexpr int ES = elem_bytes(MODE);
   // 128-byte swizzle: chunk c of row r sits at chunk (c ^ (r & 7)).
   const int c = lane & 7;
   const uint32_t a_base = smem_u32(a_dst);
-  const char *xsrc = reinterpret_cast<const char *>(p.x) + kc * 2 + c * 16;
+  const char *xsrc = ((MODE & MODE_F8) ? reinterpret_cast<const char *>(p.xq)
+                                       : reinterpret_cast<const char *>(p.x)) +
+                     kc * ES + c * 16;
 #pragma unroll
   for (int i = 0; i < kGatherGroups; ++i) {
     const int r = gw * kGatherRows + (lane >> 3) + 4 * i;
     if (tok[i] >= 0)
       cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4),
-                  xsrc + static_cast<size_t>(tok[i]) * p.d * 2);
+                  xsrc + static_cast<size_t>(tok[i]) * p.d * ES);
   }
   cp_async_arrive_noinc(bar);
 }
@@ -183,24 +191,25 @@ __device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item 
                                                        uint32_t taddr, int row_local,
                                                        const float *bias_s) {
   const bool valid = row_local < it.nrows;
-  float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E;
-  for (int c = 0; c < p.E; c += 32) {
+  const int e0 = it.j * p.n_tile;  // this item's block of experts
+  float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E + e0;
+  const float *b = bias_s + e0;
+  for (int c = 0; c < p.n_tile; c += 32) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(taddr + c, r);
     tmem_ld_wait();
     if (valid) {
-      if (c + 32 <= p.E) {
+      if (c + 32 <= p.n_tile) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
           *reinterpret_cast<float4 *>(dst + c + i) =
-              make_float4(__uint_as_float(r[i]) + bias_s[c + i],
-                          __uint_as_float(r[i + 1]) + bias_s[c + i + 1],
-                          __uint_as_float(r[i + 2]) + bias_s[c + i + 2],
-                          __uint_as_float(r[i + 3]) + bias_s[c + i + 3]);
+              make_float4(__uint_as_float(r[i]) + b[c + i], __uint_as_float(r[i + 1]) + b[c + i + 1],
+                          __uint_as_float(r[i + 2]) + b[c + i + 2],
+                          __uint_as_float(r[i + 3]) + b[c + i + 3]);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (c + i < p.E) dst[c + i] = __uint_as_float(r[i]) + bias_s[c + i];
+          if (c + i < p.n_tile) dst[c + i] = __uint_as_float(r[i]) + b[c + i];
       }
     }
   }
@@ -249,8 +258,24 @@ __device__ __forceinline__ float swiglu(float g, float u) {
   return __fdividef(g, 1.f + __expf(-g)) * u;
 }
 
+// acc[i] *= rs * col_scale[i] for N accumulator columns (MODE_F8 epilogues:
+// token or h row scale rs, weight-row scale of each column).
+template <int N>
+__device__ __forceinline__ void scale_cols(uint32_t (&acc)[N], float rs, const float *col_scale) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    const float4 c = *reinterpret_cast<const float4 *>(col_scale + i);
+    acc[i] = __float_as_uint(__uint_as_float(acc[i]) * rs * c.x);
+    acc[i + 1] = __float_as_uint(__uint_as_float(acc[i + 1]) * rs * c.y);
+    acc[i + 2] = __float_as_uint(__uint_as_float(acc[i + 2]) * rs * c.z);
+    acc[i + 3] = __float_as_uint(__uint_as_float(acc[i + 3]) * rs * c.w);
+  }
+}
+
 // GEMM1 epilogue: h = silu(gate) * up for this thread's row, fp16, 64
-// columns per store box.
+// columns per store box.  F8: the accumulators are first multiplied by the
+// token row's scale and each column's weight-row scale.
+template <bool F8>
 __device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item &it,
                                                 uint32_t taddr, int row_local, EpiStage &st,
                                                 const CUtensorMap *tm_h, const CUtensorMap *tm_hsh) {
@@ -262,21 +287,35 @@ __device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item 
   uint16_t *row_dst = shared ? p.h_shared + static_cast<size_t>(it.row0 + row_local) * p.Fs
                              : p.h + static_cast<size_t>(it.row0 + row_local) * p.F;
   const int col0 = it.j * p.n_half;
+  float rs = 1.f;
+  const float *sg = nullptr, *su = nullptr;
+  if (F8) {
+    if (valid) {
+      const int tok = shared ? it.row0 + row_local : p.perm[it.row0 + row_local] / p.k;
+      rs = p.sx[tok];
+    }
+    sg = (shared ? p.sb0_sh : p.sb0 + static_cast<size_t>(it.group) * p.F) + col0;
+    su = (shared ? p.sb1_sh : p.sb1 + static_cast<size_t>(it.group) * p.F) + col0;
+  }
   float amax = 0.f;
   for (int cb = 0; cb < p.n_half; cb += 64) {
     uint32_t packed[32];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t g[32], u[32];
-      tmem_ld_32x32b_x32(taddr + cb + 32 * half, g);
-      tmem_ld_32x32b_x32(taddr + p.n_half + cb + 32 * half, u);
+    for (int qu = 0; qu < 4; ++qu) {  // 16 gate and 16 up columns at a time
+      uint32_t g[16], u[16];
+      tmem_ld_32x32b_x16(taddr + cb + 16 * qu, g);
+      tmem_ld_32x32b_x16(taddr + p.n_half + cb + 16 * qu, u);
       tmem_ld_wait();
+      if (F8) {
+        scale_cols<16>(g, rs, sg + cb + 16 * qu);
+        scale_cols<16>(u, rs, su + cb + 16 * qu);
+      }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 8; ++i) {
         const float h0 = swiglu(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
         const float h1 = swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
         amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
-        packed[16 * half + i] = pack_f16x2(h0, h1);
+        packed[8 * qu + i] = pack_f16x2(h0, h1);
       }
     }
     store_box(st, packed, lane, full_box, valid, shared ? tm_hsh : tm_h, col0 + cb,
@@ -288,6 +327,7 @@ __device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item 
 // GEMM2 epilogue: routed rows -> routed_scale * w * o into o_out (expert-order
 // rows); shared-expert rows -> o into s_out (token rows).  fp16, 64 columns
 // per store box.
+template <bool F8>
 __device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &it, uint32_t taddr,
                                               int row_local, EpiStage &st,
                                               const CUtensorMap *tm_o, const CUtensorMap *tm_s) {
@@ -300,20 +340,26 @@ __device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &i
   if (valid && !shared) scale = p.routed_scale * p.topk_w[p.perm[it.row0 + row_local]];
   uint16_t *row_dst = (shared ? p.s_out : p.o_out) + static_cast<size_t>(it.row0 + row_local) * p.d;
   const int col0 = it.j * p.n_tile;
+  const float *sd = nullptr;
+  if (F8) {  // h row scale, then each column's weight-row scale
+    if (valid) scale *= shared ? p.sa_sh[it.row0 + row_local] : p.sa[it.row0 + row_local];
+    sd = (shared ? p.sb0_sh : p.sb0 + static_cast<size_t>(it.group) * p.d) + col0;
+  }
   float amax = 0.f;
   for (int cb = 0; cb < p.n_tile; cb += 64) {
     uint32_t packed[32];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(taddr + cb + 32 * half, r);
+    for (int qu = 0; qu < 4; ++qu) {  // 16 columns at a time
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(taddr + cb + 16 * qu, r);
       tmem_ld_wait();
+      if (F8) scale_cols<16>(r, 1.f, sd + cb + 16 * qu);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 8; ++i) {
         const float v0 = __uint_as_float(r[2 * i]) * scale;
         const float v1 = __uint_as_float(r[2 * i + 1]) * scale;
         amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));
-        packed[16 * half + i] = pack_f16x2(v0, v1);
+        packed[8 * qu + i] = pack_f16x2(v0, v1);
       }
     }
     store_box(st, packed, lane, full_box, valid, shared ? tm_s : tm_o, col0 + cb,

@@ -16,9 +16,10 @@
 //
 // The (t, j) entries are cut into chunks of kIndexChunk = 4096, one CTA of 8
 // warps per chunk, each warp owning 512 consecutive entries:
-//   index_hist_kernel     per-chunk expert histogram
-//   index_scan_kernel     one CTA: per-expert sums over chunks, exclusive
-//                         scan over experts, chunk bases, tile list
+//   index_hist_scan_kernel  per-chunk expert histogram; the CTA that
+//                         finishes last then sums per expert over chunks,
+//                         scans over experts, writes the chunk bases and the
+//                         tile lists
 //   index_scatter_kernel  per chunk: per-warp histograms and their scan give
 //                         each warp its first row per expert; each warp then
 //                         places its entries in order, ranks among equal
@@ -76,17 +77,24 @@ __device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int base = chunk * kIndexChunk + warp * kSub;
-  int *hw = h + warp * E;
-  for (int r = lane; r < kSub; r += 32) {
-    const int i = base + r;
-    if (i >= n) break;
-    const int e = topk_idx[i];
-    if (e == kNotRouted) continue;
-    if (e < 0 || e >= E) {
-      if (status) record_status(status, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
-      continue;
+  if (warp < kIdxWarps) {  // (a larger CTA's other warps only clear and wait)
+    int *hw = h + warp * E;
+    int ids[kSub / 32];  // all loads first: one memory round trip per warp
+#pragma unroll
+    for (int q = 0; q < kSub / 32; ++q) {
+      const int i = base + q * 32 + lane;
+      ids[q] = i < n ? topk_idx[i] : kNotRouted;
     }
-    atomicAdd(&hw[e], 1);
+#pragma unroll
+    for (int q = 0; q < kSub / 32; ++q) {
+      const int e = ids[q];
+      if (e == kNotRouted) continue;
+      if (e < 0 || e >= E) {
+        if (status) record_status(status, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
+        continue;
+      }
+      atomicAdd(&hw[e], 1);
+    }
   }
   __syncthreads();
 }
@@ -101,14 +109,19 @@ __device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ t
   const unsigned lt = (1u << lane) - 1u;
   int *fw = fill + warp * E;
   const int base = chunk * kIndexChunk + warp * kSub;
-  for (int r = 0; r < kSub; r += 32) {
+  int ids[kSub / 32];  // all loads first: one memory round trip per warp
+#pragma unroll
+  for (int q = 0; q < kSub / 32; ++q) {
+    const int i = base + q * 32 + lane;
+    ids[q] = i < n ? topk_idx[i] : -1;
+  }
+#pragma unroll
+  for (int q = 0; q < kSub / 32; ++q) {
+    const int r = q * 32;
     const int i = base + r + lane;
     if (base + r >= n) break;  // warp-uniform
-    int e = -1;
-    if (i < n) {
-      e = topk_idx[i];
-      if (e < 0 || e >= E) e = -1;
-    }
+    int e = ids[q];
+    if (e < 0 || e >= E) e = -1;
     const unsigned m = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(m & lt);
     if (e >= 0) {
@@ -137,19 +150,6 @@ __device__ __forceinline__ void warp_bases(int E, const int *chunk_base_e, int *
     }
   }
   __syncthreads();
-}
-
-__global__ void __launch_bounds__(kIdxWarps * 32)
-    index_hist_kernel(const int32_t *__restrict__ topk_idx, int n, int E,
-                      int *__restrict__ chunk_hist, int *status) {
-  __shared__ int h[kIdxWarps * kMaxE];
-  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, status);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int s = 0;
-#pragma unroll
-    for (int w = 0; w < kIdxWarps; ++w) s += h[w * E + e];
-    chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = s;
-  }
 }
 
 // One tile list: blocks of at most tile_rows rows of each expert in expert
@@ -197,11 +197,11 @@ __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int
     for (; c + 8 <= nchunks; c += 8) {  // eight independent loads in flight
       int v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = chunk_hist[static_cast<size_t>(c + q) * E + e];
+      for (int q = 0; q < 8; ++q) v[q] = __ldcg(&chunk_hist[static_cast<size_t>(c + q) * E + e]);
 #pragma unroll
       for (int q = 0; q < 8; ++q) cnt += v[q];
     }
-    for (; c < nchunks; ++c) cnt += chunk_hist[static_cast<size_t>(c) * E + e];
+    for (; c < nchunks; ++c) cnt += __ldcg(&chunk_hist[static_cast<size_t>(c) * E + e]);
   }
   const int off = block_exclusive_scan(e < E ? cnt : 0, warp_sums, &totals[0]);
   if (e < E) {
@@ -212,7 +212,7 @@ __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int
     for (; c + 8 <= nchunks; c += 8) {
       int v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = chunk_hist[static_cast<size_t>(c + q) * E + e];
+      for (int q = 0; q < 8; ++q) v[q] = __ldcg(&chunk_hist[static_cast<size_t>(c + q) * E + e]);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         chunk_hist[static_cast<size_t>(c + q) * E + e] = run;  // chunk base row of expert e
@@ -220,7 +220,7 @@ __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int
       }
     }
     for (; c < nchunks; ++c) {
-      const int v = chunk_hist[static_cast<size_t>(c) * E + e];
+      const int v = __ldcg(&chunk_hist[static_cast<size_t>(c) * E + e]);
       chunk_hist[static_cast<size_t>(c) * E + e] = run;
       run += v;
     }
@@ -237,13 +237,33 @@ __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int
   }
 }
 
+// Per-chunk histograms; the CTA that finishes last (a ticket counter in the
+// workspace header, zeroed by every call) then runs the scan and writes the
+// tile lists.  Nothing waits: the other CTAs simply exit.
 __global__ void __launch_bounds__(512)
-    index_scan_kernel(int *__restrict__ chunk_hist, int nchunks, int E, int T, int with_shared,
-                      int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                      Tile *__restrict__ tiles, Tile *__restrict__ tiles_pair,
-                      int *__restrict__ header) {
+    index_hist_scan_kernel(const int32_t *__restrict__ topk_idx, int n, int E, int nchunks, int T,
+                           int with_shared, int *__restrict__ chunk_hist,
+                           int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                           Tile *__restrict__ tiles, Tile *__restrict__ tiles_pair,
+                           int *__restrict__ header) {
+  __shared__ int h[kIdxWarps * kMaxE];
   __shared__ int warp_sums[32];
   __shared__ int totals[3];
+  __shared__ int ticket;
+  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, header);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) s += h[w * E + e];
+    chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = s;
+  }
+  __threadfence();  // this chunk's totals are visible before the ticket is taken
+  __syncthreads();
+  if (threadIdx.x == 0)
+    ticket = atomicAdd(&reinterpret_cast<WsHeader *>(header)->index_done, 1);
+  __syncthreads();
+  if (ticket != nchunks - 1) return;
+  __threadfence();
   scan_and_tiles(chunk_hist, nchunks, E, T, with_shared, counts, offsets, tiles, tiles_pair,
                  header, warp_sums, totals);
 }
@@ -270,25 +290,7 @@ __global__ void __launch_bounds__(512)
   __shared__ int warp_sums[32];
   __shared__ int totals[3];
   const int warp = threadIdx.x >> 5;
-  // histogram by the first eight warps (the others only clear and wait)
-  for (int i = threadIdx.x; i < kIdxWarps * E; i += blockDim.x) h[i] = 0;
-  __syncthreads();
-  if (warp < kIdxWarps) {
-    const int lane = threadIdx.x & 31;
-    int *hw = h + warp * E;
-    for (int r = lane; r < kSub; r += 32) {
-      const int i = warp * kSub + r;
-      if (i >= n) break;
-      const int e = topk_idx[i];
-      if (e == kNotRouted) continue;
-      if (e < 0 || e >= E) {
-        record_status(header, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_EXPERT_ID);
-        continue;
-      }
-      atomicAdd(&hw[e], 1);
-    }
-  }
-  __syncthreads();
+  chunk_warp_hist(topk_idx, n, E, 0, h, header);  // warps 0..7
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int s = 0;
 #pragma unroll
@@ -317,15 +319,13 @@ cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_
     *launches += 1;
     return cudaGetLastError();
   }
-  index_hist_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, status);
+  index_hist_scan_kernel<<<nchunks, 512, 0, s>>>(topk_idx, n, E, nchunks, T, with_shared,
+                                                  chunk_hist, counts, offsets, tiles, tiles_pair,
+                                                  status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  index_scan_kernel<<<1, 512, 0, s>>>(chunk_hist, nchunks, E, T, with_shared, counts, offsets,
-                                      tiles, tiles_pair, status);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
   index_scatter_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm, inv);
-  *launches += 3;
+  *launches += 2;
   return cudaGetLastError();
 }
 

@@ -23,7 +23,17 @@ constexpr int kBlockK = 64;         // K elements per pipeline stage (one 128-by
 constexpr int kStages = 4;          // shared-memory pipeline depth
 constexpr int kIndexChunk = 4096;   // (token, slot) entries per index-builder chunk
 
-enum GemmMode : int { MODE_ROUTER = 0, MODE_GEMM1 = 1, MODE_GEMM2 = 2 };
+enum GemmMode : int {
+  MODE_ROUTER = 0,
+  MODE_GEMM1 = 1,
+  MODE_GEMM2 = 2,
+  MODE_F8 = 4,  // mode bit: e4m3 operands (tcgen05 kind::f8f6f4), per-row scales
+  MODE_GEMM1_F8 = MODE_GEMM1 | MODE_F8,
+  MODE_GEMM2_F8 = MODE_GEMM2 | MODE_F8,
+};
+// K elements of one pipeline stage: one 128-byte swizzle row of A and B.
+__host__ __device__ constexpr int stage_k(int mode) { return (mode & MODE_F8) ? 128 : kBlockK; }
+__host__ __device__ constexpr int elem_bytes(int mode) { return (mode & MODE_F8) ? 1 : 2; }
 
 struct GemmParams {
   int *status;              // workspace header (status word)
@@ -47,6 +57,13 @@ struct GemmParams {
   uint16_t *o_out;          // GEMM2 out: [T*k, d] fp16, routed_scale * w * o (expert-order rows)
   uint16_t *s_out;          // GEMM2 out: [T, d] fp16 shared-expert output
   unsigned long long *trace;  // pipeline timestamps (builds with MOE_TRACE only), or null
+  // MODE_F8 launches: e4m3 codes and float32 scales (one per row)
+  const uint8_t *xq;        // GEMM1: token rows [T, d] e4m3 (gathered by cp.async)
+  const float *sx;          // GEMM1: scale of each token row of xq
+  const float *sa;          // GEMM2: scale of each expert-order row of h
+  const float *sa_sh;       // GEMM2: scale of each token row of h_shared
+  const float *sb0, *sb1;   // scales of the B rows (gate, up | down) of the routed experts
+  const float *sb0_sh, *sb1_sh;  // same for the shared expert
 };
 
 // Pipeline trace layout (MOE_TRACE builds): trace[(cta * kTraceKinds + kind) * kTraceN + n].
@@ -83,11 +100,12 @@ cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const 
 constexpr int kNotRouted = -1;
 
 // token_mask (optional, [T]): 0 = padding token, which gets kNotRouted ids
-// and zero weights.
+// and zero weights.  bias: the logit bias (its float64 refinement adds it);
+// sel_bias: a selection-only bias on the sigmoid scores (one of the two).
 cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
-                                 const float *bias, const uint8_t *token_mask, int T, int d, int E,
-                                 int k, int norm_topk, int32_t *topk_idx, float *topk_w,
-                                 cudaStream_t s);
+                                 const float *bias, const float *sel_bias,
+                                 const uint8_t *token_mask, int T, int d, int E, int k,
+                                 int norm_topk, int32_t *topk_idx, float *topk_w, cudaStream_t s);
 
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
@@ -100,6 +118,11 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, const int
 // with inv < 0 (not routed) are skipped.
 cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32_t *inv, int T,
                            int k, int d, uint16_t *y, cudaStream_t s);
+// Per-row e4m3 codes and float32 scales of a [rows, K] bf16 (or fp16) matrix;
+// K % 8 == 0; rows from *n_valid on (if given) are skipped.
+cudaError_t launch_quant_rows_e4m3(const uint16_t *src, bool is_f16, int rows,
+                                  const int32_t *n_valid, int K, uint8_t *codes, float *scales,
+                                  cudaStream_t s);
 cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int *status,
                                cudaStream_t s);
 cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s);

@@ -93,12 +93,14 @@ int pair_clusters() {
   return (dev >= 0 && dev < kMaxDevices) ? g_pair_clusters[dev] : 0;
 }
 
-// 2-D 16-bit tensor [rows, cols] (row-major), 128-byte swizzle, box 64 x box_rows.
+// 2-D tensor [rows, cols] (row-major), 128-byte swizzle, box of one 128-byte
+// row segment (64 16-bit or 128 8-bit elements) x box_rows.
 bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  const uint64_t esize = dtype == CU_TENSOR_MAP_DATA_TYPE_UINT8 ? 1 : 2;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBlockK), box_rows};
+  cuuint64_t strides[1] = {cols * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), box_rows};
   cuuint32_t es[2] = {1, 1};
   CUresult r = g_encode(m, dtype, 2, const_cast<void *>(ptr), dims,
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -115,8 +117,9 @@ struct Dims {
 };
 
 struct WsLayout {
-  size_t header, chunk_hist, tiles, tiles_pair, logits, inv, h, h_sh, o, s_out, down16, down16_sh,
-      total;
+  size_t header, chunk_hist, tiles, tiles_pair, logits, inv, h, h_sh, o, s_out, down16, down16_sh;
+  size_t xq, sx, hq, sh, hshq, shs;  // FP8 experts: e4m3 rows of x, h, h_shared and their scales
+  size_t total;
   int max_tiles;
 };
 
@@ -147,10 +150,26 @@ WsLayout ws_layout(const Dims &D) {
   L.s_out = off;  // shared-expert output, token rows
   off += align256(D.Fs > 0 ? static_cast<size_t>(D.T) * D.d * 2 : 0);
   L.down16 = L.down16_sh = off;
-  if (!(D.flags & MOE_FLAG_DOWN_F16)) {  // per-call fp16 copy of the down projections
+  // per-call fp16 copy of the down projections (16-bit path without prepared copies)
+  if (!(D.flags & (MOE_FLAG_DOWN_F16 | MOE_FLAG_FP8_EXPERTS))) {
     off += align256(static_cast<size_t>(D.E) * D.d * D.F * 2);
     L.down16_sh = off;
     off += align256(static_cast<size_t>(D.d) * D.Fs * 2);
+  }
+  L.xq = L.sx = L.hq = L.sh = L.hshq = L.shs = off;
+  if (D.flags & MOE_FLAG_FP8_EXPERTS) {
+    L.xq = off;
+    off += align256(static_cast<size_t>(D.T) * D.d);
+    L.sx = off;
+    off += align256(static_cast<size_t>(D.T) * 4);
+    L.hq = off;
+    off += align256(n * D.F);
+    L.sh = off;
+    off += align256(n * 4);
+    L.hshq = off;
+    off += align256(static_cast<size_t>(D.T) * D.Fs);
+    L.shs = off;
+    off += align256(static_cast<size_t>(D.T) * 4);
   }
   L.total = off;
   return L;
@@ -177,6 +196,9 @@ moe_status check_dims(const moe_dims_t *dims, Dims *D) {
   if (static_cast<int64_t>(D->E) * std::max(D->F, D->d) >= (int64_t(1) << 31))
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((dims->flags & MOE_FLAG_ROUTER_TENSOR) && (D->E % 16 != 0 || D->E > 256))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  // FP8 experts: K stages of 128 e4m3 elements
+  if ((dims->flags & MOE_FLAG_FP8_EXPERTS) && (D->F % 128 != 0 || D->Fs % 128 != 0))
     return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
@@ -205,19 +227,27 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
                       cudaStream_t s, int sms, int *launches) {
   const WsLayout L = ws_layout(D);
   float *logits = reinterpret_cast<float *>(wsp(ws, L.logits));
+  // A selection-only bias stays out of the logits and goes to the select kernel.
+  const float *sel_bias = (D.flags & MOE_FLAG_BIAS_SELECTION_ONLY) ? bias : nullptr;
+  if (sel_bias) bias = nullptr;
   if (use_tensor_router(D)) {
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
     p.status = reinterpret_cast<int *>(wsp(ws, L.header));
     p.n_tiles_host = (D.T + kBlockM - 1) / kBlockM;
-    p.n_ntiles = 1;
+    // Few token tiles (small T): split the experts into column blocks so that
+    // more SMs share the work; each block re-reads the token tile from L2.
+    int nsplit = 1;
+    while (nsplit < 8 && p.n_tiles_host * nsplit * 2 <= sms && D.E % (nsplit * 2 * 32) == 0)
+      nsplit *= 2;
+    p.n_ntiles = nsplit;
     p.T = D.T;
     p.d = D.d;
     p.E = D.E;
     p.k = D.k;
     p.F = D.F;
     p.Fs = D.Fs;
-    p.n_tile = D.E;
+    p.n_tile = D.E / nsplit;
     p.bias = bias;
     p.logits_out = logits;
 
@@ -226,16 +256,16 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     GemmMaps m;
     std::memset(&m, 0, sizeof(m));
     if (!make_map(&m.a, x, D.T, D.d, a_rows)) return MOE_ERR_CUDA;
-    if (!make_map(&m.b0, w_router, D.E, D.d, D.E)) return MOE_ERR_CUDA;
+    if (!make_map(&m.b0, w_router, D.E, D.d, p.n_tile)) return MOE_ERR_CUDA;
     m.b1 = m.b0;
     m.a_sh = m.a;
     m.b0_sh = m.b0;
     m.b1_sh = m.b0;
-    const int grid = std::min(sms, p.n_tiles_host);
+    const int grid = std::min(sms, p.n_tiles_host * p.n_ntiles);
     if (launch_gemm(MODE_ROUTER, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (launch_router_select(logits, static_cast<const uint16_t *>(x),
-                             static_cast<const uint16_t *>(w_router), bias, token_mask, D.T, D.d,
-                             D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
+                             static_cast<const uint16_t *>(w_router), bias, sel_bias, token_mask,
+                             D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
       return MOE_ERR_CUDA;
     *launches += 2;
     return MOE_OK;
@@ -244,8 +274,8 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
                        bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (launch_router_select(logits, static_cast<const uint16_t *>(x),
-                           static_cast<const uint16_t *>(w_router), bias, token_mask, D.T, D.d,
-                           D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
+                           static_cast<const uint16_t *>(w_router), bias, sel_bias, token_mask,
+                           D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   *launches += 2;
   return MOE_OK;
@@ -254,6 +284,30 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
 moe_status clear_header(void *ws, cudaStream_t s) {
   return cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
+
+moe_status check_routing_ptrs(const moe_routing_t *r) {
+  const void *ptrs[] = {r->topk_idx, r->topk_w, r->counts, r->offsets, r->perm};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status check_fp8_ptrs(const Dims &D, const moe_fp8_weights_t *q) {
+  const void *ptrs[] = {q->w_gate, q->w_up, q->w_down, q->s_gate, q->s_up, q->s_down};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (D.Fs > 0) {
+    const void *sh[] = {q->ws_gate, q->ws_up, q->ws_down, q->ss_gate, q->ss_up, q->ss_down};
+    for (const void *p : sh)
+      if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+// The whole layer after argument checks; q != nullptr selects the FP8 experts.
+moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_weights_t *q,
+                        const void *x, const uint8_t *token_mask, void *y,
+                        const moe_routing_t *routing, void *ws, void *stream);
 
 }  // namespace
 
@@ -346,11 +400,8 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
   if (!w || !x || !y || !routing) return MOE_ERR_INVALID_ARG;
   if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
   if (D.Fs > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down)) return MOE_ERR_INVALID_ARG;
-  if (!routing->topk_idx || !routing->topk_w || !routing->counts || !routing->offsets ||
-      !routing->perm)
-    return MOE_ERR_INVALID_ARG;
-  const void *ptrs[] = {x, y, w->w_router, w->w_gate, w->w_up, w->w_down, routing->topk_idx,
-                        routing->topk_w, routing->counts, routing->offsets, routing->perm};
+  if ((st = check_routing_ptrs(routing)) != MOE_OK) return st;
+  const void *ptrs[] = {x, y, w->w_router, w->w_gate, w->w_up, w->w_down};
   for (const void *p : ptrs)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (w->router_bias && !aligned16(w->router_bias)) return MOE_ERR_INVALID_ARG;
@@ -359,8 +410,73 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
   if (D.flags & MOE_FLAG_DOWN_F16) {
     if (!w->w_down_f16 || !aligned16(w->w_down_f16)) return MOE_ERR_INVALID_ARG;
     if (D.Fs > 0 && (!w->ws_down_f16 || !aligned16(w->ws_down_f16))) return MOE_ERR_INVALID_ARG;
+  } else if (D.flags & MOE_FLAG_FP8_EXPERTS) {
+    return MOE_ERR_INVALID_ARG;  // that workspace has no room for the per-call fp16 copy
   }
   if ((st = check_ws(D, ws, ws_bytes)) != MOE_OK) return st;
+  return forward_impl(D, w, nullptr, x, token_mask, y, routing, ws, stream);
+}
+
+moe_status moe_forward_fp8(const moe_dims_t *dims, const moe_weights_t *w,
+                           const moe_fp8_weights_t *q, const void *x, void *y,
+                           const moe_routing_t *routing, void *ws, size_t ws_bytes, void *stream) {
+  Dims D;
+  moe_status st = check_dims(dims, &D);
+  if (st != MOE_OK) return st;
+  if (!(D.flags & MOE_FLAG_FP8_EXPERTS)) return MOE_ERR_INVALID_ARG;
+  if (!w || !q || !x || !y || !routing || !w->w_router) return MOE_ERR_INVALID_ARG;
+  if ((st = check_fp8_ptrs(D, q)) != MOE_OK) return st;
+  if ((st = check_routing_ptrs(routing)) != MOE_OK) return st;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(w->w_router) ||
+      (w->router_bias && !aligned16(w->router_bias)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(D, ws, ws_bytes)) != MOE_OK) return st;
+  return forward_impl(D, w, q, x, nullptr, y, routing, ws, stream);
+}
+
+moe_status moe_prepare_fp8(const moe_dims_t *dims, const moe_weights_t *w,
+                           const moe_fp8_weights_t *q, void *ws, size_t ws_bytes, void *stream) {
+  Dims D;
+  moe_status st = check_dims(dims, &D);
+  if (st != MOE_OK) return st;
+  if (!w || !q || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (D.Fs > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_fp8_ptrs(D, q)) != MOE_OK) return st;
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  if (device_setup(&sms) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_header(ws, s)) != MOE_OK) return st;
+  const int EF = D.E * D.F, Ed = D.E * D.d;
+  struct Job { const void *src; int rows, K; void *codes; float *scales; };
+  const Job jobs[] = {{w->w_gate, EF, D.d, q->w_gate, q->s_gate},
+                      {w->w_up, EF, D.d, q->w_up, q->s_up},
+                      {w->w_down, Ed, D.F, q->w_down, q->s_down},
+                      {w->ws_gate, D.Fs, D.d, q->ws_gate, q->ss_gate},
+                      {w->ws_up, D.Fs, D.d, q->ws_up, q->ss_up},
+                      {w->ws_down, D.Fs > 0 ? D.d : 0, D.Fs, q->ws_down, q->ss_down}};
+  int launches = 0;
+  for (const Job &j : jobs) {
+    if (j.rows == 0) continue;
+    if (launch_quant_rows_e4m3(static_cast<const uint16_t *>(j.src), false, j.rows, nullptr, j.K,
+                               static_cast<uint8_t *>(j.codes), j.scales, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    ++launches;
+  }
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_weights_t *q,
+                        const void *x, const uint8_t *token_mask, void *y,
+                        const moe_routing_t *routing, void *ws, void *stream) {
+  moe_status st = MOE_OK;
+  const bool fp8 = q != nullptr;
   g_last_launches = 0;
   if (D.T == 0) return MOE_OK;
   int sms = 0;
@@ -394,7 +510,7 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
   bool pair2 = static_cast<int64_t>(D.T) * D.k >= static_cast<int64_t>(2 * kBlockM) * D.E;
   if (D.flags & MOE_FLAG_GEMM_PAIR) pair1 = pair2 = true;
   if (D.flags & MOE_FLAG_GEMM_SINGLE_CTA) pair1 = pair2 = false;
-  if (pair_grid < 2) pair1 = pair2 = false;
+  if (pair_grid < 2 || fp8) pair1 = pair2 = false;
   Tile *tiles_pair = reinterpret_cast<Tile *>(wsp(ws, L.tiles_pair));
   ev.mark();
   if (launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0,
@@ -403,10 +519,20 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
                    (pair1 || pair2) ? tiles_pair : nullptr, inv) != cudaSuccess)
     return MOE_ERR_CUDA;
 
+  // FP8 experts: e4m3 rows of x with their scales
+  uint8_t *xq = reinterpret_cast<uint8_t *>(wsp(ws, L.xq));
+  float *sx = reinterpret_cast<float *>(wsp(ws, L.sx));
+  if (fp8) {
+    if (launch_quant_rows_e4m3(static_cast<const uint16_t *>(x), false, D.T, nullptr, D.d, xq, sx,
+                               s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    launches += 1;
+  }
+
   // fp16 down projections: caller-prepared, or converted here every call
   const void *wd16 = w->w_down_f16;
   const void *wsd16 = w->ws_down_f16;
-  if (!(D.flags & MOE_FLAG_DOWN_F16)) {
+  if (!fp8 && !(D.flags & MOE_FLAG_DOWN_F16)) {
     uint16_t *dst = reinterpret_cast<uint16_t *>(wsp(ws, L.down16));
     if (launch_bf16_to_f16(static_cast<const uint16_t *>(w->w_down),
                            static_cast<size_t>(D.E) * D.d * D.F, dst, header, s) != cudaSuccess)
@@ -462,15 +588,30 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
     p.a_sh_bytes = p.a_bytes;
     GemmMaps m;
     std::memset(&m, 0, sizeof(m));
-    if (!make_map(&m.a, x, D.T, D.d, 1)) return MOE_ERR_CUDA;
-    if (!make_map(&m.b0, w->w_gate, static_cast<uint64_t>(D.E) * D.F, D.d, n_half)) return MOE_ERR_CUDA;
-    if (!make_map(&m.b1, w->w_up, static_cast<uint64_t>(D.E) * D.F, D.d, n_half)) return MOE_ERR_CUDA;
+    const CUtensorMapDataType bt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                       : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const void *wg = fp8 ? q->w_gate : w->w_gate;
+    const void *wu = fp8 ? q->w_up : w->w_up;
+    if (!make_map(&m.a, fp8 ? static_cast<const void *>(xq) : x, D.T, D.d, 1, bt))
+      return MOE_ERR_CUDA;
+    if (!make_map(&m.b0, wg, static_cast<uint64_t>(D.E) * D.F, D.d, n_half, bt)) return MOE_ERR_CUDA;
+    if (!make_map(&m.b1, wu, static_cast<uint64_t>(D.E) * D.F, D.d, n_half, bt)) return MOE_ERR_CUDA;
     m.a_sh = m.a;
+    if (fp8) {
+      p.xq = xq;
+      p.sx = sx;
+      p.sb0 = q->s_gate;
+      p.sb1 = q->s_up;
+      p.sb0_sh = q->ss_gate;
+      p.sb1_sh = q->ss_up;
+    }
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (!make_map(&m.out, h, n_rows, D.F, std::min(32, n_rows), f16)) return MOE_ERR_CUDA;
     if (D.Fs > 0) {
-      if (!make_map(&m.b0_sh, w->ws_gate, D.Fs, D.d, n_half)) return MOE_ERR_CUDA;
-      if (!make_map(&m.b1_sh, w->ws_up, D.Fs, D.d, n_half)) return MOE_ERR_CUDA;
+      if (!make_map(&m.b0_sh, fp8 ? q->ws_gate : w->ws_gate, D.Fs, D.d, n_half, bt))
+        return MOE_ERR_CUDA;
+      if (!make_map(&m.b1_sh, fp8 ? q->ws_up : w->ws_up, D.Fs, D.d, n_half, bt))
+        return MOE_ERR_CUDA;
       if (!make_map(&m.out_sh, h_sh, D.T, D.Fs, std::min(32, D.T), f16)) return MOE_ERR_CUDA;
     } else {
       m.b0_sh = m.b0;
@@ -479,9 +620,25 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
     }
     ev.mark();
     const cudaError_t e = pair1 ? launch_gemm_pair(MODE_GEMM1, p, m, pair_grid, s)
-                               : launch_gemm(MODE_GEMM1, p, m, sms, s);
+                               : launch_gemm(fp8 ? MODE_GEMM1_F8 : MODE_GEMM1, p, m, sms, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
+  }
+  // FP8 experts: e4m3 rows of h (the routed rows up to offsets[E]) and h_shared
+  uint8_t *hq = reinterpret_cast<uint8_t *>(wsp(ws, L.hq));
+  float *shq = reinterpret_cast<float *>(wsp(ws, L.sh));
+  uint8_t *hshq = reinterpret_cast<uint8_t *>(wsp(ws, L.hshq));
+  float *shs = reinterpret_cast<float *>(wsp(ws, L.shs));
+  if (fp8) {
+    if (launch_quant_rows_e4m3(h, true, n_rows, routing->offsets + D.E, D.F, hq, shq, s) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    launches += 1;
+    if (D.Fs > 0) {
+      if (launch_quant_rows_e4m3(h_sh, true, D.T, nullptr, D.Fs, hshq, shs, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      launches += 1;
+    }
   }
   // 4. GEMM2: h . W_down^T -> x (routed_scaling_factor * w) -> expert-order rows
   {
@@ -500,16 +657,25 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
     GemmMaps m;
     std::memset(&m, 0, sizeof(m));
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (!make_map(&m.a, h, n_rows, D.F, a_rows, f16)) return MOE_ERR_CUDA;
+    const CUtensorMapDataType at = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : f16;
+    if (!make_map(&m.a, fp8 ? static_cast<const void *>(hq) : h, n_rows, D.F, a_rows, at))
+      return MOE_ERR_CUDA;
     const uint32_t b_rows = pair2 ? n2 / 2 : n2;  // a pair splits B along N
-    if (!make_map(&m.b0, wd16, static_cast<uint64_t>(D.E) * D.d, D.F, b_rows, f16))
+    if (!make_map(&m.b0, fp8 ? q->w_down : wd16, static_cast<uint64_t>(D.E) * D.d, D.F, b_rows, at))
       return MOE_ERR_CUDA;
     m.b1 = m.b0;
+    if (fp8) {
+      p.sa = shq;
+      p.sa_sh = shs;
+      p.sb0 = q->s_down;
+      p.sb0_sh = q->ss_down;
+    }
     if (!make_map(&m.out, o_out, n_rows, D.d, std::min(32, n_rows), f16)) return MOE_ERR_CUDA;
     m.out_sh = m.out;
     if (D.Fs > 0) {
-      if (!make_map(&m.a_sh, h_sh, D.T, D.Fs, a_sh_rows, f16)) return MOE_ERR_CUDA;
-      if (!make_map(&m.b0_sh, wsd16, D.d, D.Fs, b_rows, f16)) return MOE_ERR_CUDA;
+      if (!make_map(&m.a_sh, fp8 ? static_cast<const void *>(hshq) : h_sh, D.T, D.Fs, a_sh_rows, at))
+        return MOE_ERR_CUDA;
+      if (!make_map(&m.b0_sh, fp8 ? q->ws_down : wsd16, D.d, D.Fs, b_rows, at)) return MOE_ERR_CUDA;
       if (!make_map(&m.out_sh, s_out, D.T, D.d, std::min(32, D.T), f16)) return MOE_ERR_CUDA;
     } else {
       m.a_sh = m.a;
@@ -518,7 +684,7 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
     m.b1_sh = m.b0_sh;
     ev.mark();
     const cudaError_t e = pair2 ? launch_gemm_pair(MODE_GEMM2, p, m, pair_grid, s)
-                               : launch_gemm(MODE_GEMM2, p, m, sms, s);
+                               : launch_gemm(fp8 ? MODE_GEMM2_F8 : MODE_GEMM2, p, m, sms, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
   }
@@ -532,6 +698,10 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
   g_last_launches = launches;
   return MOE_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 moe_status moe_prepare_down_f16(const moe_dims_t *dims, const void *w_down, const void *ws_down,
                                 void *w_down_f16, void *ws_down_f16, void *ws, size_t ws_bytes,

@@ -2,7 +2,7 @@
 //
 // One kernel template serves the three contractions of the layer:
 //
-//   MODE_ROUTER  logits[128 tokens, E] = x_tile . W_r^T (+ b), fp32 in TMEM,
+//   MODE_ROUTER  logits[128 tokens, n_tile experts] = x_tile . W_r^T (+ b), fp32 in TMEM,
 //                written out for the warp-per-token selection (sigmoid router
 //                with post-top-k normalisation: Laguna M.1/XS.2 Technical
 //                Report summary, Key claims, report §3.1).
@@ -84,6 +84,9 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
                     const __grid_constant__ CUtensorMap tm_b1_sh,
                     const __grid_constant__ CUtensorMap tm_out,
                     const __grid_constant__ CUtensorMap tm_out_sh) {
+  // BASE: the GEMM this launch computes; F8: e4m3 operands (MODE_F8 bit).
+  constexpr int BASE = MODE & 3;
+  constexpr bool F8 = (MODE & MODE_F8) != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       // GEMM1: one expect_tx arrival for the B tiles plus one cp.async
       // completion arrival from each lane of the gathering warps.
-      mbar_init(&full[s], MODE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
+      mbar_init(&full[s], BASE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -115,14 +118,14 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
     mbar_init(drain, 1);
     fence_mbar_init();
   }
-  if (MODE == MODE_ROUTER) {
+  if (BASE == MODE_ROUTER) {
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) bias_s[e] = p.bias ? p.bias[e] : 0.f;
     for (int e = p.E + threadIdx.x; e < 512; e += blockDim.x) bias_s[e] = 0.f;
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b0);
-    if (MODE == MODE_GEMM1) prefetch_tmap(&tm_b1);
+    if (BASE == MODE_GEMM1) prefetch_tmap(&tm_b1);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -133,10 +136,11 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_items = (MODE == MODE_ROUTER) ? p.n_tiles_host : (*p.n_tiles_dev) * p.n_ntiles;
-  // The down projection multiplies fp16 h by fp16 W_down; the others are bf16.
-  const uint32_t idesc =
-      MODE == MODE_GEMM2 ? idesc_f16_f32(kBlockM, p.n_tile) : idesc_bf16_f32(kBlockM, p.n_tile);
+  const int n_items = ((BASE == MODE_ROUTER) ? p.n_tiles_host : *p.n_tiles_dev) * p.n_ntiles;
+  // The down projection multiplies fp16 h by fp16 W_down, the others bf16 operands; F8
+  // launches e4m3 (whose format code equals fp16's).
+  const uint32_t idesc = (BASE == MODE_GEMM2 || F8) ? idesc_f16_f32(kBlockM, p.n_tile)
+                                                     : idesc_bf16_f32(kBlockM, p.n_tile);
   int *status = p.status;
 
   if (warp == 0 || warp >= kGather2Warp) {
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
     const bool tma_warp = warp == 0;
     const int gw = tma_warp ? (kTmaWarpGathers ? 0 : -1)
                             : (kTmaWarpGathers ? 1 : 0) + (warp - kGather2Warp);
-    const bool gathers = MODE == MODE_GEMM1 && gw >= 0;
+    const bool gathers = BASE == MODE_GEMM1 && gw >= 0;
     if (tma_warp || gathers) {
       int s = 0;
       uint32_t ph = 0;
@@ -170,8 +174,8 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
         // their rows; the rest of the stage feeds accumulator rows that the
         // epilogue discards.
         uint32_t bytes;
-        if (MODE == MODE_ROUTER) bytes = p.a_bytes + p.E * 128;
-        else if (MODE == MODE_GEMM1) bytes = 2 * p.n_half * 128;  // A arrives by cp.async
+        if (BASE == MODE_ROUTER) bytes = p.a_bytes + p.n_tile * 128;
+        else if (BASE == MODE_GEMM1) bytes = 2 * p.n_half * 128;  // A arrives by cp.async
         else bytes = (shared ? p.a_sh_bytes : p.a_bytes) + p.n_tile * 128;
         for (int kb = 0; kb < it.nk; ++kb) {
           int good = 1;
@@ -188,22 +192,22 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
           if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
           uint8_t *a_dst = sA + s * kABytes;
           uint8_t *b_dst = sB + s * kBBytesMax;
-          const int kc = kb * kBlockK;
+          const int kc = kb * stage_k(MODE);
           if (tma_warp && lane == 0) {
-            if (MODE == MODE_GEMM1) {
+            if (BASE == MODE_GEMM1) {
               const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
               tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
               tma_load_2d(b_dst + p.n_half * 128, shared ? &tm_b1_sh : &tm_b1, &full[s], kc, brow);
-            } else if (MODE == MODE_ROUTER) {
+            } else if (BASE == MODE_ROUTER) {
               tma_load_2d(a_dst, &tm_a, &full[s], kc, it.row0);
-              tma_load_2d(b_dst, &tm_b0, &full[s], kc, 0);
+              tma_load_2d(b_dst, &tm_b0, &full[s], kc, it.j * p.n_tile);
             } else {
               tma_load_2d(a_dst, shared ? &tm_a_sh : &tm_a, &full[s], kc, it.row0);
               const int brow = (shared ? 0 : it.group * p.d) + it.j * p.n_tile;
               tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &full[s], kc, brow);
             }
           }
-          if (gathers) gather_a_stage(p, tok, lane, gw, a_dst, &full[s], kc);
+          if (gathers) gather_a_stage<MODE>(p, tok, lane, gw, a_dst, &full[s], kc);
           if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_PDONE, issued);
           ++issued;
           if (++s == kStages) {
@@ -255,14 +259,18 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
             break;
           }
           MOE_TRACE_AT(p, TR_FULL, consumed);
-          if (MODE == MODE_GEMM1) fence_proxy_async_smem();  // A was written by cp.async
+          if (BASE == MODE_GEMM1) fence_proxy_async_smem();  // A was written by cp.async
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kABytes);
           const uint32_t b0 = smem_u32(sB + s * kBBytesMax);
 #pragma unroll
-          for (int kk = 0; kk < kBlockK / 16; ++kk) {
-            umma_f16_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+          for (int kk = 0; kk < 4; ++kk) {  // 4 x 32 bytes of the 128-byte rows
+            if (F8)
+              umma_f8_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
                          idesc, (kb | kk) != 0);
+            else
+              umma_f16_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+                          idesc, (kb | kk) != 0);
           }
           umma_commit(&empty[s]);
           MOE_TRACE_AT(p, TR_MMA, consumed);
@@ -301,12 +309,12 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
       if (warp == 2 && lane == 0) MOE_TRACE_AT(p, TR_EPI_START, done);
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccStride;
-      if (MODE == MODE_ROUTER) {
+      if (BASE == MODE_ROUTER) {
         router_epilogue(p, it, taddr, row_local, bias_s);
-      } else if (MODE == MODE_GEMM1) {
-        swiglu_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+      } else if (BASE == MODE_GEMM1) {
+        swiglu_epilogue<F8>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       } else {
-        down_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+        down_epilogue<F8>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
@@ -347,9 +355,17 @@ cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int gr
     case MODE_GEMM1:
       return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM1>, p, m.a, m.b0, m.b1, m.a_sh,
                                 m.b0_sh, m.b1_sh, m.out, m.out_sh);
-    default:
+    case MODE_GEMM2:
       return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM2>, p, m.a, m.b0, m.b1, m.a_sh,
                                 m.b0_sh, m.b1_sh, m.out, m.out_sh);
+    case MODE_GEMM1_F8:
+      return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM1_F8>, p, m.a, m.b0, m.b1, m.a_sh,
+                                m.b0_sh, m.b1_sh, m.out, m.out_sh);
+    case MODE_GEMM2_F8:
+      return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM2_F8>, p, m.a, m.b0, m.b1, m.a_sh,
+                                m.b0_sh, m.b1_sh, m.out, m.out_sh);
+    default:
+      return cudaErrorInvalidValue;
   }
 }
 
@@ -363,7 +379,13 @@ cudaError_t gemm_set_attributes() {
   e = cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM1>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM2>,
+  e = cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM2>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM1_F8>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM2_F8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 

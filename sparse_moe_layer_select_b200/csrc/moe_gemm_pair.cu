@@ -185,7 +185,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
               tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &lfull[s], kc, brow);
             }
           }
-          if (gathers) gather_a_stage(p, tok, lane, gw, a_dst, &lfull[s], kc);
+          if (gathers) gather_a_stage<MODE>(p, tok, lane, gw, a_dst, &lfull[s], kc);
           if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_PDONE, issued);
           ++issued;
           if (++s == kPairStages) {
@@ -314,8 +314,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       tc_fence_after();
       const Item it = pair_half(whole, rank);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kPAccStride;
-      if (MODE == MODE_GEMM1) swiglu_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
-      else down_epilogue(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+      if (MODE == MODE_GEMM1) swiglu_epilogue<false>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+      else down_epilogue<false>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + acc * 8);

@@ -11,9 +11,11 @@
 //                         one expert's logits for those 8 tokens (16-byte
 //                         loads of W_r, fp32 FMA, warp butterfly reduction).
 //   router_select_kernel  one warp per token, for both logit paths: the E
-//                         logits sit in registers (E/32 per lane); k+1 rounds
-//                         of a warp arg-max (ties to the lower expert index)
-//                         pick the experts in descending order; tokens whose
+//                         logits sit in registers (E/32 per lane) as
+//                         order-preserving integer keys; k+1 rounds of a warp
+//                         arg-max (a max- then a min-reduction, ties to the
+//                         lower expert index) pick the experts in descending
+//                         order; tokens whose
 //                         k-th and (k+1)-th logits are within kRefineBand get
 //                         the experts near that boundary re-decided on float64
 //                         logits; sigmoid and normalisation in fp32.
@@ -136,10 +138,16 @@ __device__ __forceinline__ void logits_f64_x4(const uint16_t *__restrict__ x,
   }
 }
 
-// (value, expert) order of the selection: larger logit first, equal logits
-// by lower expert id; NaN (empty slot) after everything.
-__device__ __forceinline__ bool sel_before(float va, int ea, float vb, int eb) {
-  return va > vb || (va == vb && ea < eb) || (va == va && vb != vb);
+// Order-preserving fp32 -> uint32 key (IEEE sign-magnitude to unsigned
+// order); -0 is folded onto +0 and NaN onto 0, below every number.
+__device__ __forceinline__ uint32_t logit_key(float f) {
+  if (f != f) return 0u;
+  const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 // One warp per token: each lane sorts its NPL = E/32 logits once (odd-even
@@ -151,33 +159,53 @@ __device__ __forceinline__ bool sel_before(float va, int ea, float vb, int eb) {
 // M.1/XS.2 Technical Report summary, Key claims, report §3.1; Laguna-M.1-base
 // spec sheet, Mixture of experts).
 
+// Per-warp scratch of the float64 re-decision: the band members' ids and
+// values, then the places they take.
+struct RefineScratch {
+  double vals[32];
+  int ids[32];
+  int out_e[16];
+  float out_l[16];
+};
+
 template <int NPL>
-__device__ __forceinline__ void select_token(int t, int lane, const float *__restrict__ logits,
+__device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
+                                             const float *__restrict__ logits,
                                              const uint16_t *__restrict__ x,
                                              const uint16_t *__restrict__ w_router,
-                                             const float *__restrict__ bias, int d, int E, int k,
-                                             int norm_topk, int32_t *__restrict__ topk_idx,
+                                             const float *__restrict__ bias,
+                                             const float *__restrict__ sel_bias, int d, int E,
+                                             int k, int norm_topk, int32_t *__restrict__ topk_idx,
                                              float *__restrict__ topk_w) {
   const float *row = logits + static_cast<size_t>(t) * E;
-  const float kNaN = __int_as_float(0x7fc00000);
-  float v[NPL];
+  // The selection value of expert e: its logit, or with a selection-only bias
+  // sigmoid(logit) + b_e (the weights below always use the logit).
+  auto sel_value = [&](int e) -> float {
+    const float l = row[e];
+    return sel_bias ? 1.f / (1.f + expf(-l)) + sel_bias[e] : l;
+  };
+  // Keys: an order-preserving map of the fp32 logit to uint32 (larger logit,
+  // larger key; +0 and -0 equal; NaN and the padding slots past E lowest).
+  uint32_t key[NPL];
   int ev[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
     ev[i] = lane + 32 * i;
-    v[i] = ev[i] < E ? row[ev[i]] : kNaN;
+    key[i] = ev[i] < E ? logit_key(sel_value(ev[i])) : 0u;
   }
-  // sort descending (NPL rounds of odd-even transposition)
+  // Sort each lane's list descending by key.  The list starts in ascending
+  // expert id and the odd-even transposition network swaps only strictly
+  // smaller keys forward, so equal keys stay in ascending id (stable).
 #pragma unroll
   for (int r = 0; r < NPL; ++r) {
 #pragma unroll
     for (int i = r & 1; i + 1 < NPL; i += 2) {
-      if (sel_before(v[i + 1], ev[i + 1], v[i], ev[i])) {
-        const float tv = v[i];
+      if (key[i] < key[i + 1]) {
+        const uint32_t tk = key[i];
         const int te = ev[i];
-        v[i] = v[i + 1];
+        key[i] = key[i + 1];
         ev[i] = ev[i + 1];
-        v[i + 1] = tv;
+        key[i + 1] = tk;
         ev[i + 1] = te;
       }
     }
@@ -187,87 +215,150 @@ __device__ __forceinline__ void select_token(int t, int lane, const float *__res
   float lk = 0.f, lk1 = -INFINITY;
   const int rounds = k < E ? k + 1 : k;
   for (int j = 0; j < rounds; ++j) {
-    float bv = v[0];
-    int be = ev[0];
-    const int my_head = be;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (sel_before(ov, oe, bv, be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if (my_head == be) {  // pop the head
+    // the largest head key, then the lowest expert id among the heads holding it
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t ewin =
+        __reduce_min_sync(0xffffffffu, key[0] == kmax ? static_cast<uint32_t>(ev[0]) : 0xffffffffu);
+    if (static_cast<uint32_t>(ev[0]) == ewin) {  // pop the head
 #pragma unroll
       for (int i = 0; i + 1 < NPL; ++i) {
-        v[i] = v[i + 1];
+        key[i] = key[i + 1];
         ev[i] = ev[i + 1];
       }
-      v[NPL - 1] = kNaN;
+      key[NPL - 1] = 0u;
       ev[NPL - 1] = 0x7fffffff;
     }
+    const float lv = key_logit(kmax);
     if (j < k && lane == j) {
-      my_l = bv;
-      my_e = be;
+      my_l = lv;
+      my_e = static_cast<int>(ewin);
     }
-    if (j == k - 1) lk = bv;
-    if (j == k) lk1 = bv;
+    if (j == k - 1) lk = lv;
+    if (j == k) lk1 = lv;
   }
 
   if (k < E && lk - lk1 < kRefineBand) {
-    // Candidates: every expert whose fp32 logit reaches the lower band edge
-    // (the selected ones and the band below the boundary), in ascending id.
-    // Their float64 logits decide the top k among them.
-    const float lo = 0.5f * (lk + lk1) - kRefineBand;
-    double best_l[16];
-    int best_e[16];
-    int nbest = 0;
-    for (int i = 0; i < (E + 31) / 32; ++i) {
+    // The fp32 selection values are within kRefineBand / 4 of their float64
+    // values, so with mid the midpoint of the k-th and (k+1)-th values:
+    // experts above mid + kRefineBand are in the float64 top k, those below
+    // mid - kRefineBand are not.  Only the experts inside the band are
+    // re-decided on float64 values; they fill the places after the ones
+    // above the band.
+    const float mid = 0.5f * (lk + lk1);
+    const float lo = mid - kRefineBand, hi = mid + kRefineBand;
+    const int above = __popc(__ballot_sync(0xffffffffu, lane < k && my_l > hi));
+    const unsigned lt = (1u << lane) - 1u;
+    const int nslice = (E + 31) / 32;
+    int nband = 0;
+    for (int i = 0; i < nslice; ++i) {  // band members in ascending id
       const int e_lane = lane + 32 * i;
-      const bool cand = e_lane < E && row[e_lane] >= lo;
-      unsigned m = __ballot_sync(0xffffffffu, cand);
-      while (m) {
-        int eg[4] = {0, 0, 0, 0};
-        int ng = 0;
-        while (m && ng < 4) {  // up to four candidates, ascending id
-          eg[ng++] = (__ffs(m) - 1) + 32 * i;
-          m &= m - 1;
-        }
+      float v = 0.f;
+      bool in = false;
+      if (e_lane < E) {
+        v = sel_value(e_lane);
+        in = v >= lo && v <= hi;
+      }
+      const unsigned b = __ballot_sync(0xffffffffu, in);
+      const int pos = nband + __popc(b & lt);
+      if (in && pos < 32) rs->ids[pos] = e_lane;
+      nband += __popc(b);
+    }
+    __syncwarp();
+    if (nband <= 32) {
+      for (int g0 = 0; g0 < nband; g0 += 4) {
+        int eg[4];
+        const int ng = min(4, nband - g0);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) eg[g] = rs->ids[g0 + (g < ng ? g : 0)];
         double lg[4];
         logits_f64_x4(x, w_router, bias, t, eg, ng, d, lane, lg);
-        if (lane == 0) {
-          for (int g = 0; g < ng; ++g) {
-            // sorted insert, descending logit, lower id first on ties (ids arrive ascending)
-            const double l = lg[g];
-            int pos = nbest < k ? nbest : k;
-            while (pos > 0 && l > best_l[pos - 1]) --pos;
-            if (pos < k) {
-              const int last = nbest < k ? nbest : k - 1;
-              for (int q = last; q > pos; --q) {
-                best_l[q] = best_l[q - 1];
-                best_e[q] = best_e[q - 1];
-              }
-              best_l[pos] = l;
-              best_e[pos] = eg[g];
-              if (nbest < k) ++nbest;
-            }
-          }
+        if (lane < ng) {
+          const double l = lane == 0 ? lg[0] : lane == 1 ? lg[1] : lane == 2 ? lg[2] : lg[3];
+          rs->vals[g0 + lane] =
+              sel_bias ? 1.0 / (1.0 + exp(-l)) + static_cast<double>(sel_bias[eg[lane]]) : l;
         }
       }
-    }
-    // hand the refined list to lanes 0..k-1
-    for (int q = 0; q < k; ++q) {
-      const float lq = __shfl_sync(0xffffffffu, lane == 0 ? static_cast<float>(best_l[q]) : 0.f, 0);
-      const int eq = __shfl_sync(0xffffffffu, lane == 0 ? best_e[q] : 0, 0);
-      if (lane == q) {
-        my_l = lq;
-        my_e = eq;
+      __syncwarp();
+      if (lane < nband) {  // rank: descending float64 value, lower id first on ties
+        const double vc = rs->vals[lane];
+        const int ec = rs->ids[lane];
+        int rank = 0;
+        for (int j = 0; j < nband; ++j) {
+          const double vj = rs->vals[j];
+          rank += (vj > vc || (vj == vc && rs->ids[j] < ec)) ? 1 : 0;
+        }
+        if (above + rank < k) {
+          rs->out_e[above + rank] = ec;
+          rs->out_l[above + rank] = static_cast<float>(vc);
+        }
+      }
+      __syncwarp();
+      if (lane >= above && lane < k) {
+        my_e = rs->out_e[lane];
+        my_l = rs->out_l[lane];
+      }
+      __syncwarp();
+    } else {
+      // More than 32 experts in the band (degenerate, e.g. many equal
+      // logits): every expert from the lower band edge up is re-decided,
+      // streamed four at a time into a sorted list on lane 0.
+      double best_l[16];
+      int best_e[16];
+      int nbest = 0;
+      int eg[4] = {0, 0, 0, 0};
+      int ng = 0;
+      for (int i = 0; i <= nslice; ++i) {
+        unsigned m = 0;
+        if (i < nslice) {
+          const int e_lane = lane + 32 * i;
+          m = __ballot_sync(0xffffffffu, e_lane < E && sel_value(e_lane) >= lo);
+        }
+        while (m || (i == nslice && ng > 0)) {
+          while (m && ng < 4) {
+            eg[ng++] = (__ffs(m) - 1) + 32 * i;
+            m &= m - 1;
+          }
+          if (ng < 4 && i < nslice) break;  // group not full: take more from the next slice
+          double lg[4];
+          logits_f64_x4(x, w_router, bias, t, eg, ng, d, lane, lg);
+          if (lane == 0) {
+            for (int g = 0; g < ng; ++g) {
+              // sorted insert, descending value, lower id first on ties (ids arrive ascending)
+              const double l = sel_bias
+                                   ? 1.0 / (1.0 + exp(-lg[g])) + static_cast<double>(sel_bias[eg[g]])
+                                   : lg[g];
+              int pos = nbest < k ? nbest : k;
+              while (pos > 0 && l > best_l[pos - 1]) --pos;
+              if (pos < k) {
+                const int last = nbest < k ? nbest : k - 1;
+                for (int q = last; q > pos; --q) {
+                  best_l[q] = best_l[q - 1];
+                  best_e[q] = best_e[q - 1];
+                }
+                best_l[pos] = l;
+                best_e[pos] = eg[g];
+                if (nbest < k) ++nbest;
+              }
+            }
+          }
+          ng = 0;
+        }
+      }
+      for (int q = 0; q < k; ++q) {  // hand the list to lanes 0..k-1
+        const float lq =
+            __shfl_sync(0xffffffffu, lane == 0 ? static_cast<float>(best_l[q]) : 0.f, 0);
+        const int eq = __shfl_sync(0xffffffffu, lane == 0 ? best_e[q] : 0, 0);
+        if (lane == q) {
+          my_l = lq;
+          my_e = eq;
+        }
       }
     }
   }
 
+  // With a selection-only bias the rounds carried sigmoid(l) + b: the weights
+  // take the selected experts' own logits.
+  if (sel_bias && lane < k) my_l = row[my_e];
   const float s = 1.f / (1.f + expf(-my_l));
   float sum = lane < k ? s : 0.f;
 #pragma unroll
@@ -283,6 +374,7 @@ template <int NPL>
 __global__ void __launch_bounds__(kSelectWarps * 32)
     router_select_kernel(const float *__restrict__ logits, const uint16_t *__restrict__ x,
                          const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
+                         const float *__restrict__ sel_bias,
                          const uint8_t *__restrict__ token_mask, int T, int d, int E, int k,
                          int norm_topk,
                          int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
@@ -297,7 +389,9 @@ __global__ void __launch_bounds__(kSelectWarps * 32)
     }
     return;
   }
-  select_token<NPL>(t, lane, logits, x, w_router, bias, d, E, k, norm_topk, topk_idx, topk_w);
+  __shared__ RefineScratch scratch[kSelectWarps];
+  select_token<NPL>(t, lane, &scratch[threadIdx.x >> 5], logits, x, w_router, bias, sel_bias, d,
+                    E, k, norm_topk, topk_idx, topk_w);
 }
 
 }  // namespace
@@ -321,15 +415,16 @@ cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const 
 }
 
 cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
-                                 const float *bias, const uint8_t *token_mask, int T, int d, int E,
-                                 int k, int norm_topk, int32_t *topk_idx, float *topk_w,
-                                 cudaStream_t s) {
+                                 const float *bias, const float *sel_bias,
+                                 const uint8_t *token_mask, int T, int d, int E, int k,
+                                 int norm_topk, int32_t *topk_idx, float *topk_w, cudaStream_t s) {
   const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
   const int threads = kSelectWarps * 32;
   const int npl = (E + 31) / 32;
 #define MOE_SELECT(N)                                                                          \
-  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, token_mask, T, \
-                                                     d, E, k, norm_topk, topk_idx, topk_w)
+  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, sel_bias,       \
+                                                     token_mask, T, d, E, k, norm_topk, topk_idx, \
+                                                     topk_w)
   if (npl <= 1) MOE_SELECT(1);
   else if (npl <= 2) MOE_SELECT(2);
   else if (npl <= 4) MOE_SELECT(4);

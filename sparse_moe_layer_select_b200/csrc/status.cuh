@@ -30,7 +30,8 @@ struct WsHeader {
   int site;       // Site of that error
   int n_tiles;    // 128-row tiles in the expert tile list (written by the index builder)
   int n_tiles_pair;  // 256-row tiles in the second list, when one is built
-  int pad[60];
+  int index_done;    // index builder: histogram CTAs finished (the last one scans)
+  int pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 

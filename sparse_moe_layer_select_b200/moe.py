@@ -26,13 +26,15 @@ MOE_FLAG_ROUTER_TENSOR = 2
 MOE_FLAG_DOWN_F16 = 4
 MOE_FLAG_GEMM_SINGLE_CTA = 8
 MOE_FLAG_GEMM_PAIR = 16
+MOE_FLAG_BIAS_SELECTION_ONLY = 32
+MOE_FLAG_FP8_EXPERTS = 64
 
 # Every symbol the header declares (checked by the CPU tests).
 EXPORTED = ["moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
             "moe_read_device_status", "moe_selftest_bounded_wait", "moe_status_string",
             "moe_last_launch_count", "moe_profile_next_forward", "moe_prepare_down_f16",
             "moe_logits_offset", "moe_permute_static", "moe_route_masked",
-            "moe_forward_masked"]
+            "moe_forward_masked", "moe_prepare_fp8", "moe_forward_fp8"]
 
 # Expert id of a (token, slot) pair that is not routed (a padding token).
 MOE_NOT_ROUTED = -1
@@ -59,6 +61,12 @@ class moe_weights_t(ctypes.Structure):
                 ("w_down", ctypes.c_void_p), ("ws_gate", ctypes.c_void_p),
                 ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p),
                 ("w_down_f16", ctypes.c_void_p), ("ws_down_f16", ctypes.c_void_p)]
+
+
+class moe_fp8_weights_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down",
+                 "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down")]
 
 
 class moe_routing_t(ctypes.Structure):
@@ -89,6 +97,13 @@ def lib():
         L.moe_forward.restype = ctypes.c_int
         L.moe_forward.argtypes = [D, ctypes.POINTER(moe_weights_t), P, P,
                                   ctypes.POINTER(moe_routing_t), P, ctypes.c_size_t, P]
+        L.moe_prepare_fp8.restype = ctypes.c_int
+        L.moe_prepare_fp8.argtypes = [D, ctypes.POINTER(moe_weights_t),
+                                      ctypes.POINTER(moe_fp8_weights_t), P, ctypes.c_size_t, P]
+        L.moe_forward_fp8.restype = ctypes.c_int
+        L.moe_forward_fp8.argtypes = [D, ctypes.POINTER(moe_weights_t),
+                                      ctypes.POINTER(moe_fp8_weights_t), P, P,
+                                      ctypes.POINTER(moe_routing_t), P, ctypes.c_size_t, P]
         L.moe_route_masked.restype = ctypes.c_int
         L.moe_route_masked.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_forward_masked.restype = ctypes.c_int
@@ -196,6 +211,51 @@ def prepare_down_f16(dims, W, stream=None):
     return read_device_status(hdr, stream)
 
 
+FP8_FIELDS = ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down",
+              "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down")
+
+
+def prepare_fp8(dims, W, stream=None):
+    """FP8 copies of the expert weights (moe_prepare_fp8): returns a dict of device tensors
+    (e4m3 codes as uint8, float32 row scales) and the device status."""
+    import torch
+    dev = W["w_gate"].device
+    E, F, d = W["w_gate"].shape
+    Q = {"w_gate": torch.empty((E, F, d), dtype=torch.uint8, device=dev),
+         "w_up": torch.empty((E, F, d), dtype=torch.uint8, device=dev),
+         "w_down": torch.empty((E, d, F), dtype=torch.uint8, device=dev),
+         "s_gate": torch.empty(E * F, dtype=torch.float32, device=dev),
+         "s_up": torch.empty(E * F, dtype=torch.float32, device=dev),
+         "s_down": torch.empty(E * d, dtype=torch.float32, device=dev)}
+    if W.get("ws_gate") is not None:
+        Fs = W["ws_gate"].shape[0]
+        Q.update(ws_gate=torch.empty((Fs, d), dtype=torch.uint8, device=dev),
+                 ws_up=torch.empty((Fs, d), dtype=torch.uint8, device=dev),
+                 ws_down=torch.empty((d, Fs), dtype=torch.uint8, device=dev),
+                 ss_gate=torch.empty(Fs, dtype=torch.float32, device=dev),
+                 ss_up=torch.empty(Fs, dtype=torch.float32, device=dev),
+                 ss_down=torch.empty(d, dtype=torch.float32, device=dev))
+    hdr = torch.zeros(256, dtype=torch.uint8, device=dev)
+    _check(lib().moe_prepare_fp8(ctypes.byref(dims), ctypes.byref(weights_struct(W)),
+                                 ctypes.byref(fp8_struct(Q)), _p(hdr), 256, _stream(stream)),
+           "moe_prepare_fp8")
+    return Q, read_device_status(hdr, stream)
+
+
+def fp8_struct(Q):
+    return moe_fp8_weights_t(*[None if Q.get(k) is None else Q[k].data_ptr() for k in FP8_FIELDS])
+
+
+def forward_fp8(dims, weights, fp8, x, y, routing, ws, stream=None):
+    """moe_forward_fp8 (dims.flags must include MOE_FLAG_FP8_EXPERTS)."""
+    ws_s = weights if isinstance(weights, moe_weights_t) else weights_struct(weights)
+    q_s = fp8 if isinstance(fp8, moe_fp8_weights_t) else fp8_struct(fp8)
+    r_s = routing if isinstance(routing, moe_routing_t) else routing_struct(routing)
+    _check(lib().moe_forward_fp8(ctypes.byref(dims), ctypes.byref(ws_s), ctypes.byref(q_s), _p(x),
+                                 _p(y), ctypes.byref(r_s), _p(ws), ws.numel(), _stream(stream)),
+           "moe_forward_fp8")
+
+
 def logits_offset(dims) -> int:
     return int(lib().moe_logits_offset(ctypes.byref(dims)))
 
@@ -270,7 +330,7 @@ class MoeLayer:
 
     def __init__(self, weights: dict, d_model, num_experts, num_experts_per_tok,
                  moe_intermediate_size, shared_intermediate_size, routed_scaling_factor=2.5,
-                 max_tokens=1, flags=0, device="cuda", prepare=True):
+                 max_tokens=1, flags=0, device="cuda", prepare=True, fp8=False):
         self.W = dict(weights)
         self.cfg = dict(d_model=d_model, num_experts=num_experts,
                         num_experts_per_tok=num_experts_per_tok,
@@ -278,7 +338,14 @@ class MoeLayer:
                         shared_intermediate_size=shared_intermediate_size,
                         routed_scaling_factor=routed_scaling_factor, flags=flags)
         self.device = device
-        if prepare:  # one-time fp16 copy of the down projections (model-load step)
+        self.fp8 = None
+        if fp8:  # one-time FP8 copies of the expert weights (model-load step)
+            self.cfg["flags"] |= MOE_FLAG_FP8_EXPERTS
+            self.fp8, (code, site) = prepare_fp8(self.dims(1), self.W)
+            if code != MOE_OK:
+                raise MoeError(code, f"moe_prepare_fp8 (site {site})")
+            self._q_struct = fp8_struct(self.fp8)
+        elif prepare:  # one-time fp16 copy of the down projections (model-load step)
             self.cfg["flags"] |= MOE_FLAG_DOWN_F16
             code, site = prepare_down_f16(self.dims(1), self.W)
             if code != MOE_OK:
@@ -307,5 +374,11 @@ class MoeLayer:
         if y is None:
             y = torch.empty_like(x)
         d = self.dims(T)
-        forward(d, self._ws_struct, x, y, self._r_struct, self.ws, stream, token_mask=token_mask)
+        if self.fp8 is not None:
+            if token_mask is not None:
+                raise ValueError("the FP8-expert forward takes no token mask")
+            forward_fp8(d, self._ws_struct, self._q_struct, x, y, self._r_struct, self.ws, stream)
+        else:
+            forward(d, self._ws_struct, x, y, self._r_struct, self.ws, stream,
+                    token_mask=token_mask)
         return y

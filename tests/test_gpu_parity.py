@@ -176,6 +176,103 @@ def test_padding_mask_permute_and_gather():
     assert np.array_equal(xpn[:n], h["x"][p // w.k]) and np.all(xpn[n:] == 0)
 
 
+@pytest.mark.parametrize("flags", [M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR,
+                                   M.MOE_FLAG_ROUTER_TENSOR | M.MOE_FLAG_GEMM_PAIR])
+def test_selection_only_bias(flags):
+    """Auxiliary-loss-free variant: a per-expert bias on the sigmoid scores chooses the experts,
+    the weights are the unbiased scores normalised over them."""
+    import torch
+    w = I.get("c1_tiny").with_(T=1100)
+    h, dev = _small(w)
+    rng = np.random.default_rng(77)
+    b = (rng.standard_normal(w.E) * 0.05).astype(np.float32)
+    dev = dict(dev, router_bias=torch.from_numpy(b).cuda())
+    dims = M.dims_for(w, flags=flags | M.MOE_FLAG_BIAS_SELECTION_ONLY)
+    ws = M.alloc_workspace(dims)
+    ws.fill_(0xFF)
+    routing = M.alloc_routing(dims)
+    y = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
+    M.forward(dims, dev, dev["x"], y, routing, ws)
+    torch.cuda.synchronize()
+    assert M.read_device_status(ws)[0] == 0
+    ref = O.moe_forward(h["x"], h["w_router"], h["w_gate"], h["w_up"], h["w_down"], w.k,
+                        ws_gate=h["ws_gate"], ws_up=h["ws_up"], ws_down=h["ws_down"],
+                        routed_scaling_factor=w.routed_scaling_factor,
+                        selection_bias=b.astype(np.float64))
+    gidx = routing["topk_idx"].cpu().numpy()
+    G.check_routing(gidx, routing["topk_w"].cpu().numpy(), ref, w.k)
+    plain = O.route(h["x"], h["w_router"], None, w.k)[0]
+    assert (np.sort(gidx, 1) != np.sort(plain, 1)).any(axis=1).mean() > 0.05  # the bias acts
+    same = P.same_selection_mask(gidx, ref["topk_idx"])
+    G.check_output(G.y_numpy(y), ref["y"], rows_ok=same, what="selection-only bias")
+
+
+def test_fp8_weight_quantization_matches_oracle():
+    """moe_prepare_fp8: e4m3 codes and row scales equal the oracle's (codes of +0 and -0 are
+    both accepted for zero)."""
+    w = I.get("c1_tiny").with_(d_model=256, moe_intermediate_size=256, shared_intermediate_size=128)
+    h, dev = _small(w)
+    Q, (code, _) = M.prepare_fp8(M.dims_for(w), dev)
+    assert code == 0
+    ref = O.quantize_experts_fp8(h["w_gate"], h["w_up"], h["w_down"], h["ws_gate"], h["ws_up"],
+                                 h["ws_down"])
+    for name, key, skey in (("gate", "w_gate", "s_gate"), ("up", "w_up", "s_up"),
+                            ("down", "w_down", "s_down"), ("s_gate", "ws_gate", "ss_gate"),
+                            ("s_up", "ws_up", "ss_up"), ("s_down", "ws_down", "ss_down")):
+        rc, rs = ref[name]
+        gc = Q[key].cpu().numpy().reshape(rc.shape)
+        gs = Q[skey].cpu().numpy().reshape(rs.shape)
+        assert np.array_equal(gs.view(np.uint32), rs.astype(np.float32).view(np.uint32)), name
+        zero = (O.e4m3_value(gc) == 0) & (O.e4m3_value(rc) == 0)
+        assert np.all((gc == rc) | zero), name
+
+
+@pytest.mark.parametrize("T", [64, 300])
+def test_fp8_forward_matches_fp8_oracle(T):
+    """moe_forward_fp8 against the oracle of the same FP8 method (e4m3 weights, x and h with
+    per-row scales)."""
+    import torch
+    w = I.get("c1_tiny").with_(T=T, d_model=256, moe_intermediate_size=256,
+                               shared_intermediate_size=128)
+    h, dev = _small(w)
+    layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
+                       max_tokens=w.T, fp8=True)
+    y = layer.forward(dev["x"])
+    torch.cuda.synchronize()
+    assert M.read_device_status(layer.ws)[0] == 0
+    fp8 = O.quantize_experts_fp8(h["w_gate"], h["w_up"], h["w_down"], h["ws_gate"], h["ws_up"],
+                                 h["ws_down"])
+    ref = O.moe_forward_fp8(h["x"], h["w_router"], fp8, w.k,
+                            routed_scaling_factor=w.routed_scaling_factor)
+    gidx = layer.routing["topk_idx"][:T].cpu().numpy()
+    G.check_routing(gidx, layer.routing["topk_w"][:T].cpu().numpy(), ref, w.k)
+    same = P.same_selection_mask(gidx, ref["topk_idx"])
+    G.check_output(G.y_numpy(y), ref["y"], rows_ok=same, what=f"fp8 T={T}")
+
+
+def test_fp8_decode_matches_fp8_oracle():
+    import torch
+    w = I.get("c5_decode")
+    dev = I.device_inputs(w)
+    h = G.device_to_host(dev)
+    layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
+                       max_tokens=w.T, fp8=True)
+    ring = I.device_decode_ring(w, 2)
+    fp8 = O.quantize_experts_fp8(h["w_gate"], h["w_up"], h["w_down"], h["ws_gate"], h["ws_up"],
+                                 h["ws_down"])
+    for i in range(2):
+        y = layer.forward(ring[i])
+        torch.cuda.synchronize()
+        assert M.read_device_status(layer.ws)[0] == 0
+        xi = P.to_numpy_bf16(ring[i])
+        ref = O.moe_forward_fp8(xi, h["w_router"], fp8, w.k,
+                                routed_scaling_factor=w.routed_scaling_factor)
+        gidx = layer.routing["topk_idx"][:w.T].cpu().numpy()
+        G.check_routing(gidx, layer.routing["topk_w"][:w.T].cpu().numpy(), ref, w.k)
+        same = P.same_selection_mask(gidx, ref["topk_idx"])
+        G.check_output(G.y_numpy(y), ref["y"], rows_ok=same, what=f"fp8 decode batch {i}")
+
+
 def test_permute_materialised_gather_and_counts():
     import torch
     w = I.get("c1_tiny").with_(T=1000)

@@ -301,6 +301,166 @@ def test_expert_order_against_brute_force():
             assert counts[e] == len(want)
 
 
+# ---------------------------------------------------------------- selection-only bias
+
+@pytest.mark.parametrize("E", [3, 5, 8])
+def test_selection_bias_chooses_by_biased_score_weights_unbiased(E):
+    """Auxiliary-loss-free variant: the k experts maximise sum(sigmoid(l) + b) (brute force,
+    lexicographic-min on ties), the weights are the unbiased sigmoid scores normalised over them
+    (plain Python)."""
+    rng = np.random.default_rng(30 + E)
+    d, T = 6, 30
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d)) * 0.4
+    b = rng.standard_normal(E) * 0.15
+    _, sc = _py_logits_scores(x.tolist(), wr.tolist())
+    for k in range(1, E + 1):
+        idx, w, keys, _ = O.route(x, wr, None, k, selection_bias=b)
+        for t in range(T):
+            biased = [sc[t][e] + b[e] for e in range(E)]
+            bf = _brute_force_topk(biased, k)
+            assert tuple(sorted(idx[t].tolist())) == bf, (E, k, t)
+            tot = math.fsum(sc[t][e] for e in bf)
+            for j, e in enumerate(idx[t]):
+                assert abs(w[t, j] - sc[t][e] / tot) <= 1e-15
+                assert keys[t, e] == sc[t][e] + b[e] or abs(keys[t, e] - (sc[t][e] + b[e])) < 1e-15
+
+
+def test_selection_bias_zero_is_the_plain_router_and_a_large_bias_forces_an_expert():
+    rng = np.random.default_rng(40)
+    L = _rand_layer(rng, 25, 16, 8, 4, 4)
+    a = _fwd(L, 3)
+    z = _fwd(L, 3, selection_bias=np.zeros(8))
+    assert np.array_equal(z["topk_idx"], a["topk_idx"]) and np.array_equal(z["y"], a["y"])
+    b = np.zeros(8)
+    b[5] = 2.0  # sigmoid scores lie in (0, 1): +2 puts expert 5 first for every token
+    f = _fwd(L, 3, selection_bias=b)
+    assert np.all(f["topk_idx"][:, 0] == 5)
+    _, _, s, _ = O.route(L["x"], L["w_router"], None, 3)
+    sel = np.take_along_axis(s, f["topk_idx"], axis=1)
+    assert np.allclose(f["topk_w"], sel / sel.sum(axis=1, keepdims=True), rtol=0, atol=1e-15)
+    # the pin is sensitive: weights from the biased scores, or selection on biased logits,
+    # give other results
+    keys = s + b[None, :]
+    wrong_w = np.take_along_axis(keys, f["topk_idx"], axis=1)
+    assert not np.allclose(f["topk_w"], wrong_w / wrong_w.sum(axis=1, keepdims=True))
+    lg = O.router_logits(L["x"], L["w_router"], None)
+    b2 = rng.standard_normal(8) * 0.3
+    sel_keys = O.select_topk(O.sigmoid(lg) + b2[None, :], 3)
+    sel_logits = O.select_topk(lg + b2[None, :], 3)
+    got = O.route(L["x"], L["w_router"], None, 3, selection_bias=b2)[0]
+    assert np.array_equal(got, sel_keys) and not np.array_equal(got, sel_logits)
+
+
+# ---------------------------------------------------------------- e4m3 (FP8 experts)
+
+def test_e4m3_code_table_follows_the_format():
+    v = O.e4m3_value(np.arange(256))
+    assert v[0x38] == 1.0 and v[0xB8] == -1.0 and v[0x40] == 2.0 and v[0x3C] == 1.5
+    assert v[0x7E] == 448.0 and np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9
+    assert v[0x00] == 0.0 and v[0x80] == 0.0
+    assert np.all(np.diff(v[:0x7F]) > 0)           # codes 0..0x7E strictly increasing
+    assert np.array_equal(v[0x80:0xFF], -v[:0x7F])
+
+
+def _e4m3_brute(x):
+    """Nearest finite e4m3 value by exhaustive search; ties to the even code; |x| > 448 -> 448."""
+    codes = np.array([c for c in range(256) if not np.isnan(O.e4m3_value(c))])
+    vals = O.e4m3_value(codes)
+    out = []
+    for xv in np.asarray(x, dtype=np.float64):
+        xs = min(max(xv, -448.0), 448.0)
+        dist = np.abs(vals - xs)
+        best = codes[dist == dist.min()]
+        if len(best) > 1:
+            nz = [c for c in best if O.e4m3_value(c) != 0.0] or list(best)
+            even = [c for c in nz if c % 2 == 0]
+            best = even if even else nz
+            if O.e4m3_value(best[0]) == 0.0:  # zero keeps the input's sign
+                best = [0x80 if np.signbit(xv) else 0x00]
+        out.append(best[0])
+    return np.array(out)
+
+
+def test_e4m3_rounding_against_exhaustive_search():
+    rng = np.random.default_rng(50)
+    mag = 2.0 ** rng.uniform(-12, 10, 3000)
+    x = (mag * rng.choice([-1.0, 1.0], 3000)).astype(np.float32)
+    got = O.e4m3_round(x)
+    want = _e4m3_brute(x)
+    same = (got == want) | ((O.e4m3_value(got) == 0) & (O.e4m3_value(want) == 0))
+    assert same.all(), x[~same][:5]
+
+
+def test_e4m3_ties_go_to_even_and_large_values_saturate():
+    v = O.e4m3_value(np.arange(0x7F))
+    mids = ((v[:-1] + v[1:]) / 2).astype(np.float32)
+    exact = mids.astype(np.float64) == (v[:-1] + v[1:]) / 2   # midpoints exact in float32
+    codes = O.e4m3_round(mids[exact])
+    assert np.all(codes % 2 == 0)
+    big = np.array([449, 464, 480, 500, 1e6, 3e38], np.float32)
+    assert np.all(O.e4m3_round(big) == 0x7E) and np.all(O.e4m3_round(-big) == 0xFE)
+
+
+def test_per_row_quantization_error_bound():
+    rng = np.random.default_rng(51)
+    a = (rng.standard_normal((40, 300)) * 10.0 ** rng.uniform(-3, 2, (40, 1))).astype(np.float32)
+    a[3] = 0.0
+    codes, s = O.quantize_rows_e4m3(a)
+    deq = O.dequantize_rows_e4m3(codes, s)
+    assert s[3] == 1.0 and np.all(deq[3] == 0)
+    assert np.all(np.abs(O.e4m3_value(codes)).max(axis=1)[np.arange(40) != 3] == 448.0)
+    # round to nearest: at most half a quantum (2^-4 relative to the binade, 2^-10 below 2^-6)
+    scaled = a.astype(np.float64) / s[:, None].astype(np.float64)
+    quantum = np.where(np.abs(scaled) < 2.0 ** -6, 2.0 ** -9,
+                       np.ldexp(1.0, np.frexp(np.abs(scaled))[1] - 4))
+    assert np.all(np.abs(deq / s[:, None] - scaled) <= quantum / 2 * (1 + 1e-6) + 1e-30)
+
+
+def test_fp8_forward_against_plain_python_per_token():
+    """The FP8-weight layer, token by token in plain Python: per-token x scale, per-row weight
+    scales, h rounded to fp16 then quantized per row, routing and combine as in the 16-bit
+    layer."""
+    rng = np.random.default_rng(52)
+    T, d, E, k, F, Fs = 5, 8, 3, 2, 4, 4
+    L = _rand_layer(rng, T, d, E, F, Fs, scale=0.5)
+    L = {key: (None if v is None else v.astype(np.float32)) for key, v in L.items()}
+    fp8 = O.quantize_experts_fp8(L["w_gate"], L["w_up"], L["w_down"],
+                                 L["ws_gate"], L["ws_up"], L["ws_down"])
+    out = O.moe_forward_fp8(L["x"], L["w_router"], fp8, k)
+    ref_route = O.route(L["x"], L["w_router"], None, k)
+
+    def q_row(vals):
+        amax = max(abs(float(v)) for v in vals)
+        sc = float(np.float32(np.float32(amax) / np.float32(448.0))) if amax > 0 else 1.0
+        codes = [int(O.e4m3_round(np.float32(np.float32(v) / np.float32(sc)))) for v in vals]
+        return [float(O.e4m3_value(c)) * sc for c in codes]
+
+    def mat(w):  # dequantized rows of a weight matrix
+        return [q_row(r) for r in w.tolist()]
+
+    def ffn(xq, g, u, dn):
+        h = []
+        for f in range(len(g)):
+            a = math.fsum(xq[i] * g[f][i] for i in range(len(xq)))
+            b = math.fsum(xq[i] * u[f][i] for i in range(len(xq)))
+            h.append(float(np.float32(np.float16(a / (1.0 + math.exp(-a)) * b))))
+        hq = q_row(h)
+        return [math.fsum(hq[j] * dn[o][j] for j in range(len(hq))) for o in range(len(dn))]
+
+    for t in range(T):
+        xq = q_row(L["x"][t].tolist())
+        acc = [0.0] * d
+        for j in range(k):
+            e = int(ref_route[0][t, j])
+            o = ffn(xq, mat(L["w_gate"][e]), mat(L["w_up"][e]), mat(L["w_down"][e]))
+            acc = [a + ref_route[1][t, j] * v for a, v in zip(acc, o)]
+        sh = ffn(xq, mat(L["ws_gate"]), mat(L["ws_up"]), mat(L["ws_down"]))
+        want = [2.5 * a + b for a, b in zip(acc, sh)]
+        assert np.allclose(out["y"][t], want, rtol=1e-12, atol=1e-14), t
+
+
 # ---------------------------------------------------------------- padding mask
 
 def test_padding_token_gets_shared_expert_only():
