@@ -115,7 +115,8 @@ typedef struct {
 /* FP8 copies of the expert weights (moe_prepare_fp8 writes them; caller-owned
  * device memory).  Every row of every expert matrix (one output channel) is
  * stored as e4m3 codes with one float32 scale: s = amax(|row|) / 448 (1 for
- * an all-zero row), code = e4m3(w / s), round to nearest even, saturating. */
+ * an all-zero row), code = e4m3(w * (1 / s)), round to nearest even,
+ * saturating; every step a correctly rounded float32 operation. */
 typedef struct {
     void *w_gate;     /* [E, F, d] e4m3 */
     void *w_up;       /* [E, F, d] e4m3 */
@@ -219,7 +220,8 @@ moe_status moe_prepare_fp8(const moe_dims_t *dims, const moe_weights_t *weights,
  * (e4m3 codes, one float32 scale per row, as the weights); both expert GEMMs
  * run on e4m3 operands (tcgen05 kind::f8f6f4, fp32 accumulation) with the
  * row and column scales applied to the accumulator; h is held in fp16 and
- * quantized per row before the down projection; the combine is moe_forward's.
+ * quantized per row (power-of-two row scales) before the down projection; the
+ * combine is moe_forward's.
  * `weights` supplies the router (w_router, router_bias); dims->flags must
  * include MOE_FLAG_FP8_EXPERTS (workspace size).  The expert GEMMs always run
  * on single CTAs. */

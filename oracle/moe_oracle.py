@@ -230,11 +230,13 @@ def moe_forward(x, w_router, w_gate, w_up, w_down, k, *, router_bias=None,
 # FP8 expert weights for decode (the pages name FP8 deployment of the weights
 # but no scale layout; this build defines one): every row of every expert
 # matrix (an output channel), every token row of x and every row of h gets
-# its own float32 scale, s = amax(|row|) / 448 (s = 1 for an all-zero row),
-# and the row is stored as e4m3 codes q = e4m3(row / s), the division in
-# float32.  Products of codes are exact; the GEMMs accumulate in float32 and
-# apply the row and column scales to the accumulator.  h is held in fp16
-# before it is quantized, as in the 16-bit path.
+# its own float32 scale, s = amax(|row|) / 448 (s = 1 for an all-zero row;
+# for h rounded up to a power of two), and the row is stored as e4m3 codes
+# q = e4m3(v * r) with r = 1 / s, every step one correctly rounded float32
+# operation.  Products of codes are exact;
+# the GEMMs accumulate in float32 and apply the row and column scales to the
+# accumulator.  h is held in fp16 before it is quantized, as in the 16-bit
+# path.
 
 E4M3_MAX = 448.0
 
@@ -278,17 +280,33 @@ def e4m3_round(v):
     return code.astype(np.uint8)
 
 
-def quantize_rows_e4m3(a):
+def pow2_ceil_f32(t):
+    """Smallest power of two >= t for positive normal float32 t (2^-126 below the normal
+    range), by the float32 bit pattern."""
+    t = np.asarray(t, dtype=np.float32)
+    u = t.view(np.uint32)
+    up = ((u & np.uint32(0x7F800000)) + np.uint32(0x00800000)).astype(np.uint32)
+    r = np.where((u & np.uint32(0x007FFFFF)) != 0, up, u).astype(np.uint32)
+    r = np.where(u < np.uint32(0x00800000), np.uint32(0x00800000), r).astype(np.uint32)
+    return r.view(np.float32)
+
+
+def quantize_rows_e4m3(a, pow2=False):
     """Per-row e4m3 quantization of a float32 matrix [..., K] (last axis = row).
 
     Returns (codes uint8 [..., K], scales float32 [...]): s = amax / 448 in
-    float32 (1 for an all-zero row), codes = e4m3_round(float32(a / s)).
+    float32 (1 for an all-zero row), rounded up to a power of two when pow2
+    (h rows: then every code depends on its own element only), r = 1 / s in
+    float32, codes = e4m3_round(float32(a * r)).
     """
     a = np.asarray(a, dtype=np.float32)
     amax = np.max(np.abs(a), axis=-1)
-    s = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32), np.float32(1.0))
-    s = s.astype(np.float32)
-    codes = e4m3_round((a / s[..., None]).astype(np.float32))
+    t = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    if pow2:
+        t = pow2_ceil_f32(np.where(amax > 0, t, np.float32(1.0)))
+    s = np.where(amax > 0, t, np.float32(1.0)).astype(np.float32)
+    r = (np.float32(1.0) / s).astype(np.float32)
+    codes = e4m3_round((a * r[..., None]).astype(np.float32))
     return codes, s
 
 
@@ -319,7 +337,7 @@ def moe_forward_fp8(x, w_router, fp8, k, *, router_bias=None, routed_scaling_fac
         G = xrows @ dequantize_rows_e4m3(*g).T
         U = xrows @ dequantize_rows_e4m3(*u).T
         h = (silu(G) * U).astype(np.float16).astype(np.float32)
-        hq = dequantize_rows_e4m3(*quantize_rows_e4m3(h))
+        hq = dequantize_rows_e4m3(*quantize_rows_e4m3(h, pow2=True))
         return hq @ dequantize_rows_e4m3(*dn).T
 
     gq, gs = fp8["gate"]

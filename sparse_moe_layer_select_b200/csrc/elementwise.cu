@@ -98,11 +98,22 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 // Per-row e4m3 quantization (FP8 experts): one warp per row of K 16-bit
 // values (bf16 or fp16 by `is_f16`), s = amax / 448 (1 for an all-zero
-// row), codes = e4m3(v / s) with round to nearest even and saturation to
-// +-448; the division is the IEEE float32 one.  Rows from *n_valid on (if
-// given) are skipped.
+// row; rounded up to a power of two for h rows), r = 1 / s, codes = e4m3(v * r) with round to nearest even and
+// saturation to +-448; division, reciprocal and product are correctly
+// rounded float32 operations.  Rows from *n_valid on (if given) are skipped.
+// pow2 != 0: the scale is rounded up to a power of two (exact scaling, so an
+// element's code depends on that element alone).
+__device__ __forceinline__ float row_scale(float amax, int pow2) {
+  if (!(amax > 0.f)) return 1.f;
+  const float t = __fdiv_rn(amax, 448.f);
+  if (!pow2) return t;
+  const uint32_t u = __float_as_uint(t);
+  if (u < 0x00800000u) return __uint_as_float(0x00800000u);  // below the normal range: 2^-126
+  return (u & 0x007fffffu) ? __uint_as_float((u & 0x7f800000u) + 0x00800000u) : t;
+}
+
 __global__ void __launch_bounds__(256)
-    quant_rows_e4m3_kernel(const uint16_t *__restrict__ src, int is_f16, int rows,
+    quant_rows_e4m3_kernel(const uint16_t *__restrict__ src, int is_f16, int pow2, int rows,
                            const int32_t *__restrict__ n_valid, int K,
                            uint8_t *__restrict__ codes, float *__restrict__ scales) {
   const int lane = threadIdx.x & 31;
@@ -111,35 +122,58 @@ __global__ void __launch_bounds__(256)
   auto to_f32 = [&](uint16_t b) -> float {
     return is_f16 ? __half2float(__ushort_as_half(b)) : __uint_as_float(static_cast<uint32_t>(b) << 16);
   };
+  auto vec_amax = [&](const uint4 v, float m) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      m = fmaxf(m, fmaxf(fabsf(to_f32(w[q] & 0xffffu)), fabsf(to_f32(w[q] >> 16))));
+    return m;
+  };
+  auto vec_codes = [&](const uint4 v, float rcp) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = make_float2(__fmul_rn(to_f32(w[q] & 0xffffu), rcp),
+                                   __fmul_rn(to_f32(w[q] >> 16), rcp));
+      const uint32_t two = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+      packed[q >> 1] |= (two & 0xffffu) << (16 * (q & 1));
+    }
+    return make_uint2(packed[0], packed[1]);
+  };
+  constexpr int kRegVec = 16;  // rows of up to 32 * 16 * 8 = 4096 values stay in registers
+  const int nvec = K / 8;
   for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < nrows; r += warps) {
     const uint4 *row = reinterpret_cast<const uint4 *>(src + static_cast<size_t>(r) * K);
-    float amax = 0.f;
-    for (int c = lane; c < K / 8; c += 32) {
-      const uint4 v = row[c];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        amax = fmaxf(amax, fmaxf(fabsf(to_f32(w[q] & 0xffffu)), fabsf(to_f32(w[q] >> 16))));
-    }
-    // amax >= 0: its bits order as unsigned integers
-    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
-    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
     uint2 *out = reinterpret_cast<uint2 *>(codes + static_cast<size_t>(r) * K);
-    for (int c = lane; c < K / 8; c += 32) {
-      const uint4 v = row[c];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t packed[2] = {0u, 0u};
+    float amax = 0.f;
+    if (nvec <= 32 * kRegVec) {  // one read of the row
+      uint4 v[kRegVec];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t lo = __nv_cvt_float_to_fp8(__fdiv_rn(to_f32(w[q] & 0xffffu), scale),
-                                                  __NV_SATFINITE, __NV_E4M3);
-        const uint32_t hi = __nv_cvt_float_to_fp8(__fdiv_rn(to_f32(w[q] >> 16), scale),
-                                                  __NV_SATFINITE, __NV_E4M3);
-        packed[q >> 1] |= (lo | (hi << 8)) << (16 * (q & 1));
+      for (int j = 0; j < kRegVec; ++j) {
+        const int c = lane + 32 * j;
+        v[j] = c < nvec ? row[c] : make_uint4(0, 0, 0, 0);
       }
-      out[c] = make_uint2(packed[0], packed[1]);
+#pragma unroll
+      for (int j = 0; j < kRegVec; ++j) amax = vec_amax(v[j], amax);
+      // amax >= 0: its bits order as unsigned integers
+      amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+      const float scale = row_scale(amax, pow2);
+      const float rcp = __frcp_rn(scale);
+#pragma unroll
+      for (int j = 0; j < kRegVec; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nvec) out[c] = vec_codes(v[j], rcp);
+      }
+      if (lane == 0) scales[r] = scale;
+    } else {  // longer rows: read twice
+      for (int c = lane; c < nvec; c += 32) amax = vec_amax(row[c], amax);
+      amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+      const float scale = row_scale(amax, pow2);
+      const float rcp = __frcp_rn(scale);
+      for (int c = lane; c < nvec; c += 32) out[c] = vec_codes(row[c], rcp);
+      if (lane == 0) scales[r] = scale;
     }
-    if (lane == 0) scales[r] = scale;
   }
 }
 
@@ -237,13 +271,13 @@ cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_rows_e4m3(const uint16_t *src, bool is_f16, int rows,
+cudaError_t launch_quant_rows_e4m3(const uint16_t *src, bool is_f16, bool pow2, int rows,
                                   const int32_t *n_valid, int K, uint8_t *codes, float *scales,
                                   cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const size_t threads = static_cast<size_t>(rows) * 32;
-  quant_rows_e4m3_kernel<<<grid_for(threads, 256), 256, 0, s>>>(src, is_f16 ? 1 : 0, rows, n_valid,
-                                                               K, codes, scales);
+  quant_rows_e4m3_kernel<<<grid_for(threads, 256), 256, 0, s>>>(src, is_f16 ? 1 : 0, pow2 ? 1 : 0,
+                                                               rows, n_valid, K, codes, scales);
   return cudaGetLastError();
 }
 

@@ -190,6 +190,7 @@ constexpr float kRefineBand = 2e-4f;
 __device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item &it,
                                                        uint32_t taddr, int row_local,
                                                        const float *bias_s) {
+  if ((row_local >> 5) * 32 >= it.nrows) return;  // no valid row in this warp's quarter
   const bool valid = row_local < it.nrows;
   const int e0 = it.j * p.n_tile;  // this item's block of experts
   float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E + e0;
@@ -258,17 +259,40 @@ __device__ __forceinline__ float swiglu(float g, float u) {
   return __fdividef(g, 1.f + __expf(-g)) * u;
 }
 
-// acc[i] *= rs * col_scale[i] for N accumulator columns (MODE_F8 epilogues:
-// token or h row scale rs, weight-row scale of each column).
-template <int N>
-__device__ __forceinline__ void scale_cols(uint32_t (&acc)[N], float rs, const float *col_scale) {
+// MODE_F8 epilogues: the weight-row scales of an item's columns, 8 per lane
+// (lane l holds columns 8l .. 8l+7 of a 256-column block, or 4l .. 4l+3 of
+// a 128-column one), loaded once per item; a 16-column chunk takes its 16
+// scales by warp shuffle.
+struct ColScales {
+  float4 a, b;
+};
+
+template <int PER_LANE>  // 4 or 8
+__device__ __forceinline__ ColScales load_col_scales(const float *src, int lane) {
+  ColScales c;
+  c.a = *reinterpret_cast<const float4 *>(src + PER_LANE * lane);
+  c.b = PER_LANE == 8 ? *reinterpret_cast<const float4 *>(src + PER_LANE * lane + 4) : c.a;
+  return c;
+}
+
+__device__ __forceinline__ float pick(const ColScales &c, int e) {  // e: compile-time 0..7
+  const float4 &v = e < 4 ? c.a : c.b;
+  switch (e & 3) {
+    case 0: return v.x;
+    case 1: return v.y;
+    case 2: return v.z;
+    default: return v.w;
+  }
+}
+
+// acc[i] *= rs * scale(column c0 + i), i < 16, c0 a multiple of 16.
+template <int PER_LANE>
+__device__ __forceinline__ void scale_chunk16(uint32_t (&acc)[16], float rs, const ColScales &c,
+                                              int c0) {
 #pragma unroll
-  for (int i = 0; i < N; i += 4) {
-    const float4 c = *reinterpret_cast<const float4 *>(col_scale + i);
-    acc[i] = __float_as_uint(__uint_as_float(acc[i]) * rs * c.x);
-    acc[i + 1] = __float_as_uint(__uint_as_float(acc[i + 1]) * rs * c.y);
-    acc[i + 2] = __float_as_uint(__uint_as_float(acc[i + 2]) * rs * c.z);
-    acc[i + 3] = __float_as_uint(__uint_as_float(acc[i + 3]) * rs * c.w);
+  for (int i = 0; i < 16; ++i) {
+    const float sc = __shfl_sync(0xffffffffu, pick(c, i % PER_LANE), (c0 + i) / PER_LANE);
+    acc[i] = __float_as_uint(__uint_as_float(acc[i]) * rs * sc);
   }
 }
 
@@ -281,6 +305,7 @@ __device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item 
                                                 const CUtensorMap *tm_h, const CUtensorMap *tm_hsh) {
   const bool shared = it.group == p.E;
   const int q = row_local >> 5;
+  if (q * 32 >= it.nrows) return;  // no valid row in this warp's quarter (warp-uniform)
   const int lane = row_local & 31;
   const bool valid = row_local < it.nrows;
   const bool full_box = (q + 1) * 32 <= it.nrows;
@@ -288,14 +313,16 @@ __device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item 
                              : p.h + static_cast<size_t>(it.row0 + row_local) * p.F;
   const int col0 = it.j * p.n_half;
   float rs = 1.f;
-  const float *sg = nullptr, *su = nullptr;
-  if (F8) {
+  ColScales cg{}, cu{};
+  if (F8) {  // n_half = 128 columns of gate and of up: 4 scales of each per lane
     if (valid) {
       const int tok = shared ? it.row0 + row_local : p.perm[it.row0 + row_local] / p.k;
       rs = p.sx[tok];
     }
-    sg = (shared ? p.sb0_sh : p.sb0 + static_cast<size_t>(it.group) * p.F) + col0;
-    su = (shared ? p.sb1_sh : p.sb1 + static_cast<size_t>(it.group) * p.F) + col0;
+    cg = load_col_scales<4>((shared ? p.sb0_sh : p.sb0 + static_cast<size_t>(it.group) * p.F) + col0,
+                            lane);
+    cu = load_col_scales<4>((shared ? p.sb1_sh : p.sb1 + static_cast<size_t>(it.group) * p.F) + col0,
+                            lane);
   }
   float amax = 0.f;
   for (int cb = 0; cb < p.n_half; cb += 64) {
@@ -307,8 +334,8 @@ __device__ __forceinline__ void swiglu_epilogue(const GemmParams &p, const Item 
       tmem_ld_32x32b_x16(taddr + p.n_half + cb + 16 * qu, u);
       tmem_ld_wait();
       if (F8) {
-        scale_cols<16>(g, rs, sg + cb + 16 * qu);
-        scale_cols<16>(u, rs, su + cb + 16 * qu);
+        scale_chunk16<4>(g, rs, cg, cb + 16 * qu);
+        scale_chunk16<4>(u, rs, cu, cb + 16 * qu);
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -333,6 +360,7 @@ __device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &i
                                               const CUtensorMap *tm_o, const CUtensorMap *tm_s) {
   const bool shared = it.group == p.E;
   const int q = row_local >> 5;
+  if (q * 32 >= it.nrows) return;  // no valid row in this warp's quarter (warp-uniform)
   const int lane = row_local & 31;
   const bool valid = row_local < it.nrows;
   const bool full_box = (q + 1) * 32 <= it.nrows;
@@ -340,10 +368,11 @@ __device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &i
   if (valid && !shared) scale = p.routed_scale * p.topk_w[p.perm[it.row0 + row_local]];
   uint16_t *row_dst = (shared ? p.s_out : p.o_out) + static_cast<size_t>(it.row0 + row_local) * p.d;
   const int col0 = it.j * p.n_tile;
-  const float *sd = nullptr;
-  if (F8) {  // h row scale, then each column's weight-row scale
+  ColScales cd{};
+  if (F8) {  // h row scale, then each column's weight-row scale (n_tile = 256: 8 per lane)
     if (valid) scale *= shared ? p.sa_sh[it.row0 + row_local] : p.sa[it.row0 + row_local];
-    sd = (shared ? p.sb0_sh : p.sb0 + static_cast<size_t>(it.group) * p.d) + col0;
+    cd = load_col_scales<8>((shared ? p.sb0_sh : p.sb0 + static_cast<size_t>(it.group) * p.d) + col0,
+                            lane);
   }
   float amax = 0.f;
   for (int cb = 0; cb < p.n_tile; cb += 64) {
@@ -353,7 +382,7 @@ __device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &i
       uint32_t r[16];
       tmem_ld_32x32b_x16(taddr + cb + 16 * qu, r);
       tmem_ld_wait();
-      if (F8) scale_cols<16>(r, 1.f, sd + cb + 16 * qu);
+      if (F8) scale_chunk16<8>(r, 1.f, cd, cb + 16 * qu);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float v0 = __uint_as_float(r[2 * i]) * scale;

@@ -119,8 +119,9 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, const int
 cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32_t *inv, int T,
                            int k, int d, uint16_t *y, cudaStream_t s);
 // Per-row e4m3 codes and float32 scales of a [rows, K] bf16 (or fp16) matrix;
-// K % 8 == 0; rows from *n_valid on (if given) are skipped.
-cudaError_t launch_quant_rows_e4m3(const uint16_t *src, bool is_f16, int rows,
+// K % 8 == 0; rows from *n_valid on (if given) are skipped; pow2: power-of-two
+// scales.
+cudaError_t launch_quant_rows_e4m3(const uint16_t *src, bool is_f16, bool pow2, int rows,
                                   const int32_t *n_valid, int K, uint8_t *codes, float *scales,
                                   cudaStream_t s);
 cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int *status,

@@ -197,8 +197,9 @@ moe_status check_dims(const moe_dims_t *dims, Dims *D) {
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((dims->flags & MOE_FLAG_ROUTER_TENSOR) && (D->E % 16 != 0 || D->E > 256))
     return MOE_ERR_UNSUPPORTED_SHAPE;
-  // FP8 experts: K stages of 128 e4m3 elements
-  if ((dims->flags & MOE_FLAG_FP8_EXPERTS) && (D->F % 128 != 0 || D->Fs % 128 != 0))
+  // FP8 experts: K stages of 128 e4m3 elements; 256-column down-projection tiles
+  if ((dims->flags & MOE_FLAG_FP8_EXPERTS) &&
+      (D->F % 128 != 0 || D->Fs % 128 != 0 || D->d % 256 != 0))
     return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
@@ -459,8 +460,8 @@ moe_status moe_prepare_fp8(const moe_dims_t *dims, const moe_weights_t *w,
   int launches = 0;
   for (const Job &j : jobs) {
     if (j.rows == 0) continue;
-    if (launch_quant_rows_e4m3(static_cast<const uint16_t *>(j.src), false, j.rows, nullptr, j.K,
-                               static_cast<uint8_t *>(j.codes), j.scales, s) != cudaSuccess)
+    if (launch_quant_rows_e4m3(static_cast<const uint16_t *>(j.src), false, false, j.rows, nullptr,
+                               j.K, static_cast<uint8_t *>(j.codes), j.scales, s) != cudaSuccess)
       return MOE_ERR_CUDA;
     ++launches;
   }
@@ -523,8 +524,8 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
   uint8_t *xq = reinterpret_cast<uint8_t *>(wsp(ws, L.xq));
   float *sx = reinterpret_cast<float *>(wsp(ws, L.sx));
   if (fp8) {
-    if (launch_quant_rows_e4m3(static_cast<const uint16_t *>(x), false, D.T, nullptr, D.d, xq, sx,
-                               s) != cudaSuccess)
+    if (launch_quant_rows_e4m3(static_cast<const uint16_t *>(x), false, false, D.T, nullptr, D.d,
+                               xq, sx, s) != cudaSuccess)
       return MOE_ERR_CUDA;
     launches += 1;
   }
@@ -630,12 +631,13 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
   uint8_t *hshq = reinterpret_cast<uint8_t *>(wsp(ws, L.hshq));
   float *shs = reinterpret_cast<float *>(wsp(ws, L.shs));
   if (fp8) {
-    if (launch_quant_rows_e4m3(h, true, n_rows, routing->offsets + D.E, D.F, hq, shq, s) !=
+    // h rows: power-of-two scales (see launch_quant_rows_e4m3)
+    if (launch_quant_rows_e4m3(h, true, true, n_rows, routing->offsets + D.E, D.F, hq, shq, s) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
     launches += 1;
     if (D.Fs > 0) {
-      if (launch_quant_rows_e4m3(h_sh, true, D.T, nullptr, D.Fs, hshq, shs, s) != cudaSuccess)
+      if (launch_quant_rows_e4m3(h_sh, true, true, D.T, nullptr, D.Fs, hshq, shs, s) != cudaSuccess)
         return MOE_ERR_CUDA;
       launches += 1;
     }

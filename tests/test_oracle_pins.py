@@ -403,6 +403,27 @@ def test_e4m3_ties_go_to_even_and_large_values_saturate():
     assert np.all(O.e4m3_round(big) == 0x7E) and np.all(O.e4m3_round(-big) == 0xFE)
 
 
+def test_power_of_two_row_scales():
+    """pow2 scales: the smallest power of two >= amax / 448, so every scaled value lies in
+    (-448, 448] and scaling is exact (codes depend on each element alone)."""
+    rng = np.random.default_rng(53)
+    a = (rng.standard_normal((30, 64)) * 10.0 ** rng.uniform(-4, 3, (30, 1))).astype(np.float32)
+    a[0, :] = 0.0
+    a[1, :] = 0.0
+    a[1, :3] = [448.0, -1.0, 2.0]      # amax / 448 = 1 exactly: the scale stays 1
+    codes, s = O.quantize_rows_e4m3(a, pow2=True)
+    mant, ex = np.frexp(s.astype(np.float64))
+    assert np.all(mant == 0.5)                                     # powers of two
+    t = np.max(np.abs(a), axis=1).astype(np.float32) / np.float32(448.0)
+    nz = t > 0
+    assert np.all(s[nz] >= t[nz]) and np.all(s[nz] / 2 < t[nz]) and s[0] == 1.0 and s[1] == 1.0
+    assert np.all(np.abs(O.e4m3_value(codes)) <= 448.0)
+    # exact scaling: the codes equal those of each element divided by the scale
+    want = O.e4m3_round((a.astype(np.float64) / s[:, None]).astype(np.float32))
+    same = (codes == want) | ((O.e4m3_value(codes) == 0) & (O.e4m3_value(want) == 0))
+    assert same.all()
+
+
 def test_per_row_quantization_error_bound():
     rng = np.random.default_rng(51)
     a = (rng.standard_normal((40, 300)) * 10.0 ** rng.uniform(-3, 2, (40, 1))).astype(np.float32)
@@ -431,10 +452,13 @@ def test_fp8_forward_against_plain_python_per_token():
     out = O.moe_forward_fp8(L["x"], L["w_router"], fp8, k)
     ref_route = O.route(L["x"], L["w_router"], None, k)
 
-    def q_row(vals):
+    def q_row(vals, pow2=False):
         amax = max(abs(float(v)) for v in vals)
         sc = float(np.float32(np.float32(amax) / np.float32(448.0))) if amax > 0 else 1.0
-        codes = [int(O.e4m3_round(np.float32(np.float32(v) / np.float32(sc)))) for v in vals]
+        if pow2 and amax > 0:
+            sc = 2.0 ** math.ceil(math.log2(sc))  # exact for these (normal) values
+        rc = np.float32(np.float32(1.0) / np.float32(sc))
+        codes = [int(O.e4m3_round(np.float32(np.float32(v) * rc))) for v in vals]
         return [float(O.e4m3_value(c)) * sc for c in codes]
 
     def mat(w):  # dequantized rows of a weight matrix
@@ -446,7 +470,7 @@ def test_fp8_forward_against_plain_python_per_token():
             a = math.fsum(xq[i] * g[f][i] for i in range(len(xq)))
             b = math.fsum(xq[i] * u[f][i] for i in range(len(xq)))
             h.append(float(np.float32(np.float16(a / (1.0 + math.exp(-a)) * b))))
-        hq = q_row(h)
+        hq = q_row(h, pow2=True)
         return [math.fsum(hq[j] * dn[o][j] for j in range(len(hq))) for o in range(len(dn))]
 
     for t in range(T):
