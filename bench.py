@@ -70,6 +70,27 @@ def measured_traffic(workload, stage, fp8=False):
     return e["dram_bytes_per_launch"]
 
 
+def max_over_ranks(value, world, device="cuda"):
+    """The largest of every rank's value (each rank calls it); the value itself for one rank."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_step, steps, world, seconds):
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_step * steps * world / seconds
+
+
+def replica_seed(w, rank):
+    """Seed of a replica's token batch: rank 0 uses the workload's seed, the others their own."""
+    return w.seed + rank
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -220,7 +241,7 @@ def run_ours(args):
     w = I.get(args.workload)
     dev = I.device_inputs(w)
     if rank > 0:  # each replica routes its own tokens
-        I.generate_cuda(dev["x"], w.seed + rank, I.TID_X, w.sigma_x)
+        I.generate_cuda(dev["x"], replica_seed(w, rank), I.TID_X, w.sigma_x)
     decode = w.decode_batches > 0
     ring = I.device_decode_ring(w, min(w.decode_batches, 1000)) if decode else None
     layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
@@ -299,17 +320,14 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    # the timed steps carry no stage markers (events between the layer's kernels would
-    # break their programmatic overlap); a second, marked pass gives the stage times
+    # the timed steps carry no stage markers (events recorded between the layer's kernels);
+    # a second, marked pass gives the stage times
     elapsed = timed_loop()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([elapsed], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, world)
     code, site = M.read_device_status(layer.ws)
     if code != 0:
         raise RuntimeError(f"device status {M.status_string(code)} at site {site}")
@@ -390,12 +408,8 @@ def run_ours(args):
         s_out.wait_event(last)
         b.record(s_out)
         torch.cuda.synchronize()
-        te = a.elapsed_time(b) / 1e3
-        if world > 1:
-            t = torch.tensor([te], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            te = float(t.item())
-        e2e = {"value": w.T * args.steps * world / te, "unit": "tokens/s",
+        te = max_over_ranks(a.elapsed_time(b) / 1e3, world)
+        e2e = {"value": job_tokens_per_s(w.T, args.steps, world, te), "unit": "tokens/s",
                "h2d_bytes_per_step": w.T * w.d_model * 2, "d2h_bytes_per_step": w.T * w.d_model * 2,
                "overlap": "input copy, layer and output copy on three streams, two buffers"}
 
@@ -447,7 +461,8 @@ def run_ours(args):
                          f"({secs:.1f} s)"}
 
     line = {
-        "metric": METRIC, "value": w.T * args.steps * world / elapsed, "unit": "tokens/s",
+        "metric": METRIC, "value": job_tokens_per_s(w.T, args.steps, world, elapsed),
+        "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16",

@@ -1,0 +1,72 @@
+"""Host-side logic of the multi-GPU bench path (replicas), on CPU with gloo ranks."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, port, results):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=2)
+    try:
+        elapsed = 0.25 + 0.5 * rank                     # the slower rank sets the job time
+        slowest = bench.max_over_ranks(elapsed, 2, device="cpu")
+        value = bench.job_tokens_per_s(4096, 10, 2, slowest)
+        results.put((rank, slowest, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_job_throughput_with_two_gloo_ranks():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.SimpleQueue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get() for _ in range(2))
+    for rank, slowest, value in got:
+        assert slowest == 0.75                            # max over the ranks, on every rank
+        assert value == 4096 * 10 * 2 / 0.75              # all ranks' tokens / slowest time
+
+
+def test_replica_seeds_differ_per_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_moe_layer_select_b200 import inputs as I
+    w = I.get("c2_xs2_small")
+    seeds = [bench.replica_seed(w, r) for r in range(8)]
+    assert seeds[0] == w.seed and len(set(seeds)) == 8
+
+
+@pytest.mark.parametrize("rank,world,lines", [(1, 2, 0), (0, 1, 1)])
+def test_reference_arm_prints_on_rank_zero_only(rank, world, lines):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3", "--workload", "c1_tiny"],
+                       capture_output=True, text=True, env=env, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(out) == lines
+    if lines:
+        d = json.loads(out[0])
+        assert d["impl"] == "reference" and d["config"]["workload"] == "c1_tiny"
+        assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
