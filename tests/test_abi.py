@@ -90,6 +90,42 @@ def test_argument_errors_return_before_any_launch(L):
     assert _call_forward(f) == M.MOE_ERR_UNSUPPORTED_SHAPE
 
 
+def _fp8_struct(missing=None):
+    vals = {n: (1 << 24) + 4096 * i for i, n in enumerate(M.FP8_FIELDS)}
+    if missing:
+        vals[missing] = None
+    return M.moe_fp8_weights_t(*[vals[n] for n in M.FP8_FIELDS])
+
+
+def _call_forward_fp8(dims, q=None, x=256, y=512, ws=4096, ws_bytes=1 << 40):
+    w = M.moe_weights_t(1024, None, 2048, 4096, 8192, 16384, 32768, 65536)
+    r = M.moe_routing_t(1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20)
+    q = q or _fp8_struct()
+    return M.lib().moe_forward_fp8(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(q),
+                                   ctypes.c_void_p(x), ctypes.c_void_p(y), ctypes.byref(r),
+                                   ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def test_fp8_argument_errors_return_before_any_launch(L):
+    f8 = M.MOE_FLAG_FP8_EXPERTS
+    d = M.make_dims(64, 256, 16, 4, 128, 128, flags=f8)
+    # e4m3 rows of x and h on top of a workspace without the per-call fp16 copy of W_down
+    assert M.workspace_size(d) > M.workspace_size(
+        M.make_dims(64, 256, 16, 4, 128, 128, flags=M.MOE_FLAG_DOWN_F16))
+    assert _call_forward_fp8(M.make_dims(64, 256, 16, 4, 128, 128)) == M.MOE_ERR_INVALID_ARG
+    assert M.workspace_size(M.make_dims(64, 256, 16, 4, 192, 128, flags=f8)) == 0
+    assert _call_forward_fp8(M.make_dims(64, 256, 16, 4, 192, 128, flags=f8)) == \
+        M.MOE_ERR_UNSUPPORTED_SHAPE                                        # F % 128
+    assert _call_forward_fp8(M.make_dims(64, 384, 16, 4, 128, 128, flags=f8)) == \
+        M.MOE_ERR_UNSUPPORTED_SHAPE                                        # d % 256
+    assert _call_forward_fp8(d, q=_fp8_struct("s_down")) == M.MOE_ERR_INVALID_ARG
+    assert _call_forward_fp8(d, q=_fp8_struct("ss_gate")) == M.MOE_ERR_INVALID_ARG
+    assert _call_forward_fp8(d, x=256 + 8) == M.MOE_ERR_INVALID_ARG
+    # the 16-bit forward cannot use a workspace sized for FP8 without prepared fp16 W_down
+    assert _call_forward(d) == M.MOE_ERR_INVALID_ARG
+    assert _call_forward_fp8(M.make_dims(0, 256, 16, 4, 128, 128, flags=f8)) == M.MOE_OK
+
+
 def test_zero_tokens_is_a_noop(L):
     d = M.make_dims(0, 256, 16, 4, 128, 128)
     assert _call_forward(d) == M.MOE_OK
