@@ -317,7 +317,15 @@ def dequantize_rows_e4m3(codes, scales):
 def quantize_experts_fp8(w_gate, w_up, w_down, ws_gate=None, ws_up=None, ws_down=None):
     """FP8 copies of the expert weights (bf16 bit patterns or floats in), one
     scale per output row: gate/up [E, F] (rows of [E, F, d]), down [E, d]."""
-    f = lambda w: None if w is None else quantize_rows_e4m3(bf16_to_f64(w).astype(np.float32))
+    def f(w):
+        if w is None:
+            return None
+        w = np.asarray(w)
+        if w.ndim == 2:
+            return quantize_rows_e4m3(bf16_to_f64(w).astype(np.float32))
+        parts = [quantize_rows_e4m3(bf16_to_f64(w[e]).astype(np.float32))  # expert by expert
+                 for e in range(w.shape[0])]
+        return np.stack([c for c, _ in parts]), np.stack([sc for _, sc in parts])
     return {"gate": f(w_gate), "up": f(w_up), "down": f(w_down),
             "s_gate": f(ws_gate), "s_up": f(ws_up), "s_down": f(ws_down)}
 

@@ -252,18 +252,20 @@ def test_fp8_forward_matches_fp8_oracle(T):
 
 @pytest.mark.parametrize("Fs", [0, 512])
 def test_fp8_xs2_widths_full_oracle(Fs):
-    """FP8 experts at the XS.2 widths (d=2048, E=256, top-8, F=512), T=600 (ragged tiles
-    everywhere), with and without the shared expert."""
+    """FP8 experts at the XS.2 widths (d=2048, F=512; 16 experts, top-4 keep the float64
+    oracle's weight quantization short), T=600 (ragged tiles everywhere), with and without
+    the shared expert."""
     import torch
-    w = I.get("c2_xs2_small").with_(T=600, shared_intermediate_size=Fs)
+    w = I.get("c2_xs2_small").with_(T=600, num_experts=16, num_experts_per_tok=4,
+                                    shared_intermediate_size=Fs)
     h, dev = _small(w)
     layer = M.MoeLayer(dev, w.d_model, w.E, w.k, w.F, w.Fs, w.routed_scaling_factor,
                        max_tokens=w.T, fp8=True)
     y = layer.forward(dev["x"])
     torch.cuda.synchronize()
     assert M.read_device_status(layer.ws)[0] == 0
-    fp8 = O.quantize_experts_fp8(h["w_gate"], h["w_up"], h["w_down"], h["ws_gate"], h["ws_up"],
-                                 h["ws_down"])
+    fp8 = O.quantize_experts_fp8(h["w_gate"], h["w_up"], h["w_down"], h.get("ws_gate"),
+                                 h.get("ws_up"), h.get("ws_down"))
     ref = O.moe_forward_fp8(h["x"], h["w_router"], fp8, w.k,
                             routed_scaling_factor=w.routed_scaling_factor)
     gidx = layer.routing["topk_idx"][:w.T].cpu().numpy()
