@@ -233,9 +233,9 @@ def run_ours(args):
     from tests import parity as P  # bf16 -> numpy helper only
 
     world, rank, local = dist_env()
+    torch.cuda.set_device(local)
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
     M.lib()
 
     w = I.get(args.workload)
