@@ -44,15 +44,42 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
+def _code_tokens(text):
+    """C/C++/CUDA source with comments removed and whitespace collapsed, so that a
+    comment-only edit leaves the hash (and the traffic keyed to it) unchanged."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (" ".join(line.split()) for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_sources_sha1():
-    """Hash of the CUDA sources: DRAM traffic taken by ncu is valid only for these."""
+    """Hash of the CUDA sources' code (comments and blank space ignored): DRAM traffic
+    taken by ncu is valid only for these."""
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "sparse_moe_layer_select_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + b"\0" + _code_tokens(f.read()).encode())
     return h.hexdigest()
 
 
@@ -282,8 +309,9 @@ def run_ours(args):
     if code != 0:
         raise RuntimeError(f"device status {M.status_string(code)} at site {site}")
     launches_per_step = M.last_launch_count() + (1 if decode else 0)
-    if decode and not args.no_graph:
-        # decode: the layer is captured once in a CUDA graph and replayed per batch
+    if not args.no_graph:
+        # the layer is captured once in a CUDA graph and replayed per step (decode: per
+        # fresh batch copied into the same input buffer)
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
@@ -335,11 +363,12 @@ def run_ours(args):
     stage_ms = {}
     marked_ms = None
     if graph is not None:
-        # events recorded inside a graph cannot be timed: the stage breakdown of the
-        # decode workload comes from five eager calls after the timed graph replays
+        # events recorded inside a graph cannot be timed: the stage breakdown comes from
+        # five eager calls after the timed graph replays
         acc = np.zeros(len(M.FORWARD_STAGES))
         for i in range(5):
-            x_buf.copy_(ring[i % ring.shape[0]], non_blocking=True)
+            if decode:
+                x_buf.copy_(ring[i % ring.shape[0]], non_blocking=True)
             evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(M.FORWARD_STAGES) + 1)]
             M.profile_next_forward(evs)
             layer.forward(x_buf, y)
@@ -559,7 +588,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
-                    help="decode: launch each step instead of replaying a CUDA graph")
+                    help="launch each step's kernels instead of replaying a CUDA graph")
     ap.add_argument("--single-cta", action="store_true",
                     help="force the single-CTA (M=128) expert GEMM engine")
     ap.add_argument("--pair", action="store_true",

@@ -17,15 +17,20 @@
 //                expert and one d-column block; the
 //                epilogue multiplies each row by routed_scaling_factor * w
 //                (the 2.5 modulation of the routed sum: Technical Report
-//                summary, report §3.1) and writes it, in fp16, to that
-//                (token, slot)'s row of the slot buffer; shared-expert rows go
-//                to the last slot with scale 1.
+//                summary, report §3.1) and writes it, in fp16, to its
+//                expert-order row of O (the combine reads O through the
+//                inverse permutation); shared-expert rows go, unscaled, to
+//                the token's row of S.
+//   MODE_F8 | *  the same two expert GEMMs on e4m3 operands (tcgen05
+//                kind::f8f6f4, K=32 per instruction); the epilogues apply the
+//                per-row activation scale and per-column weight scale.
 //
 // Roles inside a CTA (one CTA per SM, persistent over items):
 //   warp 0      producer: fills a kStages-deep ring of (A, B) stages with
 //               TMA tiles (GEMM1: the B tiles only).
-//   warps 6..   GEMM1: gather the A rows by cp.async through the expert-order
-//               permutation, a share of the 128 rows each (gemm_common.cuh).
+//   warps 6..   GEMM1: kGatherWarps warps gather the A rows by cp.async
+//               through the expert-order permutation, an equal share of the
+//               128 rows each (gemm_common.cuh).
 //   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma
 //               (M=128, N<=256, K=16 per instruction) into one of two
 //               accumulator buffers and commits stage releases.

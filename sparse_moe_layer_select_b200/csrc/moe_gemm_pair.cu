@@ -107,7 +107,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_b0);
     prefetch_tmap(&tm_b1);
-    prefetch_tmap(&tm_a);  // GEMM1: the gather4 map of x (one-row boxes)
+    prefetch_tmap(&tm_a);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kPTmemCols);

@@ -1,11 +1,9 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers with bounded
-// waits, TMA tile / gather4 loads, and the tcgen05 (5th-generation tensor
+// waits, TMA tile loads and stores, cp.async, and the tcgen05 (5th-generation tensor
 // core + tensor memory) instructions used by the expert and router GEMMs.
 //
 // Written from the PTX ISA descriptions of these instructions.  No cluster
-// multicast form is used anywhere in this library.  (tile::gather4 is kept
-// for reference; the expert GEMM gathers rows with cp.async instead, which
-// moves 512 bytes per warp instruction against 512 bytes per TMA gather4.)
+// multicast form is used anywhere in this library.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -106,19 +104,6 @@ __device__ __forceinline__ void bulk_wait_read_le1() {
 // Wait until all of this thread's bulk groups have completed.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// Row gather: four rows (r0..r3) of one column box, written as four
-// consecutive box rows.  The tensor map's box is one row high.
-__device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, uint64_t *bar,
-                                            int32_t col, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
 }
 
 // 16-byte asynchronous global->shared copy (cp.async, L2-only caching).

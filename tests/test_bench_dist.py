@@ -70,3 +70,26 @@ def test_reference_arm_prints_on_rank_zero_only(rank, world, lines):
         d = json.loads(out[0])
         assert d["impl"] == "reference" and d["config"]["workload"] == "c1_tiny"
         assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_source_hash_ignores_comments_but_not_code():
+    sys.path.insert(0, ROOT)
+    import bench
+    base = 'int f(int a) {  // doubles a\n  return a * 2;  /* "x" */\n}\n'
+    comments = '// header\nint f(int a) {\n\n  return a * 2;\n}\n/* trailer\n   two lines */\n'
+    code = 'int f(int a) {\n  return a * 3;\n}\n'
+    literal = 'const char *s = "// not a comment";\n'
+    assert bench._code_tokens(base) == bench._code_tokens(comments)
+    assert bench._code_tokens(base) != bench._code_tokens(code)
+    assert "// not a comment" in bench._code_tokens(literal)
+
+
+def test_stored_traffic_matches_the_sources():
+    sys.path.insert(0, ROOT)
+    import bench
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        stored = json.load(f)
+    if stored.get("sources_sha1") != bench.kernel_sources_sha1():
+        assert bench.measured_traffic("c3_xs2_prefill_zipf", "gemm1_swiglu") is None
+    else:
+        assert bench.measured_traffic("c3_xs2_prefill_zipf", "gemm1_swiglu") is not None
