@@ -285,9 +285,11 @@ def run_ours(args):
     graph = None
 
     def step(i, events=None):
+        """One step: a graph replay when a graph is captured, else (and always for the
+        stage-marked pass) the layer's kernels launched one by one."""
         if decode:
             x_buf.copy_(ring[i % ring.shape[0]], non_blocking=True)
-        if graph is not None:
+        if graph is not None and events is None:
             graph.replay()
             return
         if events is not None:
@@ -360,30 +362,15 @@ def run_ours(args):
     if code != 0:
         raise RuntimeError(f"device status {M.status_string(code)} at site {site}")
 
-    stage_ms = {}
-    marked_ms = None
-    if graph is not None:
-        # events recorded inside a graph cannot be timed: the stage breakdown comes from
-        # five eager calls after the timed graph replays
-        acc = np.zeros(len(M.FORWARD_STAGES))
-        for i in range(5):
-            if decode:
-                x_buf.copy_(ring[i % ring.shape[0]], non_blocking=True)
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(M.FORWARD_STAGES) + 1)]
-            M.profile_next_forward(evs)
-            layer.forward(x_buf, y)
-            torch.cuda.synchronize()
-            acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(M.FORWARD_STAGES))]
-        for j, name in enumerate(M.FORWARD_STAGES):
-            stage_ms[name] = float(acc[j] / 5)
-    else:
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
-              for _ in range(args.steps)]
-        marked_elapsed = timed_loop(ev)
-        for j, name in enumerate(M.FORWARD_STAGES):
-            stage_ms[name] = float(np.mean([ev[i][j].elapsed_time(ev[i][j + 1])
-                                            for i in range(args.steps)]))
-        marked_ms = marked_elapsed / args.steps * 1e3
+    # stage times: K more steps, launched eagerly with an event at each stage boundary
+    # (events recorded inside a captured graph cannot be timed)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
+          for _ in range(args.steps)]
+    marked_elapsed = timed_loop(ev)
+    stage_ms = {name: float(np.mean([ev[i][j].elapsed_time(ev[i][j + 1])
+                                     for i in range(args.steps)]))
+                for j, name in enumerate(M.FORWARD_STAGES)}
+    marked_ms = marked_elapsed / args.steps * 1e3
 
     # end to end through the C ABI: pinned host batch in, host output back, every step
     e2e = None
