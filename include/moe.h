@@ -241,7 +241,10 @@ moe_status moe_prepare_down_f16(const moe_dims_t *dims, const void *w_down, cons
                                 void *stream);
 
 /* Byte offset of the fp32 router logits [T, E] (bias included) that
- * moe_route and moe_forward leave in the workspace. */
+ * moe_route and moe_forward leave in the workspace.  (For small T the
+ * tensor-core router splits d into up to 4 slices; their partial logits sit
+ * in the planes after this one, and the selection kernel sums them, in slice
+ * order, into this plane.) */
 size_t moe_logits_offset(const moe_dims_t *dims);
 
 /* Synchronises `stream`, then returns the device-side status word of `ws`

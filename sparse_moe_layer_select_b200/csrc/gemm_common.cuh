@@ -25,6 +25,7 @@ struct Item {
   int nrows;   // valid rows (<= 128)
   int j;       // N tile index
   int nk;      // K blocks
+  int kb0;     // first K block (ROUTER K slices; 0 otherwise)
   bool skip;   // no work (N tile beyond this group's width)
 };
 
@@ -42,16 +43,20 @@ __device__ __forceinline__ Item decode_tile(const GemmParams &p, int item, int4 
   constexpr int BASE = MODE & 3;
   constexpr int KB = stage_k(MODE);
   Item it;
-  if (BASE == MODE_ROUTER) {  // item = (128-token tile, block of n_tile experts)
-    const int ti = item / p.n_ntiles;
+  if (BASE == MODE_ROUTER) {  // item = (128-token tile, block of n_tile experts, K slice)
+    const int per_tile = p.n_ntiles * p.ksplit;
+    const int ti = item / per_tile;
+    const int r = item - ti * per_tile;
     it.group = -1;
     it.row0 = ti * kBlockM;
     it.nrows = min(kBlockM, p.T - it.row0);
-    it.j = item - ti * p.n_ntiles;
-    it.nk = p.d / KB;
+    it.j = r / p.ksplit;
+    it.nk = p.d / KB / p.ksplit;
+    it.kb0 = (r - it.j * p.ksplit) * it.nk;
     it.skip = false;
     return it;
   }
+  it.kb0 = 0;
   const int ti = item / p.n_ntiles;
   it.j = item - ti * p.n_ntiles;
   it.group = t.x;
@@ -184,17 +189,22 @@ __device__ __forceinline__ void gather_a_stage(const GemmParams &p, const int (&
 // router_cc.cu); far above twice the fp32 logit error of either logit path.
 constexpr float kRefineBand = 2e-4f;
 
-// Router epilogue: each thread owns one token row and writes its E fp32
-// logits (bias added) as 16-byte vectors; selection happens in the
-// warp-per-token select kernel that follows.
+// Router epilogue: each thread owns one token row and writes its fp32
+// logits of the item's experts as 16-byte vectors, into the plane of the
+// item's K slice (the bias goes into slice 0's plane; zeros otherwise);
+// selection happens in the warp-per-token select kernel that follows.
 __device__ __forceinline__ void router_epilogue(const GemmParams &p, const Item &it,
                                                        uint32_t taddr, int row_local,
                                                        const float *bias_s) {
   if ((row_local >> 5) * 32 >= it.nrows) return;  // no valid row in this warp's quarter
   const bool valid = row_local < it.nrows;
   const int e0 = it.j * p.n_tile;  // this item's block of experts
-  float *dst = p.logits_out + static_cast<size_t>(it.row0 + row_local) * p.E + e0;
-  const float *b = bias_s + e0;
+  const int slice = it.kb0 / it.nk;
+  float *dst = p.logits_out + static_cast<size_t>(slice) * p.T * p.E +
+               static_cast<size_t>(it.row0 + row_local) * p.E + e0;
+  // bias_s holds 512 entries, zero past E; E and n_tile are at most 256, so its
+  // last n_tile entries are zeros for the slices after the first.
+  const float *b = bias_s + (slice == 0 ? e0 : 512 - p.n_tile);
   for (int c = 0; c < p.n_tile; c += 32) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(taddr + c, r);

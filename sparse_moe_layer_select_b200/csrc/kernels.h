@@ -41,6 +41,7 @@ struct GemmParams {
   const int *n_tiles_dev;   // GEMM1/GEMM2: number of tiles (device)
   int n_tiles_host;         // ROUTER: number of row tiles
   int n_ntiles;             // N tiles per row tile (max over groups)
+  int ksplit;               // ROUTER: K slices; slice s writes partial logits at s * T * E
   int T, d, E, k, F, Fs;
   int n_half;               // GEMM1: gate (and up) columns per N tile
   int n_tile;               // MMA N of this launch
@@ -51,7 +52,7 @@ struct GemmParams {
   const int *perm;          // GEMM1/GEMM2: expert-order rows -> t * k + j
   const float *topk_w;      // GEMM2
   const float *bias;        // ROUTER (may be null)
-  float *logits_out;        // ROUTER out: [T, E] fp32 logits incl. bias
+  float *logits_out;        // ROUTER out: [ksplit][T, E] fp32 partial logits, bias in slice 0
   uint16_t *h;              // GEMM1 out: [T*k, F] fp16 (expert-order rows)
   uint16_t *h_shared;       // GEMM1 out: [T, Fs] fp16
   uint16_t *o_out;          // GEMM2 out: [T*k, d] fp16, routed_scale * w * o (expert-order rows)
@@ -102,10 +103,14 @@ constexpr int kNotRouted = -1;
 // token_mask (optional, [T]): 0 = padding token, which gets kNotRouted ids
 // and zero weights.  bias: the logit bias (its float64 refinement adds it);
 // sel_bias: a selection-only bias on the sigmoid scores (one of the two).
-cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
-                                 const float *bias, const float *sel_bias,
-                                 const uint8_t *token_mask, int T, int d, int E, int k,
-                                 int norm_topk, int32_t *topk_idx, float *topk_w, cudaStream_t s);
+// nsplit > 1: logits holds nsplit partial [T, E] planes (K slices of the
+// router GEMM); each token's logits are their sum in plane order, written
+// back into plane 0 before the selection.
+cudaError_t launch_router_select(float *logits, int nsplit, const uint16_t *x,
+                                 const uint16_t *w_router, const float *bias,
+                                 const float *sel_bias, const uint8_t *token_mask, int T, int d,
+                                 int E, int k, int norm_topk, int32_t *topk_idx, float *topk_w,
+                                 cudaStream_t s);
 
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,

@@ -123,6 +123,22 @@ struct WsLayout {
   int max_tiles;
 };
 
+bool use_tensor_router(const Dims &D);
+
+// K slices of the tensor-core router GEMM: with few 128-token tiles, up to 4
+// slices of d (each slice's CTAs write partial logits, summed in slice order
+// by the select kernel), so that about one CTA per SM streams its share of x
+// once instead of a few CTAs streaming whole rows.  A function of the
+// dimensions only, since the workspace holds one logit plane per slice.
+constexpr int kRouterSplitSms = 148;
+int router_ksplit(const Dims &D) {
+  if (!use_tensor_router(D)) return 1;
+  const int tiles = (D.T + kBlockM - 1) / kBlockM;
+  int ks = 1;
+  while (ks < 4 && tiles * ks * 2 <= kRouterSplitSms && (D.d / kBlockK) % (ks * 2) == 0) ks *= 2;
+  return ks;
+}
+
 WsLayout ws_layout(const Dims &D) {
   WsLayout L;
   const size_t n = static_cast<size_t>(D.T) * D.k;
@@ -137,8 +153,8 @@ WsLayout ws_layout(const Dims &D) {
   off += align256(static_cast<size_t>(L.max_tiles) * sizeof(Tile));
   L.tiles_pair = off;  // 256-row tiles (CTA-pair GEMMs); fewer than the 128-row ones
   off += align256(static_cast<size_t>(L.max_tiles) * sizeof(Tile));
-  L.logits = off;
-  off += align256(static_cast<size_t>(D.T) * D.E * 4);
+  L.logits = off;  // plane 0: the logits; planes 1..: partial logits of the router's K slices
+  off += align256(static_cast<size_t>(router_ksplit(D)) * D.T * D.E * 4);
   L.inv = off;
   off += align256(n * 4);
   L.h = off;
@@ -236,10 +252,12 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     std::memset(&p, 0, sizeof(p));
     p.status = reinterpret_cast<int *>(wsp(ws, L.header));
     p.n_tiles_host = (D.T + kBlockM - 1) / kBlockM;
-    // Few token tiles (small T): split the experts into column blocks so that
-    // more SMs share the work; each block re-reads the token tile from L2.
+    p.ksplit = router_ksplit(D);
+    // Still few items (small T): split the experts into column blocks too, so
+    // that more SMs share the work; each block re-reads the token tile from L2.
     int nsplit = 1;
-    while (nsplit < 8 && p.n_tiles_host * nsplit * 2 <= sms && D.E % (nsplit * 2 * 32) == 0)
+    while (nsplit < 8 && p.n_tiles_host * p.ksplit * nsplit * 2 <= sms &&
+           D.E % (nsplit * 2 * 32) == 0)
       nsplit *= 2;
     p.n_ntiles = nsplit;
     p.T = D.T;
@@ -262,9 +280,9 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     m.a_sh = m.a;
     m.b0_sh = m.b0;
     m.b1_sh = m.b0;
-    const int grid = std::min(sms, p.n_tiles_host * p.n_ntiles);
+    const int grid = std::min(sms, p.n_tiles_host * p.n_ntiles * p.ksplit);
     if (launch_gemm(MODE_ROUTER, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_router_select(logits, static_cast<const uint16_t *>(x),
+    if (launch_router_select(logits, p.ksplit, static_cast<const uint16_t *>(x),
                              static_cast<const uint16_t *>(w_router), bias, sel_bias, token_mask,
                              D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -274,7 +292,7 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
   if (launch_router_cc(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(w_router),
                        bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (launch_router_select(logits, static_cast<const uint16_t *>(x),
+  if (launch_router_select(logits, 1, static_cast<const uint16_t *>(x),
                            static_cast<const uint16_t *>(w_router), bias, sel_bias, token_mask,
                            D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
     return MOE_ERR_CUDA;

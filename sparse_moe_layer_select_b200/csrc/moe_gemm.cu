@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_items = ((BASE == MODE_ROUTER) ? p.n_tiles_host : *p.n_tiles_dev) * p.n_ntiles;
+  const int n_items = (BASE == MODE_ROUTER) ? p.n_tiles_host * p.n_ntiles * p.ksplit
+                                            : *p.n_tiles_dev * p.n_ntiles;
   // The down projection multiplies fp16 h by fp16 W_down, the others bf16 operands; F8
   // launches e4m3 (whose format code equals fp16's).
   const uint32_t idesc = (BASE == MODE_GEMM2 || F8) ? idesc_f16_f32(kBlockM, p.n_tile)
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
           if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_ISSUE, issued);
           uint8_t *a_dst = sA + s * kABytes;
           uint8_t *b_dst = sB + s * kBBytesMax;
-          const int kc = kb * stage_k(MODE);
+          const int kc = (it.kb0 + kb) * stage_k(MODE);
           if (tma_warp && lane == 0) {
             if (BASE == MODE_GEMM1) {
               const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;

@@ -170,20 +170,50 @@ struct RefineScratch {
 
 template <int NPL>
 __device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
-                                             const float *__restrict__ logits,
+                                             float *__restrict__ logits, int nsplit, int T,
                                              const uint16_t *__restrict__ x,
                                              const uint16_t *__restrict__ w_router,
                                              const float *__restrict__ bias,
                                              const float *__restrict__ sel_bias, int d, int E,
                                              int k, int norm_topk, int32_t *__restrict__ topk_idx,
                                              float *__restrict__ topk_w) {
-  const float *row = logits + static_cast<size_t>(t) * E;
-  // The selection value of expert e: its logit, or with a selection-only bias
-  // sigmoid(logit) + b_e (the weights below always use the logit).
-  auto sel_value = [&](int e) -> float {
-    const float l = row[e];
+  float *row = logits + static_cast<size_t>(t) * E;
+  // This lane's logits (experts lane + 32 i): all loads first, one memory
+  // round trip.  With K slices (nsplit <= 4) the partial planes are summed in
+  // slice order and the sum is written back into plane 0, where the rest of
+  // the selection (and any later reader) finds the logits.
+  float lv[NPL];
+  {
+    const size_t plane = static_cast<size_t>(T) * E;
+    float part[4][NPL];
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        part[sl][i] = (sl < nsplit && e < E) ? row[sl * plane + e] : 0.f;
+      }
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      float l = part[0][i];
+#pragma unroll
+      for (int sl = 1; sl < 4; ++sl)
+        if (sl < nsplit) l += part[sl][i];
+      lv[i] = l;
+    }
+    if (nsplit > 1) {
+#pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (lane + 32 * i < E) row[lane + 32 * i] = lv[i];
+      __syncwarp();
+    }
+  }
+  // The selection value of expert e with logit l: l, or with a selection-only
+  // bias sigmoid(l) + b_e (the weights below always use the logit).
+  auto sel_of = [&](int e, float l) -> float {
     return sel_bias ? 1.f / (1.f + expf(-l)) + sel_bias[e] : l;
   };
+  auto sel_value = [&](int e) -> float { return sel_of(e, row[e]); };
   // Keys: an order-preserving map of the fp32 logit to uint32 (larger logit,
   // larger key; +0 and -0 equal; NaN and the padding slots past E lowest).
   uint32_t key[NPL];
@@ -191,7 +221,7 @@ __device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
     ev[i] = lane + 32 * i;
-    key[i] = ev[i] < E ? logit_key(sel_value(ev[i])) : 0u;
+    key[i] = ev[i] < E ? logit_key(sel_of(ev[i], lv[i])) : 0u;
   }
   // Sort each lane's list descending by key.  The list starts in ascending
   // expert id and the odd-even transposition network swaps only strictly
@@ -372,7 +402,7 @@ __device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
 
 template <int NPL>
 __global__ void __launch_bounds__(kSelectWarps * 32)
-    router_select_kernel(const float *__restrict__ logits, const uint16_t *__restrict__ x,
+    router_select_kernel(float *__restrict__ logits, int nsplit, const uint16_t *__restrict__ x,
                          const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
                          const float *__restrict__ sel_bias,
                          const uint8_t *__restrict__ token_mask, int T, int d, int E, int k,
@@ -390,8 +420,8 @@ __global__ void __launch_bounds__(kSelectWarps * 32)
     return;
   }
   __shared__ RefineScratch scratch[kSelectWarps];
-  select_token<NPL>(t, lane, &scratch[threadIdx.x >> 5], logits, x, w_router, bias, sel_bias, d,
-                    E, k, norm_topk, topk_idx, topk_w);
+  select_token<NPL>(t, lane, &scratch[threadIdx.x >> 5], logits, nsplit, T, x, w_router, bias,
+                    sel_bias, d, E, k, norm_topk, topk_idx, topk_w);
 }
 
 }  // namespace
@@ -414,15 +444,16 @@ cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const 
   return cudaGetLastError();
 }
 
-cudaError_t launch_router_select(const float *logits, const uint16_t *x, const uint16_t *w_router,
-                                 const float *bias, const float *sel_bias,
-                                 const uint8_t *token_mask, int T, int d, int E, int k,
-                                 int norm_topk, int32_t *topk_idx, float *topk_w, cudaStream_t s) {
+cudaError_t launch_router_select(float *logits, int nsplit, const uint16_t *x,
+                                 const uint16_t *w_router, const float *bias,
+                                 const float *sel_bias, const uint8_t *token_mask, int T, int d,
+                                 int E, int k, int norm_topk, int32_t *topk_idx, float *topk_w,
+                                 cudaStream_t s) {
   const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
   const int threads = kSelectWarps * 32;
   const int npl = (E + 31) / 32;
 #define MOE_SELECT(N)                                                                          \
-  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, x, w_router, bias, sel_bias,       \
+  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, nsplit, x, w_router, bias, sel_bias, \
                                                      token_mask, T, d, E, k, norm_topk, topk_idx, \
                                                      topk_w)
   if (npl <= 1) MOE_SELECT(1);

@@ -441,6 +441,35 @@ def test_router_logits_error_against_float64(flags):
     assert err < 1e-4 / 4, err
 
 
+@pytest.mark.parametrize("T", [1024, 4096, 6000, 10000])
+def test_router_k_slices_against_float64(T):
+    """The tensor-core router splits d into 4 slices (T <= 4736), 2 (T <= 9472) or none; the
+    select kernel sums the slices' partial logits.  The summed logits against the oracle's
+    float64 logits, and the routing against the oracle's, at each split (XS.2 widths)."""
+    import torch
+    w = I.get("c2_xs2_small").with_(T=T)
+    dev = {"x": torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda"),
+           "w_router": torch.empty((w.E, w.d_model), dtype=torch.bfloat16, device="cuda")}
+    I.generate_cuda(dev["x"], w.seed, I.TID_X, w.sigma_x)
+    I.generate_cuda(dev["w_router"], w.seed, I.TID_W_ROUTER, w.sigma_router)
+    dims = M.dims_for(w, flags=M.MOE_FLAG_ROUTER_TENSOR)
+    ws = M.alloc_workspace(dims)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((w.T, w.k), dtype=torch.float32, device="cuda")
+    M.route(dims, dev["x"], dev["w_router"], None, idx, wt, ws)
+    torch.cuda.synchronize()
+    code, site = M.read_device_status(ws)
+    assert code == 0, (M.status_string(code), site)
+    off = M.logits_offset(dims)
+    got = ws[off:off + w.T * w.E * 4].view(torch.float32).view(w.T, w.E).cpu().numpy()
+    xh, wh = P.to_numpy_bf16(dev["x"]), P.to_numpy_bf16(dev["w_router"])
+    ref_l = O.router_logits(xh, wh, None)
+    assert float(np.abs(got - ref_l).max()) < 1e-4 / 4
+    ref = O.route(xh, wh, None, w.k)
+    G.check_routing(idx.cpu().numpy(), wt.cpu().numpy(),
+                    {"topk_idx": ref[0], "topk_w": ref[1], "scores": ref[2]}, w.k)
+
+
 def test_prepared_down_weights_match_per_call_conversion():
     import torch
     w = I.get("c1_tiny").with_(T=500)
