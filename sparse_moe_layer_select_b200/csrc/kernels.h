@@ -106,11 +106,22 @@ constexpr int kNotRouted = -1;
 // nsplit > 1: logits holds nsplit partial [T, E] planes (K slices of the
 // router GEMM); each token's logits are their sum in plane order, written
 // back into plane 0 before the selection.
+// ix (optional): the index builder's outputs; when the batch's T * k entries
+// form one index chunk and E <= 256, the selection kernel also builds the
+// index (expert order and tile lists) and *indexed is set.
+struct SelectIndexOut {
+  int with_shared;
+  int *chunk_hist;
+  int32_t *counts, *offsets, *perm, *inv;
+  Tile *tiles, *tiles_pair;
+  int *header;
+};
 cudaError_t launch_router_select(float *logits, int nsplit, const uint16_t *x,
                                  const uint16_t *w_router, const float *bias,
                                  const float *sel_bias, const uint8_t *token_mask, int T, int d,
                                  int E, int k, int norm_topk, int32_t *topk_idx, float *topk_w,
-                                 cudaStream_t s);
+                                 cudaStream_t s, const SelectIndexOut *ix = nullptr,
+                                 bool *indexed = nullptr);
 
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,

@@ -241,7 +241,9 @@ bool use_tensor_router(const Dims &D) {
 // then the warp-per-token selection kernel.
 moe_status route_impl(const Dims &D, const void *x, const void *w_router, const float *bias,
                       const uint8_t *token_mask, int32_t *topk_idx, float *topk_w, void *ws,
-                      cudaStream_t s, int sms, int *launches) {
+                      cudaStream_t s, int sms, int *launches,
+                      const SelectIndexOut *ix = nullptr, bool *indexed = nullptr) {
+  if (indexed) *indexed = false;
   const WsLayout L = ws_layout(D);
   float *logits = reinterpret_cast<float *>(wsp(ws, L.logits));
   // A selection-only bias stays out of the logits and goes to the select kernel.
@@ -284,7 +286,8 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     if (launch_gemm(MODE_ROUTER, p, m, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (launch_router_select(logits, p.ksplit, static_cast<const uint16_t *>(x),
                              static_cast<const uint16_t *>(w_router), bias, sel_bias, token_mask,
-                             D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
+                             D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s, ix,
+                             indexed) != cudaSuccess)
       return MOE_ERR_CUDA;
     *launches += 2;
     return MOE_OK;
@@ -294,7 +297,8 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     return MOE_ERR_CUDA;
   if (launch_router_select(logits, 1, static_cast<const uint16_t *>(x),
                            static_cast<const uint16_t *>(w_router), bias, sel_bias, token_mask,
-                           D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s) != cudaSuccess)
+                           D.T, D.d, D.E, D.k, D.norm, topk_idx, topk_w, s, ix,
+                           indexed) != cudaSuccess)
     return MOE_ERR_CUDA;
   *launches += 2;
   return MOE_OK;
@@ -513,17 +517,12 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
   int launches = 0;
   EventMarker ev(s);
 
-  // 1. router
-  ev.mark();
-  st = route_impl(D, x, w->w_router, w->router_bias, token_mask, routing->topk_idx,
-                  routing->topk_w, ws, s, sms, &launches);
-  if (st != MOE_OK) return st;
-  // 2. expert order + tile lists.  Engines, as measured on B200: the gate/up
-  // GEMM runs on single CTAs (128-row tiles; with its A rows gathered by
-  // cp.async, the CTA-pair engine lost 12-14% to it at the large prefill
-  // shapes); the down GEMM runs on CTA pairs (256-row tiles, half of B per
-  // SM) when the average expert fills a 256-row tile, below that single CTAs
-  // waste less of the tensor core.  The flags force one engine for both.
+  // Engines, as measured on B200: the gate/up GEMM runs on single CTAs
+  // (128-row tiles; with its A rows gathered by cp.async, the CTA-pair engine
+  // lost 12-14% to it at the large prefill shapes); the down GEMM runs on CTA
+  // pairs (256-row tiles, half of B per SM) when the average expert fills a
+  // 256-row tile, below that single CTAs waste less of the tensor core.  The
+  // flags force one engine for both.
   const int pair_grid = 2 * std::min(pair_clusters(), sms / 2);  // all pairs co-resident
   bool pair1 = false;
   bool pair2 = static_cast<int64_t>(D.T) * D.k >= static_cast<int64_t>(2 * kBlockM) * D.E;
@@ -531,11 +530,29 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
   if (D.flags & MOE_FLAG_GEMM_SINGLE_CTA) pair1 = pair2 = false;
   if (pair_grid < 2 || fp8) pair1 = pair2 = false;
   Tile *tiles_pair = reinterpret_cast<Tile *>(wsp(ws, L.tiles_pair));
+  SelectIndexOut ix;
+  ix.with_shared = D.Fs > 0;
+  ix.chunk_hist = reinterpret_cast<int *>(wsp(ws, L.chunk_hist));
+  ix.counts = routing->counts;
+  ix.offsets = routing->offsets;
+  ix.perm = routing->perm;
+  ix.inv = inv;
+  ix.tiles = tiles;
+  ix.tiles_pair = (pair1 || pair2) ? tiles_pair : nullptr;
+  ix.header = header;
+
+  // 1. router (for a decode-sized batch its selection kernel also builds the index)
   ev.mark();
-  if (launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0,
-                   reinterpret_cast<int *>(wsp(ws, L.chunk_hist)), tiles, header, routing->counts,
-                   routing->offsets, routing->perm, s, &launches,
-                   (pair1 || pair2) ? tiles_pair : nullptr, inv) != cudaSuccess)
+  bool indexed = false;
+  st = route_impl(D, x, w->w_router, w->router_bias, token_mask, routing->topk_idx,
+                  routing->topk_w, ws, s, sms, &launches, &ix, &indexed);
+  if (st != MOE_OK) return st;
+  // 2. expert order + tile lists
+  ev.mark();
+  if (!indexed &&
+      launch_index(routing->topk_idx, D.T, D.k, D.E, D.Fs > 0, ix.chunk_hist, tiles, header,
+                   routing->counts, routing->offsets, routing->perm, s, &launches, ix.tiles_pair,
+                   inv) != cudaSuccess)
     return MOE_ERR_CUDA;
 
   // FP8 experts: e4m3 rows of x with their scales

@@ -24,7 +24,9 @@
 #include <cfloat>
 
 #include "gemm_common.cuh"
+#include "index_common.cuh"
 #include "kernels.h"
+#include "status.cuh"
 
 namespace moe {
 
@@ -52,11 +54,23 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   const int t0 = blockIdx.x * kTokPerCta;
   const int nt = min(kTokPerCta, T - t0);
   const int vec_per_row = d / 8;
-  for (int i = threadIdx.x; i < kTokPerCta * vec_per_row; i += blockDim.x) {
-    const int r = i / vec_per_row;
-    const int c = i - r * vec_per_row;
-    xs4[i] = r < nt ? reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t0 + r) * d)[c]
-                    : make_uint4(0, 0, 0, 0);
+  const int n_vec = kTokPerCta * vec_per_row;
+  // Stage the tokens: each thread's loads are issued together (kStageLoads at
+  // a time), then stored, so the staging costs about one memory round trip.
+  constexpr int kStageLoads = 8;
+  for (int i0 = threadIdx.x; i0 < n_vec; i0 += kStageLoads * blockDim.x) {
+    uint4 v[kStageLoads];
+#pragma unroll
+    for (int u = 0; u < kStageLoads; ++u) {
+      const int i = i0 + u * blockDim.x;
+      const int r = i / vec_per_row;
+      v[u] = (i < n_vec && r < nt)
+                 ? reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t0 + r) * d)[i - r * vec_per_row]
+                 : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kStageLoads; ++u)
+      if (i0 + u * blockDim.x < n_vec) xs4[i0 + u * blockDim.x] = v[u];
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5;
@@ -66,15 +80,28 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     float acc[kTokPerCta];
 #pragma unroll
     for (int r = 0; r < kTokPerCta; ++r) acc[r] = 0.f;
-    for (int c = lane; c < vec_per_row; c += 32) {
-      float wf[8];
-      bf16x8_to_f32(wr[c], wf);
+    // this lane's weight vectors of the expert row, kWLoads loads in flight at a time
+    constexpr int kWLoads = 8;
+    for (int c0 = lane; c0 < vec_per_row; c0 += 32 * kWLoads) {
+      uint4 wv[kWLoads];
 #pragma unroll
-      for (int r = 0; r < kTokPerCta; ++r) {
-        float xf[8];
-        bf16x8_to_f32(xs4[r * vec_per_row + c], xf);
+      for (int u = 0; u < kWLoads; ++u) {
+        const int c = c0 + 32 * u;
+        wv[u] = c < vec_per_row ? wr[c] : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[r] = fmaf(xf[i], wf[i], acc[r]);
+      for (int u = 0; u < kWLoads; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= vec_per_row) break;
+        float wf[8];
+        bf16x8_to_f32(wv[u], wf);
+#pragma unroll
+        for (int r = 0; r < kTokPerCta; ++r) {
+          float xf[8];
+          bf16x8_to_f32(xs4[r * vec_per_row + c], xf);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[r] = fmaf(xf[i], wf[i], acc[r]);
+        }
       }
     }
 #pragma unroll
@@ -400,6 +427,25 @@ __device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
   }
 }
 
+// Routes one token per warp (padding tokens get kNotRouted ids and zero weights).
+template <int NPL>
+__device__ __forceinline__ void select_or_pad(int t, int lane, RefineScratch *rs, float *logits,
+                                              int nsplit, int T, const uint16_t *x,
+                                              const uint16_t *w_router, const float *bias,
+                                              const float *sel_bias, const uint8_t *token_mask,
+                                              int d, int E, int k, int norm_topk,
+                                              int32_t *topk_idx, float *topk_w) {
+  if (token_mask != nullptr && token_mask[t] == 0) {
+    if (lane < k) {
+      topk_idx[static_cast<size_t>(t) * k + lane] = kNotRouted;
+      topk_w[static_cast<size_t>(t) * k + lane] = 0.f;
+    }
+    return;
+  }
+  select_token<NPL>(t, lane, rs, logits, nsplit, T, x, w_router, bias, sel_bias, d, E, k,
+                    norm_topk, topk_idx, topk_w);
+}
+
 template <int NPL>
 __global__ void __launch_bounds__(kSelectWarps * 32)
     router_select_kernel(float *__restrict__ logits, int nsplit, const uint16_t *__restrict__ x,
@@ -408,20 +454,49 @@ __global__ void __launch_bounds__(kSelectWarps * 32)
                          const uint8_t *__restrict__ token_mask, int T, int d, int E, int k,
                          int norm_topk,
                          int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+  __shared__ RefineScratch scratch[kSelectWarps];
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
   if (t >= T) return;
-  if (token_mask != nullptr && token_mask[t] == 0) {
-    // padding token: not routed (no experts, zero weights)
-    if (lane < k) {
-      topk_idx[static_cast<size_t>(t) * k + lane] = kNotRouted;
-      topk_w[static_cast<size_t>(t) * k + lane] = 0.f;
-    }
-    return;
-  }
+  select_or_pad<NPL>(t, lane, &scratch[threadIdx.x >> 5], logits, nsplit, T, x, w_router, bias,
+                     sel_bias, token_mask, d, E, k, norm_topk, topk_idx, topk_w);
+}
+
+// The same selection, then, for a batch whose T * k entries form a single
+// index chunk (decode-sized), the index builder in the CTA that finishes
+// last (a ticket in the workspace header; the other CTAs simply exit): the
+// expert order and tile lists come out of this launch, with no index launch
+// and no second read of the routing from a cold kernel.  Needs E <= 256 (one
+// scan thread per expert).
+template <int NPL>
+__global__ void __launch_bounds__(kSelectWarps * 32)
+    router_select_index_kernel(float *__restrict__ logits, int nsplit,
+                               const uint16_t *__restrict__ x,
+                               const uint16_t *__restrict__ w_router,
+                               const float *__restrict__ bias, const float *__restrict__ sel_bias,
+                               const uint8_t *__restrict__ token_mask, int T, int d, int E, int k,
+                               int norm_topk, int32_t *__restrict__ topk_idx,
+                               float *__restrict__ topk_w, SelectIndexOut ix) {
   __shared__ RefineScratch scratch[kSelectWarps];
-  select_token<NPL>(t, lane, &scratch[threadIdx.x >> 5], logits, nsplit, T, x, w_router, bias,
-                    sel_bias, d, E, k, norm_topk, topk_idx, topk_w);
+  __shared__ int h[idx::kIdxWarps * idx::kMaxE];
+  __shared__ int warp_sums[32];
+  __shared__ int totals[3];
+  __shared__ int ticket;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
+  if (t < T)
+    select_or_pad<NPL>(t, lane, &scratch[threadIdx.x >> 5], logits, nsplit, T, x, w_router, bias,
+                       sel_bias, token_mask, d, E, k, norm_topk, topk_idx, topk_w);
+  __threadfence();  // this CTA's routing is visible before its ticket is taken
+  __syncthreads();
+  if (threadIdx.x == 0)
+    ticket = atomicAdd(&reinterpret_cast<WsHeader *>(ix.header)->index_done, 1);
+  __syncthreads();
+  if (ticket != static_cast<int>(gridDim.x) - 1) return;
+  __threadfence();
+  idx::index_single_cta(topk_idx, T * k, E, T, ix.with_shared, ix.chunk_hist, ix.counts,
+                        ix.offsets, ix.perm, ix.inv, ix.tiles, ix.tiles_pair, ix.header, h,
+                        warp_sums, totals);
 }
 
 }  // namespace
@@ -448,14 +523,24 @@ cudaError_t launch_router_select(float *logits, int nsplit, const uint16_t *x,
                                  const uint16_t *w_router, const float *bias,
                                  const float *sel_bias, const uint8_t *token_mask, int T, int d,
                                  int E, int k, int norm_topk, int32_t *topk_idx, float *topk_w,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, const SelectIndexOut *ix, bool *indexed) {
   const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
   const int threads = kSelectWarps * 32;
   const int npl = (E + 31) / 32;
-#define MOE_SELECT(N)                                                                          \
-  router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, nsplit, x, w_router, bias, sel_bias, \
-                                                     token_mask, T, d, E, k, norm_topk, topk_idx, \
-                                                     topk_w)
+  const bool fuse = ix != nullptr && static_cast<int64_t>(T) * k <= kIndexChunk &&
+                    E <= threads && E <= idx::kMaxE;
+  if (indexed) *indexed = fuse;
+#define MOE_SELECT(N)                                                                           \
+  do {                                                                                          \
+    if (fuse)                                                                                   \
+      router_select_index_kernel<N><<<blocks, threads, 0, s>>>(                                 \
+          logits, nsplit, x, w_router, bias, sel_bias, token_mask, T, d, E, k, norm_topk,       \
+          topk_idx, topk_w, *ix);                                                               \
+    else                                                                                        \
+      router_select_kernel<N><<<blocks, threads, 0, s>>>(logits, nsplit, x, w_router, bias,     \
+                                                         sel_bias, token_mask, T, d, E, k,      \
+                                                         norm_topk, topk_idx, topk_w);          \
+  } while (0)
   if (npl <= 1) MOE_SELECT(1);
   else if (npl <= 2) MOE_SELECT(2);
   else if (npl <= 4) MOE_SELECT(4);

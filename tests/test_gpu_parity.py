@@ -587,6 +587,38 @@ def test_full_size_workloads(name, n_sample):
     G.check_output(G.y_numpy(y)[rows], ref["y"], rows_ok=same, what=name)
 
 
+@pytest.mark.parametrize("T,Fs", [(64, 512), (512, 512), (512, 0), (513, 512)])
+def test_select_kernel_builds_the_decode_index(T, Fs):
+    """T * k <= 4096 (one index chunk) and E <= 256: the router's selection kernel also builds
+    the expert order and tile lists (its last CTA); T=513 takes the separate index kernels.
+    counts / offsets / perm against the oracle's expert order of the GPU selection, the launch
+    count, and y on a sample of tokens against the oracle (XS.2 widths, with and without the
+    shared expert)."""
+    w = I.get("c2_xs2_small").with_(T=T, shared_intermediate_size=Fs)
+    h, dev = _device_workload(w)
+    y, routing, _ = G.run_forward(w, dev)
+    launches = M.last_launch_count()
+    gidx = routing["topk_idx"].cpu().numpy()
+    c, o, p = O.expert_order(gidx, w.E)
+    assert np.array_equal(routing["counts"].cpu().numpy(), c)
+    assert np.array_equal(routing["offsets"].cpu().numpy(), o)
+    assert np.array_equal(routing["perm"].cpu().numpy(), p)
+    ridx, rw, scores, _ = O.route(h["x"], h["w_router"], None, w.k)
+    G.check_routing(gidx, routing["topk_w"].cpu().numpy(),
+                    {"topk_idx": ridx, "topk_w": rw, "scores": scores}, w.k)
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(w.T, size=min(w.T, 48), replace=False))
+    ref = G.oracle_forward(w, h, rows=rows)
+    same = P.same_selection_mask(gidx[rows], ref["topk_idx"])
+    G.check_output(G.y_numpy(y)[rows], ref["y"], rows_ok=same, what=f"T={T} Fs={Fs}")
+    # router logits, selection (+ index when fused), [two index kernels], W_down and (with
+    # a shared expert) its W_down converted to fp16 (bf16 weights passed), gate/up, down,
+    # combine
+    fused = T * w.k <= 4096
+    expected = 2 + (0 if fused else 2) + (2 if Fs else 1) + 3
+    assert launches == expected, (launches, expected)
+
+
 def test_decode_fresh_batches():
     import torch
     w = I.get("c5_decode")
