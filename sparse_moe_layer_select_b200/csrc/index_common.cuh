@@ -48,22 +48,24 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int *
 
 // Per-warp expert histograms of one chunk into h[kIdxWarps][E] (shared).
 __device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk_idx, int n,
-                                                int E, int chunk, int *h, int *status) {
+                                                int E, int chunk, int *h, int *status,
+                                                int sub = kSub) {
   for (int i = threadIdx.x; i < kIdxWarps * E; i += blockDim.x) h[i] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int base = chunk * kIndexChunk + warp * kSub;
+  const int base = chunk * kIndexChunk + warp * sub;
   if (warp < kIdxWarps) {  // (a larger CTA's other warps only clear and wait)
     int *hw = h + warp * E;
     int ids[kSub / 32];  // all loads first: one memory round trip per warp
 #pragma unroll
     for (int q = 0; q < kSub / 32; ++q) {
       const int i = base + q * 32 + lane;
-      ids[q] = i < n ? __ldcg(&topk_idx[i]) : kNotRouted;
+      ids[q] = (q * 32 < sub && i < n) ? __ldcg(&topk_idx[i]) : kNotRouted;
     }
 #pragma unroll
     for (int q = 0; q < kSub / 32; ++q) {
+      if (q * 32 >= sub) break;
       const int e = ids[q];
       if (e == kNotRouted) continue;
       if (e < 0 || e >= E) {
@@ -76,27 +78,29 @@ __device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk
   __syncthreads();
 }
 
-// Each warp places its 512 entries: fill[warp][e] holds its next row of e.
+// Each warp places its `sub` consecutive entries (512 in a multi-chunk
+// batch; fewer, spread over all eight warps, in a single small chunk):
+// fill[warp][e] holds its next row of e.
 __device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ topk_idx, int n,
                                                    int E, int chunk, int *fill,
                                                    int32_t *__restrict__ perm,
-                                                   int32_t *__restrict__ inv) {
+                                                   int32_t *__restrict__ inv, int sub = kSub) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   int *fw = fill + warp * E;
-  const int base = chunk * kIndexChunk + warp * kSub;
+  const int base = chunk * kIndexChunk + warp * sub;
   int ids[kSub / 32];  // all loads first: one memory round trip per warp
 #pragma unroll
   for (int q = 0; q < kSub / 32; ++q) {
     const int i = base + q * 32 + lane;
-    ids[q] = i < n ? __ldcg(&topk_idx[i]) : -1;
+    ids[q] = (q * 32 < sub && i < n) ? __ldcg(&topk_idx[i]) : -1;
   }
 #pragma unroll
   for (int q = 0; q < kSub / 32; ++q) {
     const int r = q * 32;
     const int i = base + r + lane;
-    if (base + r >= n) break;  // warp-uniform
+    if (r >= sub || base + r >= n) break;  // warp-uniform
     int e = ids[q];
     if (e < 0 || e >= E) e = -1;
     const unsigned m = __match_any_sync(0xffffffffu, e);
@@ -228,7 +232,9 @@ __device__ __forceinline__ void index_single_cta(const int32_t *__restrict__ top
                                                  Tile *__restrict__ tiles_pair, int *header, int *h,
                                                  int *warp_sums, int *totals) {
   const int warp = threadIdx.x >> 5;
-  chunk_warp_hist(topk_idx, n, E, 0, h, header);  // warps 0..7
+  // entries per warp: the chunk spread over all eight warps, in whole warps of entries
+  const int sub = max(32, (n + kIdxWarps * 32 - 1) / (kIdxWarps * 32) * 32);
+  chunk_warp_hist(topk_idx, n, E, 0, h, header, sub);  // warps 0..7
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int s = 0;
 #pragma unroll
@@ -240,7 +246,7 @@ __device__ __forceinline__ void index_single_cta(const int32_t *__restrict__ top
                  warp_sums, totals);
   __syncthreads();
   warp_bases(E, chunk_hist, h);
-  if (warp < kIdxWarps) chunk_warp_scatter(topk_idx, n, E, 0, h, perm, inv);
+  if (warp < kIdxWarps) chunk_warp_scatter(topk_idx, n, E, 0, h, perm, inv, sub);
 }
 
 }  // namespace idx
