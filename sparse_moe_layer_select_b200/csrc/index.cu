@@ -14,8 +14,9 @@
 //              (128 for single-CTA GEMMs, 256 for CTA-pair GEMMs), in expert
 //              order, followed by the shared expert's token blocks.
 //
-// The (t, j) entries are cut into chunks of kIndexChunk = 4096, one CTA of 8
-// warps per chunk, each warp owning 512 consecutive entries:
+// The (t, j) entries are cut into chunks of index_chunk_entries(n) (1024 to
+// 4096, kernels.h), one CTA of 8 warps per chunk, each warp owning an eighth
+// of the chunk's consecutive entries:
 //   index_hist_scan_kernel  per-chunk expert histogram; the CTA that
 //                         finishes last then sums per expert over chunks,
 //                         scans over experts, writes the chunk bases and the
@@ -46,12 +47,12 @@ __global__ void __launch_bounds__(512)
                            int with_shared, int *__restrict__ chunk_hist,
                            int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                            Tile *__restrict__ tiles, Tile *__restrict__ tiles_pair,
-                           int *__restrict__ header) {
+                           int *__restrict__ header, int sub) {
   __shared__ int h[kIdxWarps * kMaxE];
   __shared__ int warp_sums[32];
   __shared__ int totals[3];
   __shared__ int ticket;
-  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, header);
+  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, header, sub);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int s = 0;
 #pragma unroll
@@ -72,11 +73,11 @@ __global__ void __launch_bounds__(512)
 __global__ void __launch_bounds__(kIdxWarps * 32)
     index_scatter_kernel(const int32_t *__restrict__ topk_idx, int n, int E,
                          const int *__restrict__ chunk_base, int32_t *__restrict__ perm,
-                         int32_t *__restrict__ inv) {
+                         int32_t *__restrict__ inv, int sub) {
   __shared__ int h[kIdxWarps * kMaxE];
-  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, nullptr);
+  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, nullptr, sub);
   warp_bases(E, chunk_base + static_cast<size_t>(blockIdx.x) * E, h);
-  chunk_warp_scatter(topk_idx, n, E, blockIdx.x, h, perm, inv);
+  chunk_warp_scatter(topk_idx, n, E, blockIdx.x, h, perm, inv, sub);
 }
 
 // All of the above for a single chunk (n <= kIndexChunk), in one CTA of 512
@@ -101,7 +102,8 @@ cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_
                          int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
                          Tile *tiles_pair, int32_t *inv) {
   const int n = T * k;
-  const int nchunks = (n + kIndexChunk - 1) / kIndexChunk;
+  const int chunk = index_chunk_entries(n);
+  const int nchunks = (n + chunk - 1) / chunk;
   if (nchunks == 1) {
     index_single_kernel<<<1, 512, 0, s>>>(topk_idx, n, E, T, with_shared, chunk_hist, counts,
                                           offsets, perm, inv, tiles, tiles_pair, status);
@@ -110,10 +112,11 @@ cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_
   }
   index_hist_scan_kernel<<<nchunks, 512, 0, s>>>(topk_idx, n, E, nchunks, T, with_shared,
                                                   chunk_hist, counts, offsets, tiles, tiles_pair,
-                                                  status);
+                                                  status, chunk / kIdxWarps);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  index_scatter_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm, inv);
+  index_scatter_kernel<<<nchunks, kIdxWarps * 32, 0, s>>>(topk_idx, n, E, chunk_hist, perm, inv,
+                                                          chunk / kIdxWarps);
   *launches += 2;
   return cudaGetLastError();
 }

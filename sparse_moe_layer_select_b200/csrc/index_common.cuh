@@ -54,7 +54,7 @@ __device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int base = chunk * kIndexChunk + warp * sub;
+  const int base = (chunk * kIdxWarps + warp) * sub;  // chunks of kIdxWarps * sub entries
   if (warp < kIdxWarps) {  // (a larger CTA's other warps only clear and wait)
     int *hw = h + warp * E;
     int ids[kSub / 32];  // all loads first: one memory round trip per warp
@@ -89,7 +89,7 @@ __device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ t
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   int *fw = fill + warp * E;
-  const int base = chunk * kIndexChunk + warp * sub;
+  const int base = (chunk * kIdxWarps + warp) * sub;  // chunks of kIdxWarps * sub entries
   int ids[kSub / 32];  // all loads first: one memory round trip per warp
 #pragma unroll
   for (int q = 0; q < kSub / 32; ++q) {

@@ -21,7 +21,17 @@ struct Tile {
 constexpr int kBlockM = 128;        // rows per tile (tcgen05 M)
 constexpr int kBlockK = 64;         // K elements per pipeline stage (one 128-byte swizzle row)
 constexpr int kStages = 4;          // shared-memory pipeline depth
-constexpr int kIndexChunk = 4096;   // (token, slot) entries per index-builder chunk
+constexpr int kIndexChunk = 4096;   // (token, slot) entries per index-builder chunk (at most)
+
+// Entries per index-builder chunk for a batch of n (token, slot) entries: one
+// chunk up to kIndexChunk; above that a power of two from 1024 to kIndexChunk,
+// so that mid-sized batches still spread over 32-48 CTAs (one per chunk).
+__host__ __device__ inline int index_chunk_entries(int64_t n) {
+  if (n <= kIndexChunk) return kIndexChunk;
+  int c = 1024;
+  while (c < kIndexChunk && static_cast<int64_t>(c) * 48 < n) c *= 2;
+  return c;
+}
 
 enum GemmMode : int {
   MODE_ROUTER = 0,

@@ -142,7 +142,7 @@ int router_ksplit(const Dims &D) {
 WsLayout ws_layout(const Dims &D) {
   WsLayout L;
   const size_t n = static_cast<size_t>(D.T) * D.k;
-  const size_t nchunks = (n + kIndexChunk - 1) / kIndexChunk;
+  const size_t nchunks = (n + index_chunk_entries(n) - 1) / index_chunk_entries(n);
   L.max_tiles = static_cast<int>((n + kBlockM - 1) / kBlockM + D.E + (D.T + kBlockM - 1) / kBlockM);
   size_t off = 0;
   L.header = off;

@@ -67,7 +67,7 @@ extern "C" moe_status moe_permute_static(const moe_dims_t *dims, const int32_t *
     if (reinterpret_cast<uintptr_t>(p) & 15) return MOE_ERR_INVALID_ARG;
   if (static_cast<int64_t>(T) * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
   const size_t n = static_cast<size_t>(T) * k;
-  const size_t nchunks = std::max<size_t>((n + kIndexChunk - 1) / kIndexChunk, 1);
+  const size_t nchunks = std::max<size_t>((n + index_chunk_entries(n) - 1) / index_chunk_entries(n), 1);
   const size_t max_tiles = (n + kBlockM - 1) / kBlockM + E;
   const size_t off_hist = a256(sizeof(WsHeader));
   const size_t off_tiles = off_hist + a256(nchunks * E * sizeof(int));
