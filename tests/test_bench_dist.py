@@ -93,3 +93,25 @@ def test_stored_traffic_matches_the_sources():
         assert bench.measured_traffic("c3_xs2_prefill_zipf", "gemm1_swiglu") is None
     else:
         assert bench.measured_traffic("c3_xs2_prefill_zipf", "gemm1_swiglu") is not None
+
+
+def test_stage_work_of_the_t4096_workload():
+    """Algorithmic work behind the roofline numbers, against sums done by hand for the
+    T=4096 XS.2 workload (d=2048, E=256, k=8, F=Fs=512) with every expert touched."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from sparse_moe_layer_select_b200 import inputs as I
+    w = I.get("c2_xs2_small")
+    work = bench.stage_work(w, np.ones(256, dtype=np.int64))
+    # W_gate + W_up of 256 experts (2 x 512 x 2048 bf16 each) = 1073741824, shared gate + up
+    # 4194304, x 16777216, h (32768 routed + 4096 shared rows of 512 fp16) 37748736
+    assert work["gemm1_swiglu"]["bytes"] == 1132462080
+    # 4 d F per routed row (gate and up, 2 flops per MAC) + the same per shared row
+    assert work["gemm1_swiglu"]["flops"] == 4 * 2048 * 512 * (32768 + 4096)
+    # W_down 536870912 + shared 2097152 + h 37748736 + O and S (9 rows of 2048 fp16 per token)
+    assert work["gemm2_down_scale"]["bytes"] == 536870912 + 2097152 + 37748736 + 4096 * 9 * 4096
+    # half the expert weight bytes with e4m3, plus a float32 scale per weight row
+    f8 = bench.stage_work(w, np.ones(256, dtype=np.int64), fp8=True)
+    assert f8["gemm1_swiglu"]["bytes"] == (1073741824 + 4194304) // 2 + 16777216 + 37748736 + \
+        4 * (256 * (2 * 512 + 2048) + 2 * 512 + 2048)
