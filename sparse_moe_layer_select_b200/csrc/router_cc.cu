@@ -18,7 +18,13 @@
 //                         order; tokens whose
 //                         k-th and (k+1)-th logits are within kRefineBand get
 //                         the experts near that boundary re-decided on float64
-//                         logits; sigmoid and normalisation in fp32.
+//                         logits; sigmoid and normalisation in fp32.  When
+//                         the tensor-core router split d into K slices, the
+//                         warp first sums the slices' partial logits (slice
+//                         order) and writes the sum back to the first plane.
+//   router_select_index_kernel  the same, then, for a batch whose T * k
+//                         entries form one index chunk, the index builder
+//                         (index_common.cuh) in whichever CTA finishes last.
 #include <cuda_bf16.h>
 
 #include <cfloat>
