@@ -64,6 +64,24 @@ def test_workspace_size_and_shape_limits(L):
     assert M.workspace_size(d) == 0
 
 
+def test_workspace_holds_one_logit_plane_per_router_slice(L):
+    """The tensor-core router (T >= 1024 at E = 256) cuts d into 4 K slices up to 37 token
+    tiles (T <= 4736), 2 up to 74 (T <= 9472), none above, and the workspace holds one fp32
+    [T, E] logit plane per slice: the size jumps by about three planes at T = 1024 (no slices
+    on the CUDA-core router below) and drops by about two planes just past T = 4736 and
+    about one just past T = 9472."""
+    def ws(T):
+        return M.workspace_size(M.make_dims(T, 2048, 256, 8, 512, 512))
+    plane = lambda T: T * 256 * 4
+    per_token = ws(2001) - ws(2000)          # growth of everything else, per token
+    assert 0 < per_token < 200_000
+    assert ws(1024) - ws(1023) > 3 * plane(1023) - 2 * per_token
+    assert ws(4736) - ws(4737) > 2 * plane(4736) - 2 * per_token
+    assert ws(9472) - ws(9473) > plane(9472) - 2 * per_token
+    # T = 2000 grows by four planes per token, T = 20000 by one (256-byte section alignment)
+    assert abs((ws(20001) - ws(20000)) - (per_token - 3 * 256 * 4)) < 2048
+
+
 def _call_forward(dims, x=256, y=512, ws=4096, ws_bytes=1 << 40, weights=None, routing=None):
     w = weights or M.moe_weights_t(1024, None, 2048, 4096, 8192, 16384, 32768, 65536)
     r = routing or M.moe_routing_t(1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20)
