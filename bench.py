@@ -70,16 +70,23 @@ def _code_tokens(text):
     return "\n".join(line for line in lines if line)
 
 
+# The sources the expert GEMM kernels are compiled from (the kernels whose ncu DRAM
+# traffic profiles/ncu_traffic.json records), including the shared header of all kernels.
+GEMM_SOURCES = ("gemm_common.cuh", "kernels.h", "moe_gemm.cu", "moe_gemm_pair.cu", "ptx.cuh",
+                "status.cuh")
+
+
 def kernel_sources_sha1():
-    """Hash of the CUDA sources' code (comments and blank space ignored): DRAM traffic
-    taken by ncu is valid only for these."""
+    """Hash of the expert GEMM kernels' sources (code only: comments and blank space
+    ignored, and the public header they include): DRAM traffic taken by ncu is valid only
+    for these."""
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "sparse_moe_layer_select_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), encoding="utf-8") as f:
-                h.update(name.encode() + b"\0" + _code_tokens(f.read()).encode())
+    paths = [os.path.join(csrc, n) for n in GEMM_SOURCES] + [os.path.join(ROOT, "include", "moe.h")]
+    for path in paths:
+        with open(path, encoding="utf-8") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + _code_tokens(f.read()).encode())
     return h.hexdigest()
 
 
