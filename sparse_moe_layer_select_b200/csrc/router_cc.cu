@@ -123,6 +123,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
 }
 
 constexpr int kSelectWarps = 8;
+// CTAs per SM the selection kernels are compiled for: four 8-warp CTAs (<= 64
+// registers a thread) keep a 4096-token batch within one wave on 148 SMs.
+constexpr int kSelectCtasPerSm = 4;
 
 // kRefineBand (gemm_common.cuh): width of the ambiguous band around the
 // k-th/(k+1)-th boundary, in logit units.  It is far above twice the largest
@@ -453,7 +456,7 @@ __device__ __forceinline__ void select_or_pad(int t, int lane, RefineScratch *rs
 }
 
 template <int NPL>
-__global__ void __launch_bounds__(kSelectWarps * 32)
+__global__ void __launch_bounds__(kSelectWarps * 32, kSelectCtasPerSm)
     router_select_kernel(float *__restrict__ logits, int nsplit, const uint16_t *__restrict__ x,
                          const uint16_t *__restrict__ w_router, const float *__restrict__ bias,
                          const float *__restrict__ sel_bias,
@@ -475,7 +478,7 @@ __global__ void __launch_bounds__(kSelectWarps * 32)
 // and no second read of the routing from a cold kernel.  Needs E <= 256 (one
 // scan thread per expert).
 template <int NPL>
-__global__ void __launch_bounds__(kSelectWarps * 32)
+__global__ void __launch_bounds__(kSelectWarps * 32, kSelectCtasPerSm)
     router_select_index_kernel(float *__restrict__ logits, int nsplit,
                                const uint16_t *__restrict__ x,
                                const uint16_t *__restrict__ w_router,
