@@ -26,7 +26,7 @@
  *   is the legacy default stream).  No call synchronises the host except
  *   moe_read_device_status, so the sequence can be captured in a CUDA graph.
  * - Every device pointer must be 16-byte aligned.  Shape limits: d_model a
- *   multiple of 128; F and Fs multiples of 64 (Fs = 0: no shared expert);
+ *   multiple of 64; F and Fs multiples of 64 (Fs = 0: no shared expert);
  *   1 <= k <= min(E, 16); E <= 512.  Anything else returns
  *   MOE_ERR_UNSUPPORTED_SHAPE before anything is launched.
  * - T = 0 is a no-op that returns MOE_OK.
@@ -98,6 +98,25 @@ typedef struct {
 /* Size the workspace for moe_forward_fp8 (required by it; F and Fs must be
  * multiples of 128). */
 #define MOE_FLAG_FP8_EXPERTS 64
+/* Combine by reduction: the down GEMM adds every scaled routed row
+ * (routed_scaling_factor * w * E_e(x)) and every shared-expert row straight
+ * into an fp32 accumulator row of its token (bulk reduce-adds performed at
+ * L2), and a last kernel rounds the accumulator to bf16 y.  No fp16
+ * contribution rows are written or read back, and the sums stay in fp32; the
+ * order of a token's k + 1 additions is not fixed, so repeated runs can differ
+ * in the last bits of the fp32 sum (and then, rarely, by one bf16 step of y).
+ * Without the flag the combine is a separate deterministic kernel over fp16
+ * contribution rows.  Not with moe_forward_fp8. */
+#define MOE_FLAG_COMBINE_REDUCE 128
+/* Fused expert kernel: one persistent tcgen05 kernel runs the gate/up GEMM,
+ * keeps the SwiGLU activation h in tensor memory (fp16, never written to
+ * device memory), runs the down GEMM with its A operand read from tensor
+ * memory, and adds routed_scaling_factor * w * o (shared expert: o) into
+ * fp32 token rows as MOE_FLAG_COMBINE_REDUCE does (so results are rounded as
+ * with that flag).  F and Fs multiples of 128, d_model a multiple of 128; an
+ * FFN wider than 512 runs in parts of at most 512 columns whose partial down
+ * projections add up in the same rows.  Not with moe_forward_fp8. */
+#define MOE_FLAG_FUSED_EXPERTS 256
 
 typedef struct {
     const void *w_router;      /* [E, d] bf16 */
@@ -270,14 +289,18 @@ moe_status moe_profile_next_forward(void **events, int32_t n_events);
 #define MOE_STATIC_SCRATCH_BYTES (512u * 1024u)
 
 /* moe_permute without a workspace, for callers that cannot allocate device
- * memory (code that runs inside another runtime's memory pool, plugins whose
- * host process owns all device memory, or work being captured into a CUDA
- * graph where an allocation would break the capture).  The paper has no
- * counterpart to this entry point; it is a deployment convenience.
+ * memory (code that runs inside another runtime's memory pool, or plugins
+ * whose host process owns all device memory).  The paper has no counterpart
+ * to this entry point; it is a deployment convenience.
  * Same outputs as moe_permute without x / x_perm: counts [E], offsets [E + 1],
  * perm [T * k].  Its scratch is one static device array of
- * MOE_STATIC_SCRATCH_BYTES per GPU, held from library load to process exit;
- * enough for T * k up to 262144 at E = 256.  Dims that need more return
+ * MOE_STATIC_SCRATCH_BYTES per GPU, held from library load to process exit.
+ * With n = T * k, chunk = 4096 for n <= 4096, else the smallest of 1024,
+ * 2048, 4096 with 48 * chunk >= n (4096 at most), and r(b) = b rounded up to
+ * a multiple of 256, the call needs
+ *   256 + r(4 * E * ceil(n / chunk)) + r(16 * (ceil(n / 128) + E))
+ * bytes, which must not exceed MOE_STATIC_SCRATCH_BYTES: n up to 1,384,448 at
+ * E = 256, 823,296 at E = 512.  Dims that need more return
  * MOE_ERR_UNSUPPORTED_SHAPE, and nothing is launched.  The first call on each
  * device looks up the array's device address (cudaGetSymbolAddress, with that
  * device current): make that first call before any stream capture.  Every

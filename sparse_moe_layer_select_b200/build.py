@@ -16,8 +16,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
          "--expt-relaxed-constexpr"]
 
-MOE_SOURCES = ["moe_api.cu", "moe_gemm.cu", "moe_gemm_pair.cu", "router_cc.cu", "index.cu",
-               "elementwise.cu", "permute_static.cu"]
+MOE_SOURCES = ["moe_api.cu", "moe_gemm.cu", "moe_gemm_pair.cu", "moe_fused.cu", "router_cc.cu",
+               "index.cu", "elementwise.cu", "permute_static.cu"]
 GEN_SOURCES = ["gen.cu"]
 
 

@@ -9,6 +9,9 @@
 //                       w_t,j, stored in expert order) and the shared-expert row: the
 //                       combine of the routed sum with the always-on shared expert
 //                       (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1)
+//   finalize_kernel     y = bf16(yacc): the fp32 token rows of the reduce combine
+//                       (the down GEMM added every scaled contribution and the
+//                       shared-expert row into them) rounded once
 //   bf16_to_f16_kernel  fp16 copy of the down-projection weights (round to nearest
 //                       even; values beyond the fp16 range are reported)
 //   selftest_wait_kernel  a bounded wait on a flag nothing sets (timeout self-test)
@@ -93,6 +96,25 @@ __global__ void __launch_bounds__(kCombineThreads)
     }
     __syncthreads();  // next token's indices staged; this token's reads done
     buf ^= 1;
+  }
+}
+
+// y = bf16(yacc): the reduce combine's fp32 accumulator rounded once (RNE), 8
+// values per thread (two 16-byte loads, one 16-byte store), grid-stride.
+__global__ void __launch_bounds__(256)
+    finalize_kernel(const float4 *__restrict__ yacc, size_t n_vec8, uint4 *__restrict__ y) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = __ldcs(&yacc[2 * i]);
+    const float4 b = __ldcs(&yacc[2 * i + 1]);
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
+    const __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y);
+    const __nv_bfloat162 p3 = __floats2bfloat162_rn(b.z, b.w);
+    y[i] = make_uint4(*reinterpret_cast<const uint32_t *>(&p0),
+                      *reinterpret_cast<const uint32_t *>(&p1),
+                      *reinterpret_cast<const uint32_t *>(&p2),
+                      *reinterpret_cast<const uint32_t *>(&p3));
   }
 }
 
@@ -254,6 +276,13 @@ cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32
     combine_kernel<8><<<grid, kCombineThreads, 0, s>>>(o4, s4, inv, T, k, vpr, y4);
   else
     combine_kernel<16><<<grid, kCombineThreads, 0, s>>>(o4, s4, inv, T, k, vpr, y4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float *yacc, size_t n, uint16_t *y, cudaStream_t s) {
+  const size_t n_vec8 = n / 8;
+  finalize_kernel<<<grid_for(n_vec8, 256), 256, 0, s>>>(reinterpret_cast<const float4 *>(yacc),
+                                                        n_vec8, reinterpret_cast<uint4 *>(y));
   return cudaGetLastError();
 }
 

@@ -407,6 +407,69 @@ __device__ __forceinline__ void down_epilogue(const GemmParams &p, const Item &i
   if (valid && amax > kF16Max) record_status(p.status, MOE_ERR_DEVICE_BOUNDS, SITE_SLOT_FP16_RANGE);
 }
 
+// GEMM2 epilogue of the reduce combine: each row's routed_scale * w * o (a
+// shared-expert row: o) is added into its token's fp32 accumulator row.  The
+// warp's 8 KB staging holds its 32 rows x 64 fp32 columns (256 bytes a row);
+// every lane stages its own row and issues that row's bulk reduce-adds, which
+// the L2 performs (the order of a token's k + 1 additions is not fixed).
+// Within a row the sixteen 16-byte chunks are stored rotated by (lane & 7)
+// places, so that the warp's shared-memory stores spread over all banks; the
+// rotated row then goes out as two bulk reductions (the chunks from the
+// rotation point on, then the wrapped ones).
+__device__ __forceinline__ void down_epilogue_reduce_cols(const GemmParams &p, const Item &it,
+                                                          uint32_t taddr, int row_local,
+                                                          EpiStage &st, int col0, int ncols) {
+  const bool shared = it.group == p.E;
+  const int q = row_local >> 5;
+  if (q * 32 >= it.nrows) return;  // no valid row in this warp's quarter (warp-uniform)
+  const int lane = row_local & 31;
+  const bool valid = row_local < it.nrows;
+  float scale = 1.f;
+  int tok = 0;
+  if (valid) {
+    if (shared) {
+      tok = it.row0 + row_local;
+    } else {
+      const int pr = p.perm[it.row0 + row_local];
+      tok = pr / p.k;
+      scale = p.routed_scale * p.topk_w[pr];
+    }
+  }
+  float *dst = p.yacc + static_cast<size_t>(tok) * p.d + col0;
+  uint8_t *row_buf = st.buf + lane * 256;
+  const int rot = lane & 7;
+  for (int cb = 0; cb < ncols; cb += 64) {
+    bulk_wait_read_all();  // this lane's previous reductions have read its staged row
+#pragma unroll
+    for (int qu = 0; qu < 4; ++qu) {  // 16 columns (four 16-byte chunks) at a time
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(taddr + cb + 16 * qu, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int pos = (4 * qu + i + rot) & 15;
+        *reinterpret_cast<float4 *>(row_buf + pos * 16) =
+            make_float4(__uint_as_float(r[4 * i]) * scale, __uint_as_float(r[4 * i + 1]) * scale,
+                        __uint_as_float(r[4 * i + 2]) * scale,
+                        __uint_as_float(r[4 * i + 3]) * scale);
+      }
+    }
+    if (valid) {
+      fence_proxy_async_smem();  // the staged row is visible to the bulk copy
+      // memory chunks rot..15 hold columns 0 .. 4 (16 - rot) - 1, chunks 0..rot-1 the rest
+      bulk_reduce_add_f32(dst + cb, row_buf + rot * 16, static_cast<uint32_t>(16 - rot) * 16);
+      if (rot) bulk_reduce_add_f32(dst + cb + 4 * (16 - rot), row_buf, static_cast<uint32_t>(rot) * 16);
+      bulk_commit_group();
+    }
+  }
+}
+
+// The reduce epilogue of an item's N tile (GEMM2 with MODE_RED).
+__device__ __forceinline__ void down_epilogue_reduce(const GemmParams &p, const Item &it,
+                                                     uint32_t taddr, int row_local, EpiStage &st) {
+  down_epilogue_reduce_cols(p, it, taddr, row_local, st, it.j * p.n_tile, p.n_tile);
+}
+
 // The part of an item that one CTA of a pair owns: rows [128 r, 128 r + 128).
 __device__ __forceinline__ Item pair_half(Item it, int rank) {
   it.row0 += rank * kBlockM;

@@ -40,6 +40,10 @@ enum GemmMode : int {
   MODE_F8 = 4,  // mode bit: e4m3 operands (tcgen05 kind::f8f6f4), per-row scales
   MODE_GEMM1_F8 = MODE_GEMM1 | MODE_F8,
   MODE_GEMM2_F8 = MODE_GEMM2 | MODE_F8,
+  // mode bit of GEMM2: the epilogue adds each scaled row into its token's fp32
+  // accumulator row (bulk reduce-add) instead of writing fp16 contribution rows
+  MODE_RED = 8,
+  MODE_GEMM2_RED = MODE_GEMM2 | MODE_RED,
 };
 // K elements of one pipeline stage: one 128-byte swizzle row of A and B.
 __host__ __device__ constexpr int stage_k(int mode) { return (mode & MODE_F8) ? 128 : kBlockK; }
@@ -67,6 +71,10 @@ struct GemmParams {
   uint16_t *h_shared;       // GEMM1 out: [T, Fs] fp16
   uint16_t *o_out;          // GEMM2 out: [T*k, d] fp16, routed_scale * w * o (expert-order rows)
   uint16_t *s_out;          // GEMM2 out: [T, d] fp16 shared-expert output
+  float *yacc;              // MODE_GEMM2_RED / fused out: [T, d] fp32 accumulator (zeroed before)
+  // fused expert kernel: the FFN width is cut into parts of fp (routed) / fp_sh
+  // (shared) columns, n_parts / n_parts_sh of them; n_ntiles = the larger count
+  int n_parts, n_parts_sh, fp, fp_sh;
   unsigned long long *trace;  // pipeline timestamps (builds with MOE_TRACE only), or null
   // MODE_F8 launches: e4m3 codes and float32 scales (one per row)
   const uint8_t *xq;        // GEMM1: token rows [T, d] e4m3 (gathered by cp.async)
@@ -95,6 +103,16 @@ struct GemmMaps {
   CUtensorMap a, b0, b1, a_sh, b0_sh, b1_sh;
   CUtensorMap out, out_sh;  // epilogue TMA stores: 64 columns x 32 rows, 128-byte swizzle
 };
+
+// Tensor maps of the fused expert kernel (128-row boxes of 64 columns).
+struct FusedMaps {
+  CUtensorMap gate, up, down, gate_sh, up_sh, down_sh;
+};
+
+// The fused expert FFN (gate/up GEMM, SwiGLU into tensor memory, down GEMM with
+// A from tensor memory, modulation and reduce combine into p.yacc); grid = SMs.
+size_t gemm_fused_smem_bytes();
+cudaError_t launch_gemm_fused(const GemmParams &p, const FusedMaps &m, int grid, cudaStream_t s);
 
 size_t gemm_smem_bytes();
 cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int grid,
@@ -144,6 +162,8 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *perm, const int
 // with inv < 0 (not routed) are skipped.
 cudaError_t launch_combine(const uint16_t *o, const uint16_t *s_out, const int32_t *inv, int T,
                            int k, int d, uint16_t *y, cudaStream_t s);
+// y = bf16(yacc), n elements (a multiple of 8).
+cudaError_t launch_finalize(const float *yacc, size_t n, uint16_t *y, cudaStream_t s);
 // Per-row e4m3 codes and float32 scales of a [rows, K] bf16 (or fp16) matrix;
 // K % 8 == 0; rows from *n_valid on (if given) are skipped; pow2: power-of-two
 // scales.
@@ -153,5 +173,9 @@ cudaError_t launch_quant_rows_e4m3(const uint16_t *src, bool is_f16, bool pow2, 
 cudaError_t launch_bf16_to_f16(const uint16_t *src, size_t n, uint16_t *dst, int *status,
                                cudaStream_t s);
 cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s);
+
+// Sets what moe_last_launch_count() reports on this host thread (entry points
+// implemented outside moe_api.cu).
+void set_last_launch_count(int n);
 
 }  // namespace moe

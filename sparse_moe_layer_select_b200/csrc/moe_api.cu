@@ -18,6 +18,7 @@ namespace moe {
 cudaError_t gemm_set_attributes();
 cudaError_t gemm_pair_set_attributes();
 cudaError_t gemm_pair_max_clusters(int *clusters);
+cudaError_t gemm_fused_set_attributes();
 }
 
 namespace {
@@ -81,6 +82,8 @@ cudaError_t device_setup(int *sms) {
     if (e != cudaSuccess) return e;
     e = gemm_pair_max_clusters(&g_pair_clusters[dev]);
     if (e != cudaSuccess) return e;
+    e = gemm_fused_set_attributes();
+    if (e != cudaSuccess) return e;
     g_attrs[dev] = true;
   }
   *sms = g_sms[dev];
@@ -117,7 +120,8 @@ struct Dims {
 };
 
 struct WsLayout {
-  size_t header, chunk_hist, tiles, tiles_pair, logits, inv, h, h_sh, o, s_out, down16, down16_sh;
+  size_t header, chunk_hist, tiles, tiles_pair, logits, inv, h, h_sh, o, s_out, yacc, down16,
+      down16_sh;
   size_t xq, sx, hq, sh, hshq, shs;  // FP8 experts: e4m3 rows of x, h, h_shared and their scales
   size_t total;
   int max_tiles;
@@ -157,14 +161,24 @@ WsLayout ws_layout(const Dims &D) {
   off += align256(static_cast<size_t>(router_ksplit(D)) * D.T * D.E * 4);
   L.inv = off;
   off += align256(n * 4);
-  L.h = off;
-  off += align256(n * D.F * 2);
-  L.h_sh = off;
-  off += align256(static_cast<size_t>(D.T) * D.Fs * 2);
-  L.o = off;  // routed contributions, expert-order rows
-  off += align256(n * D.d * 2);
-  L.s_out = off;  // shared-expert output, token rows
-  off += align256(D.Fs > 0 ? static_cast<size_t>(D.T) * D.d * 2 : 0);
+  const bool fused = (D.flags & MOE_FLAG_FUSED_EXPERTS) != 0;
+  L.h = L.h_sh = off;
+  if (!fused) {  // the fused kernel keeps h in tensor memory
+    L.h = off;
+    off += align256(n * D.F * 2);
+    L.h_sh = off;
+    off += align256(static_cast<size_t>(D.T) * D.Fs * 2);
+  }
+  L.o = L.s_out = L.yacc = off;
+  if (D.flags & (MOE_FLAG_COMBINE_REDUCE | MOE_FLAG_FUSED_EXPERTS)) {
+    L.yacc = off;  // fp32 token rows the down GEMM reduces into
+    off += align256(static_cast<size_t>(D.T) * D.d * 4);
+  } else {
+    L.o = off;  // routed contributions, expert-order rows
+    off += align256(n * D.d * 2);
+    L.s_out = off;  // shared-expert output, token rows
+    off += align256(D.Fs > 0 ? static_cast<size_t>(D.T) * D.d * 2 : 0);
+  }
   L.down16 = L.down16_sh = off;
   // per-call fp16 copy of the down projections (16-bit path without prepared copies)
   if (!(D.flags & (MOE_FLAG_DOWN_F16 | MOE_FLAG_FP8_EXPERTS))) {
@@ -191,6 +205,14 @@ WsLayout ws_layout(const Dims &D) {
   return L;
 }
 
+// Width of one part of an FFN of width f in the fused kernel: f split into the
+// fewest equal parts of at most 512 columns; 0 if a part is not a multiple of 128.
+int fused_part(int f) {
+  if (f <= 0 || f % 128 != 0) return 0;
+  const int parts = (f + 511) / 512;
+  return (f % parts == 0 && (f / parts) % 128 == 0) ? f / parts : 0;
+}
+
 moe_status check_dims(const moe_dims_t *dims, Dims *D) {
   if (dims == nullptr || dims->struct_size != sizeof(moe_dims_t)) return MOE_ERR_INVALID_ARG;
   D->T = dims->T;
@@ -203,7 +225,7 @@ moe_status check_dims(const moe_dims_t *dims, Dims *D) {
   D->norm = dims->norm_topk_prob ? 1 : 0;
   D->flags = dims->flags;
   if (D->T < 0) return MOE_ERR_INVALID_ARG;
-  if (D->d < 128 || D->d % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D->d < 64 || D->d % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (D->E < 1 || D->E > 512) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (D->k < 1 || D->k > 16 || D->k > D->E) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (D->F < 64 || D->F % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -216,6 +238,10 @@ moe_status check_dims(const moe_dims_t *dims, Dims *D) {
   // FP8 experts: K stages of 128 e4m3 elements; 256-column down-projection tiles
   if ((dims->flags & MOE_FLAG_FP8_EXPERTS) &&
       (D->F % 128 != 0 || D->Fs % 128 != 0 || D->d % 256 != 0))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  // fused experts: 128-column chunks of each FFN part and 128-column d tiles
+  if ((dims->flags & MOE_FLAG_FUSED_EXPERTS) &&
+      (D->d % 128 != 0 || fused_part(D->F) == 0 || (D->Fs > 0 && fused_part(D->Fs) == 0)))
     return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
@@ -334,6 +360,11 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
 
 }  // namespace
 
+namespace moe {
+// Launch accounting of entry points implemented in other files.
+void set_last_launch_count(int n) { g_last_launches = n; }
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_size(const moe_dims_t *dims) {
@@ -446,7 +477,9 @@ moe_status moe_forward_fp8(const moe_dims_t *dims, const moe_weights_t *w,
   Dims D;
   moe_status st = check_dims(dims, &D);
   if (st != MOE_OK) return st;
-  if (!(D.flags & MOE_FLAG_FP8_EXPERTS)) return MOE_ERR_INVALID_ARG;
+  if (!(D.flags & MOE_FLAG_FP8_EXPERTS) ||
+      (D.flags & (MOE_FLAG_COMBINE_REDUCE | MOE_FLAG_FUSED_EXPERTS)))
+    return MOE_ERR_INVALID_ARG;
   if (!w || !q || !x || !y || !routing || !w->w_router) return MOE_ERR_INVALID_ARG;
   if ((st = check_fp8_ptrs(D, q)) != MOE_OK) return st;
   if ((st = check_routing_ptrs(routing)) != MOE_OK) return st;
@@ -511,8 +544,11 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
   Tile *tiles = reinterpret_cast<Tile *>(wsp(ws, L.tiles));
   uint16_t *h = reinterpret_cast<uint16_t *>(wsp(ws, L.h));
   uint16_t *h_sh = reinterpret_cast<uint16_t *>(wsp(ws, L.h_sh));
-  uint16_t *o_out = reinterpret_cast<uint16_t *>(wsp(ws, L.o));
-  uint16_t *s_out = D.Fs > 0 ? reinterpret_cast<uint16_t *>(wsp(ws, L.s_out)) : nullptr;
+  const bool fused = (D.flags & MOE_FLAG_FUSED_EXPERTS) != 0 && !fp8;
+  const bool reduce = ((D.flags & MOE_FLAG_COMBINE_REDUCE) != 0 || fused) && !fp8;
+  uint16_t *o_out = reduce ? nullptr : reinterpret_cast<uint16_t *>(wsp(ws, L.o));
+  uint16_t *s_out = (D.Fs > 0 && !reduce) ? reinterpret_cast<uint16_t *>(wsp(ws, L.s_out)) : nullptr;
+  float *yacc = reduce ? reinterpret_cast<float *>(wsp(ws, L.yacc)) : nullptr;
   int32_t *inv = reinterpret_cast<int32_t *>(wsp(ws, L.inv));
   int launches = 0;
   EventMarker ev(s);
@@ -541,8 +577,12 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
   ix.tiles_pair = (pair1 || pair2) ? tiles_pair : nullptr;
   ix.header = header;
 
-  // 1. router (for a decode-sized batch its selection kernel also builds the index)
+  // 1. router (for a decode-sized batch its selection kernel also builds the index); the
+  // reduce combine's fp32 token rows are zeroed first (counted in the router stage)
   ev.mark();
+  if (reduce &&
+      cudaMemsetAsync(yacc, 0, static_cast<size_t>(D.T) * D.d * sizeof(float), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   bool indexed = false;
   st = route_impl(D, x, w->w_router, w->router_bias, token_mask, routing->topk_idx,
                   routing->topk_w, ws, s, sms, &launches, &ix, &indexed);
@@ -587,7 +627,8 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
 
   const int n_rows = D.T * D.k;
   const int n_half = (D.F % 128 == 0 && D.Fs % 128 == 0) ? 128 : 64;
-  const int n2 = (D.d % 256 == 0) ? 256 : 128;
+  // down-projection N tile: the widest of 256 / 128 / 64 columns that divides d
+  const int n2 = (D.d % 256 == 0) ? 256 : (D.d % 128 == 0) ? 128 : 64;
 
   GemmParams base;
   std::memset(&base, 0, sizeof(base));
@@ -607,6 +648,50 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
   base.h_shared = h_sh;
   base.o_out = o_out;
   base.s_out = s_out;
+  base.yacc = yacc;
+
+  if (fused) {
+    // 3+4. the fused expert kernel: gate/up GEMM, SwiGLU into tensor memory, down GEMM
+    // with A from tensor memory, modulation and reduce combine into yacc
+    GemmParams p = base;
+    p.tiles = tiles;
+    p.n_tiles_dev = n_tiles;
+    p.fp = fused_part(D.F);
+    p.n_parts = D.F / p.fp;
+    p.fp_sh = D.Fs > 0 ? fused_part(D.Fs) : 128;
+    p.n_parts_sh = D.Fs > 0 ? D.Fs / p.fp_sh : 0;
+    p.n_ntiles = std::max(p.n_parts, p.n_parts_sh);
+    p.x = static_cast<const uint16_t *>(x);
+    FusedMaps m;
+    std::memset(&m, 0, sizeof(m));
+    const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&m.gate, w->w_gate, static_cast<uint64_t>(D.E) * D.F, D.d, 128) ||
+        !make_map(&m.up, w->w_up, static_cast<uint64_t>(D.E) * D.F, D.d, 128) ||
+        !make_map(&m.down, wd16, static_cast<uint64_t>(D.E) * D.d, D.F, 128, f16))
+      return MOE_ERR_CUDA;
+    if (D.Fs > 0) {
+      if (!make_map(&m.gate_sh, w->ws_gate, D.Fs, D.d, 128) ||
+          !make_map(&m.up_sh, w->ws_up, D.Fs, D.d, 128) ||
+          !make_map(&m.down_sh, wsd16, D.d, D.Fs, 128, f16))
+        return MOE_ERR_CUDA;
+    } else {
+      m.gate_sh = m.gate;
+      m.up_sh = m.up;
+      m.down_sh = m.down;
+    }
+    ev.mark();
+    if (launch_gemm_fused(p, m, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    launches += 1;
+    ev.mark();  // (no separate down GEMM)
+    ev.mark();
+    if (launch_finalize(yacc, static_cast<size_t>(D.T) * D.d, static_cast<uint16_t *>(y), s) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    launches += 1;
+    ev.mark();
+    g_last_launches = launches;
+    return MOE_OK;
+  }
 
   // 3. GEMM1: gathered x rows . [W_gate | W_up]^T -> SwiGLU -> h (bf16)
   {
@@ -707,29 +792,35 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
       p.sb0 = q->s_down;
       p.sb0_sh = q->ss_down;
     }
-    if (!make_map(&m.out, o_out, n_rows, D.d, std::min(32, n_rows), f16)) return MOE_ERR_CUDA;
+    // (the reduce combine stores no rows through tensor maps: out / out_sh stay unused)
+    if (reduce) m.out = m.a;
+    else if (!make_map(&m.out, o_out, n_rows, D.d, std::min(32, n_rows), f16)) return MOE_ERR_CUDA;
     m.out_sh = m.out;
     if (D.Fs > 0) {
       if (!make_map(&m.a_sh, fp8 ? static_cast<const void *>(hshq) : h_sh, D.T, D.Fs, a_sh_rows, at))
         return MOE_ERR_CUDA;
       if (!make_map(&m.b0_sh, fp8 ? q->ws_down : wsd16, D.d, D.Fs, b_rows, at)) return MOE_ERR_CUDA;
-      if (!make_map(&m.out_sh, s_out, D.T, D.d, std::min(32, D.T), f16)) return MOE_ERR_CUDA;
+      if (!reduce && !make_map(&m.out_sh, s_out, D.T, D.d, std::min(32, D.T), f16))
+        return MOE_ERR_CUDA;
     } else {
       m.a_sh = m.a;
       m.b0_sh = m.b0;
     }
     m.b1_sh = m.b0_sh;
     ev.mark();
-    const cudaError_t e = pair2 ? launch_gemm_pair(MODE_GEMM2, p, m, pair_grid, s)
-                               : launch_gemm(fp8 ? MODE_GEMM2_F8 : MODE_GEMM2, p, m, sms, s);
+    const int mode2 = reduce ? MODE_GEMM2_RED : MODE_GEMM2;
+    const cudaError_t e = pair2 ? launch_gemm_pair(mode2, p, m, pair_grid, s)
+                               : launch_gemm(fp8 ? MODE_GEMM2_F8 : mode2, p, m, sms, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     launches += 1;
   }
-  // 5. combine: y = bf16(sum of the scaled routed rows + shared row)
+  // 5. combine: y = bf16(sum of the scaled routed rows + shared row); with the reduce
+  // combine the down GEMM already summed them in fp32, and y is that sum rounded
   ev.mark();
-  if (launch_combine(o_out, s_out, inv, D.T, D.k, D.d, static_cast<uint16_t *>(y), s) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  const cudaError_t ec =
+      reduce ? launch_finalize(yacc, static_cast<size_t>(D.T) * D.d, static_cast<uint16_t *>(y), s)
+             : launch_combine(o_out, s_out, inv, D.T, D.k, D.d, static_cast<uint16_t *>(y), s);
+  if (ec != cudaSuccess) return MOE_ERR_CUDA;
   launches += 1;
   ev.mark();
   g_last_launches = launches;

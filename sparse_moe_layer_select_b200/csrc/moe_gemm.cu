@@ -319,6 +319,8 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
         router_epilogue(p, it, taddr, row_local, bias_s);
       } else if (BASE == MODE_GEMM1) {
         swiglu_epilogue<F8>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+      } else if (MODE & MODE_RED) {
+        down_epilogue_reduce(p, it, taddr, row_local, st);
       } else {
         down_epilogue<F8>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       }
@@ -331,7 +333,7 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
         aph ^= 1;
       }
     }
-    if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
+    bulk_wait_all();  // this thread's output stores / reductions are complete
   }
 
   tc_fence_before();
@@ -370,6 +372,9 @@ cudaError_t launch_gemm(int mode, const GemmParams &p, const GemmMaps &m, int gr
     case MODE_GEMM2_F8:
       return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM2_F8>, p, m.a, m.b0, m.b1, m.a_sh,
                                 m.b0_sh, m.b1_sh, m.out, m.out_sh);
+    case MODE_GEMM2_RED:
+      return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<MODE_GEMM2_RED>, p, m.a, m.b0, m.b1, m.a_sh,
+                                m.b0_sh, m.b1_sh, m.out, m.out_sh);
     default:
       return cudaErrorInvalidValue;
   }
@@ -389,6 +394,9 @@ cudaError_t gemm_set_attributes() {
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM1_F8>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM2_RED>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(moe_gemm_kernel<MODE_GEMM2_F8>,

@@ -71,6 +71,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                          const __grid_constant__ CUtensorMap tm_b1_sh,
                          const __grid_constant__ CUtensorMap tm_out,
                          const __grid_constant__ CUtensorMap tm_out_sh) {
+  constexpr int BASE = MODE & 3;  // the GEMM; MODE_RED: the reduce-combine epilogue
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -94,7 +95,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&full[s], 2);
       // own loads: one expect_tx arrival (+ one cp.async arrival per gathering lane)
-      mbar_init(&lfull[s], MODE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
+      mbar_init(&lfull[s], BASE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -123,7 +124,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int cluster_id = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
   int *status = p.status;
-  const int half_b_rows = MODE == MODE_GEMM1 ? p.n_half : p.n_tile / 2;
+  const int half_b_rows = BASE == MODE_GEMM1 ? p.n_half : p.n_tile / 2;
 
   if (warp == 0 || warp >= kPairGather2Warp) {
     // ------------------------------------------------------------ loads
@@ -133,7 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const bool tma_warp = warp == 0;
     const int gw = tma_warp ? (kTmaWarpGathers ? 0 : -1)
                             : (kTmaWarpGathers ? 1 : 0) + (warp - kPairGather2Warp);
-    const bool gathers = MODE == MODE_GEMM1 && gw >= 0;
+    const bool gathers = BASE == MODE_GEMM1 && gw >= 0;
     if (tma_warp || gathers) {
       int s = 0;
       uint32_t ph = 0;
@@ -153,7 +154,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           gather_tokens(p, it, raw, tok);
         }
         walk.prefetch(p);
-        const uint32_t bytes = MODE == MODE_GEMM1
+        const uint32_t bytes = BASE == MODE_GEMM1
                                    ? static_cast<uint32_t>(half_b_rows * 128)
                                    : (shared ? p.a_sh_bytes : p.a_bytes) + half_b_rows * 128;
         for (int kb = 0; kb < whole.nk; ++kb) {
@@ -173,7 +174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           uint8_t *b_dst = sB + s * kPBBytes;
           const int kc = kb * kBlockK;
           if (tma_warp && lane == 0) {
-            if (MODE == MODE_GEMM1) {
+            if (BASE == MODE_GEMM1) {
               // leader: gate rows; peer: up rows of the same column block
               const int brow = (shared ? 0 : it.group * p.F) + it.j * p.n_half;
               const CUtensorMap *tm =
@@ -234,7 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           }
           MOE_TRACE_AT(p, TR_LANDED, relayed);
           ++relayed;
-          if (MODE == MODE_GEMM1) fence_proxy_async_smem();  // rows written by cp.async
+          if (BASE == MODE_GEMM1) fence_proxy_async_smem();  // rows written by cp.async
           mbar_arrive_cluster(leader_full0 + s * 8);
           if (++s == kPairStages) {
             s = 0;
@@ -247,7 +248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (leader && lane == 0) {
-      const uint32_t idesc = MODE == MODE_GEMM2 ? idesc_f16_f32(2 * kBlockM, p.n_tile)
+      const uint32_t idesc = BASE == MODE_GEMM2 ? idesc_f16_f32(2 * kBlockM, p.n_tile)
                                                 : idesc_bf16_f32(2 * kBlockM, p.n_tile);
       int s = 0;
       uint32_t ph = 0;
@@ -314,7 +315,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       tc_fence_after();
       const Item it = pair_half(whole, rank);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kPAccStride;
-      if (MODE == MODE_GEMM1) swiglu_epilogue<false>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+      if (BASE == MODE_GEMM1) swiglu_epilogue<false>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
+      else if (MODE & MODE_RED) down_epilogue_reduce(p, it, taddr, row_local, st);
       else down_epilogue<false>(p, it, taddr, row_local, st, &tm_out, &tm_out_sh);
       tc_fence_before();
       __syncwarp();
@@ -326,7 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         aph ^= 1;
       }
     }
-    if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
+    bulk_wait_all();  // this thread's output stores / reductions are complete
   }
 
   tc_fence_before();
@@ -350,14 +352,22 @@ cudaError_t launch_gemm_pair(int mode, const GemmParams &p, const GemmMaps &m, i
   if (mode == MODE_GEMM1)
     return cudaLaunchKernelEx(&cfg, moe_gemm_pair_kernel<MODE_GEMM1>, p, m.a, m.b0, m.b1, m.a_sh,
                               m.b0_sh, m.b1_sh, m.out, m.out_sh);
-  return cudaLaunchKernelEx(&cfg, moe_gemm_pair_kernel<MODE_GEMM2>, p, m.a, m.b0, m.b1, m.a_sh,
-                            m.b0_sh, m.b1_sh, m.out, m.out_sh);
+  if (mode == MODE_GEMM2_RED)
+    return cudaLaunchKernelEx(&cfg, moe_gemm_pair_kernel<MODE_GEMM2_RED>, p, m.a, m.b0, m.b1,
+                              m.a_sh, m.b0_sh, m.b1_sh, m.out, m.out_sh);
+  if (mode == MODE_GEMM2)
+    return cudaLaunchKernelEx(&cfg, moe_gemm_pair_kernel<MODE_GEMM2>, p, m.a, m.b0, m.b1, m.a_sh,
+                              m.b0_sh, m.b1_sh, m.out, m.out_sh);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t gemm_pair_set_attributes() {
   const int smem = static_cast<int>(gemm_pair_smem_bytes());
   cudaError_t e = cudaFuncSetAttribute(moe_gemm_pair_kernel<MODE_GEMM1>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(moe_gemm_pair_kernel<MODE_GEMM2_RED>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(moe_gemm_pair_kernel<MODE_GEMM2>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

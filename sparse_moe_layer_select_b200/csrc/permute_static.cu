@@ -2,9 +2,8 @@
 // callers that cannot allocate device memory.
 //
 // Some callers can't call cudaMalloc: code running inside another runtime's
-// memory pool or arena that forbids outside allocations, plugins loaded into a
-// host process that owns all device memory, or a step being captured into a
-// CUDA graph where an allocation would break the capture.  For them the
+// memory pool or arena that forbids outside allocations, or plugins loaded
+// into a host process that owns all device memory.  For them the
 // index builder's scratch (status word, per-chunk expert histograms, tile
 // list) lives in a file-scope device array of fixed size instead of a
 // caller-provided workspace.  Every GPU that loads this library keeps the
@@ -23,8 +22,10 @@ namespace {
 
 using namespace moe;
 
-// MOE_STATIC_SCRATCH_BYTES (512 KiB): room for T*k up to 262144 (token, slot)
-// pairs at E = 256 (status word, 256 chunk histograms of E ints, tile list).
+// MOE_STATIC_SCRATCH_BYTES (512 KiB): status word, per-chunk expert histograms
+// and the 128-row tile list, each section rounded up to 256 bytes (the size
+// test in moe_permute_static; T * k up to 1,384,448 pairs at E = 256 and
+// 823,296 at E = 512).
 static __device__ __align__(256) unsigned char g_permute_scratch[MOE_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -72,6 +73,7 @@ extern "C" moe_status moe_permute_static(const moe_dims_t *dims, const int32_t *
   const size_t off_hist = a256(sizeof(WsHeader));
   const size_t off_tiles = off_hist + a256(nchunks * E * sizeof(int));
   const size_t need = off_tiles + a256(max_tiles * sizeof(Tile));
+  set_last_launch_count(0);
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;
   void *base = nullptr;
@@ -84,5 +86,6 @@ extern "C" moe_status moe_permute_static(const moe_dims_t *dims, const int32_t *
                    reinterpret_cast<Tile *>(b + off_tiles), reinterpret_cast<int *>(b), counts,
                    offsets, perm, s, &launches) != cudaSuccess)
     return MOE_ERR_CUDA;
+  set_last_launch_count(launches);
   return MOE_OK;
 }

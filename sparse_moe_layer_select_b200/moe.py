@@ -28,6 +28,8 @@ MOE_FLAG_GEMM_SINGLE_CTA = 8
 MOE_FLAG_GEMM_PAIR = 16
 MOE_FLAG_BIAS_SELECTION_ONLY = 32
 MOE_FLAG_FP8_EXPERTS = 64
+MOE_FLAG_COMBINE_REDUCE = 128
+MOE_FLAG_FUSED_EXPERTS = 256
 
 # Every symbol the header declares (checked by the CPU tests).
 EXPORTED = ["moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
@@ -140,10 +142,10 @@ def make_dims(T, d_model, num_experts, num_experts_per_tok, moe_intermediate_siz
                       norm_topk_prob, flags)
 
 
-def dims_for(w, T=None, flags=0):
+def dims_for(w, T=None, flags=0, norm_topk_prob=1):
     """moe_dims_t of an inputs.Workload (optionally with another token count)."""
     return make_dims(w.T if T is None else T, w.d_model, w.E, w.k, w.F, w.Fs,
-                     w.routed_scaling_factor, 1, flags)
+                     w.routed_scaling_factor, norm_topk_prob, flags)
 
 
 def _p(t):

@@ -34,11 +34,11 @@ def device_to_host(dev):
     return out
 
 
-def run_forward(w, dev, T=None, flags=0, x=None):
+def run_forward(w, dev, T=None, flags=0, x=None, norm_topk_prob=1):
     """One moe_forward call; returns (y, routing dict, ws)."""
     import torch
     T = w.T if T is None else T
-    dims = M.dims_for(w, T=T, flags=flags)
+    dims = M.dims_for(w, T=T, flags=flags, norm_topk_prob=norm_topk_prob)
     ws = M.alloc_workspace(dims)
     ws.fill_(0xFF)  # poison: reads of never-written workspace surface as NaN
     routing = M.alloc_routing(dims)
@@ -51,12 +51,13 @@ def run_forward(w, dev, T=None, flags=0, x=None):
     return y, routing, ws
 
 
-def oracle_forward(w, h, rows=None, routing=None):
+def oracle_forward(w, h, rows=None, routing=None, norm_topk_prob=True):
     x = h["x"] if rows is None else h["x"][rows]
     return O.moe_forward(x, h["w_router"], h["w_gate"], h["w_up"], h["w_down"], w.k,
                          router_bias=h.get("router_bias"), ws_gate=h.get("ws_gate"),
                          ws_up=h.get("ws_up"), ws_down=h.get("ws_down"),
-                         routed_scaling_factor=w.routed_scaling_factor, routing=routing)
+                         routed_scaling_factor=w.routed_scaling_factor, routing=routing,
+                         norm_topk_prob=norm_topk_prob)
 
 
 def check_routing(gpu_idx, gpu_w, ref, k, max_diff_frac=1e-3):

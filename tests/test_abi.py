@@ -51,7 +51,8 @@ def test_workspace_size_and_shape_limits(L):
     n = M.workspace_size(ok)
     # slots alone: T * (k + 1) * d * 2 bytes
     assert n >= 4096 * 9 * 2048 * 2 and n % 256 == 0
-    bad = [M.make_dims(64, 100, 16, 4, 128, 128),      # d not a multiple of 128
+    bad = [M.make_dims(64, 100, 16, 4, 128, 128),      # d not a multiple of 64
+           M.make_dims(64, 96, 16, 4, 128, 128),       # d not a multiple of 64
            M.make_dims(64, 256, 16, 17, 128, 128),     # k > 16
            M.make_dims(64, 256, 4, 5, 128, 128),       # k > E
            M.make_dims(64, 256, 1024, 4, 128, 128),    # E > 512
@@ -62,6 +63,28 @@ def test_workspace_size_and_shape_limits(L):
     d = M.make_dims(64, 256, 16, 4, 128, 128)
     d.struct_size = 4
     assert M.workspace_size(d) == 0
+
+
+def test_fused_and_reduce_combine_shape_rules_and_workspace(L):
+    """The fused kernel needs F, Fs, d multiples of 128 and FFN parts (<= 512 columns, equal)
+    of whole 128-column chunks; its workspace holds no h and no fp16 contribution rows, only
+    the fp32 token rows (so does the reduce combine's, which keeps h)."""
+    F_ = M.MOE_FLAG_FUSED_EXPERTS
+    R_ = M.MOE_FLAG_COMBINE_REDUCE
+    for ok in [(4096, 2048, 256, 8, 512, 512), (64, 256, 16, 4, 1024, 1024),
+               (64, 256, 16, 4, 768, 0), (64, 256, 16, 4, 1536, 128)]:
+        assert M.workspace_size(M.make_dims(*ok, flags=F_)) > 0, ok
+    for bad in [(64, 256, 16, 4, 640, 128),    # two parts of 320: not whole 128-column chunks
+                (64, 256, 16, 4, 192, 128),    # F not a multiple of 128
+                (64, 192, 16, 4, 128, 128)]:   # d not a multiple of 128
+        assert M.workspace_size(M.make_dims(*bad, flags=F_)) == 0, bad
+    T, d, E, k, F, Fs = 4096, 2048, 256, 8, 512, 512
+    base = M.workspace_size(M.make_dims(T, d, E, k, F, Fs))
+    red = M.workspace_size(M.make_dims(T, d, E, k, F, Fs, flags=R_))
+    fus = M.workspace_size(M.make_dims(T, d, E, k, F, Fs, flags=F_))
+    slots, yacc, h = T * (k + 1) * d * 2, T * d * 4, (T * k + T) * F * 2
+    assert abs((base - red) - (slots - yacc)) < 4096
+    assert abs((red - fus) - h) < 4096
 
 
 def test_workspace_holds_one_logit_plane_per_router_slice(L):

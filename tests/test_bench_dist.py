@@ -97,7 +97,9 @@ def test_stored_traffic_matches_the_sources():
 
 def test_stage_work_of_the_t4096_workload():
     """Algorithmic work behind the roofline numbers, against sums done by hand for the
-    T=4096 XS.2 workload (d=2048, E=256, k=8, F=Fs=512) with every expert touched."""
+    T=4096 XS.2 workload (d=2048, E=256, k=8, F=Fs=512) with every expert touched.  The
+    stages' "bytes" are the method's own (weights once, x, y); the intermediates (h, the
+    routed contributions, the shared output) are counted apart."""
     sys.path.insert(0, ROOT)
     import numpy as np
     import bench
@@ -105,13 +107,25 @@ def test_stage_work_of_the_t4096_workload():
     w = I.get("c2_xs2_small")
     work = bench.stage_work(w, np.ones(256, dtype=np.int64))
     # W_gate + W_up of 256 experts (2 x 512 x 2048 bf16 each) = 1073741824, shared gate + up
-    # 4194304, x 16777216, h (32768 routed + 4096 shared rows of 512 fp16) 37748736
-    assert work["gemm1_swiglu"]["bytes"] == 1132462080
+    # 4194304, x 16777216
+    assert work["gemm1_swiglu"]["bytes"] == 1073741824 + 4194304 + 16777216
+    # h: 32768 routed + 4096 shared rows of 512 fp16
+    assert work["gemm1_swiglu"]["inter_bytes"] == 37748736
     # 4 d F per routed row (gate and up, 2 flops per MAC) + the same per shared row
     assert work["gemm1_swiglu"]["flops"] == 4 * 2048 * 512 * (32768 + 4096)
-    # W_down 536870912 + shared 2097152 + h 37748736 + O and S (9 rows of 2048 fp16 per token)
-    assert work["gemm2_down_scale"]["bytes"] == 536870912 + 2097152 + 37748736 + 4096 * 9 * 4096
+    # W_down 536870912 + shared 2097152; h read, O and S written (9 rows of 2048 fp16 per token)
+    assert work["gemm2_down_scale"]["bytes"] == 536870912 + 2097152
+    assert work["gemm2_down_scale"]["inter_bytes"] == 37748736 + 4096 * 9 * 4096
+    # y written
+    assert work["combine"]["bytes"] == 4096 * 2048 * 2
+    # the layer: 1.61 GB of expert weights + shared 6.3 MB + router 1 MB + x, y 33.6 MB
+    # (+ the routing arrays, 0.66 MB)
+    lb = bench.layer_bytes(work)
+    assert lb == (1073741824 + 536870912 + 3 * 2097152 + 1048576 + 2 * 16777216
+                  + 4096 * 8 * 8 + 4096 * 8 * 12 + 256 * 8)
+    assert 1.64e9 < lb < 1.66e9
     # half the expert weight bytes with e4m3, plus a float32 scale per weight row
     f8 = bench.stage_work(w, np.ones(256, dtype=np.int64), fp8=True)
-    assert f8["gemm1_swiglu"]["bytes"] == (1073741824 + 4194304) // 2 + 16777216 + 37748736 + \
-        4 * (256 * (2 * 512 + 2048) + 2 * 512 + 2048)
+    assert f8["gemm1_swiglu"]["bytes"] == (1073741824 + 4194304) // 2 + 16777216 + \
+        4 * (256 * 2 * 512 + 2 * 512)
+    assert f8["gemm2_down_scale"]["bytes"] == (536870912 + 2097152) // 2 + 4 * (256 * 2048 + 2048)

@@ -416,6 +416,73 @@ def test_exact_ties_go_to_lower_expert_index(flags):
     G.check_output(G.y_numpy(y), ref["y"], what="ties")
 
 
+ROUTERS = [M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR]
+
+
+@pytest.mark.parametrize("router", ROUTERS)
+def test_more_than_32_experts_in_the_refine_band(router):
+    """40 of 64 experts share one router row, so for every token the k-th and (k+1)-th
+    places (k = 8) lie among 40 exactly tied experts: more than a warp's worth of band
+    members, which the select kernel re-decides through its streamed fallback.  Inputs are
+    small dyadic numbers, so every logit is exact in fp32 and float64 on both sides; the
+    tied experts' logit (8) is far above every other expert's.  The oracle gives the 8
+    lowest ids among the tied ones, in ascending id (equal scores), each with weight 1/8."""
+    import torch
+    T, d, E, k = 200, 256, 64, 8
+    w = I.get("c1_tiny").with_(T=T, d_model=d, num_experts=E, num_experts_per_tok=k)
+    rng = np.random.default_rng(40)
+    h = I.host_inputs(w)
+    x = rng.integers(-1, 2, size=(T, d)).astype(np.float64)
+    x[:, 0] = 1.0
+    wr = rng.integers(-1, 2, size=(E, d)).astype(np.float64) * 2.0 ** -4
+    wr[:, 0] = 0.0
+    tied = np.arange(10, 50)
+    wr[tied] = 0.0
+    wr[tied, 0] = 8.0
+    h["x"] = I.f64_to_bf16_bits(x)
+    h["w_router"] = I.f64_to_bf16_bits(wr)
+    dev = G.host_to_device(h)
+    y, routing, ws = G.run_forward(w, dev, flags=router)
+    ref = G.oracle_forward(w, h)
+    want = np.tile(np.arange(10, 10 + k), (T, 1))
+    assert np.array_equal(ref["topk_idx"], want)
+    idx = routing["topk_idx"].cpu().numpy()
+    assert np.array_equal(idx, want), idx[:3]
+    assert np.array_equal(routing["topk_w"].cpu().numpy(), np.full((T, k), 0.125, np.float32))
+    off = M.logits_offset(M.dims_for(w, flags=router))
+    logits = ws[off:off + T * E * 4].view(torch.float32).view(T, E).cpu().numpy()
+    assert np.array_equal(logits[:, tied], np.full((T, tied.size), 8.0, np.float32))
+    G.check_output(G.y_numpy(y), ref["y"], what="40-way tie")
+
+
+@pytest.mark.parametrize("router,engine", [(M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_GEMM_SINGLE_CTA),
+                                           (M.MOE_FLAG_ROUTER_TENSOR, M.MOE_FLAG_GEMM_PAIR)])
+def test_unnormalised_weights(router, engine):
+    """norm_topk_prob = 0: every weight is the selected expert's own sigmoid score (the
+    oracle's branch is pinned by a plain-Python evaluation); the routed sum uses them as
+    they are."""
+    w = I.get("c1_tiny").with_(T=300)
+    h, dev = _small(w)
+    y, routing, _ = G.run_forward(w, dev, flags=router | engine, norm_topk_prob=0)
+    ref = G.oracle_forward(w, h, norm_topk_prob=False)
+    assert np.all(np.abs(ref["topk_w"].sum(axis=1) - 1.0) > 1e-3)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
+    G.check_output(G.y_numpy(y), ref["y"], what="norm_topk_prob=0")
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+@pytest.mark.parametrize("d", [64, 192, 320])
+def test_d_model_multiple_of_64(d, engine):
+    """d_model only a multiple of 64: the down projection runs on 64-column N tiles (and
+    the router on 3 or 5 K blocks); ragged token tiles, full oracle."""
+    w = I.get("c1_tiny").with_(T=300, d_model=d)
+    h, dev = _small(w)
+    y, routing, _ = G.run_forward(w, dev, flags=engine)
+    ref = G.oracle_forward(w, h)
+    G.check_routing(routing["topk_idx"].cpu().numpy(), routing["topk_w"].cpu().numpy(), ref, w.k)
+    G.check_output(G.y_numpy(y), ref["y"], what=f"d={d}")
+
+
 @pytest.mark.parametrize("flags", [M.MOE_FLAG_ROUTER_CUDA_CORE, M.MOE_FLAG_ROUTER_TENSOR])
 def test_router_logits_error_against_float64(flags):
     """fp32 logits of both router paths against the oracle's float64 logits (XS.2 widths)."""

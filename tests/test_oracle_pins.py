@@ -242,6 +242,33 @@ def test_full_layer_against_plain_python_per_token():
         assert np.allclose(out["y"][t], ref, rtol=1e-12, atol=1e-14)
 
 
+def test_unnormalised_weights_are_the_selected_sigmoid_scores():
+    """norm_topk_prob off (a config key of the spec sheet; both Laguna models set it on):
+    each weight is the selected expert's own sigmoid score, with no division by the sum.
+    Every token evaluated by definition in plain Python."""
+    rng = np.random.default_rng(21)
+    T, d, E, k, F, Fs = 6, 5, 6, 3, 3, 2
+    L = _rand_layer(rng, T, d, E, F, Fs, scale=0.7)
+    out = _fwd(L, k, norm_topk_prob=False)
+    _, sc = _py_logits_scores(L["x"].tolist(), L["w_router"].tolist())
+    for t in range(T):
+        sel = _brute_force_topk(sc[t], k)
+        assert sorted(out["topk_idx"][t].tolist()) == list(sel)
+        got_w = dict(zip(out["topk_idx"][t].tolist(), out["topk_w"][t].tolist()))
+        assert all(math.isclose(got_w[e], sc[t][e], rel_tol=1e-14) for e in sel)
+        acc = [0.0] * d
+        for e in sel:
+            o = _py_swiglu(L["x"][t].tolist(), L["w_gate"][e].tolist(), L["w_up"][e].tolist(),
+                           L["w_down"][e].tolist())
+            acc = [a + sc[t][e] * v for a, v in zip(acc, o)]
+        s = _py_swiglu(L["x"][t].tolist(), L["ws_gate"].tolist(), L["ws_up"].tolist(),
+                       L["ws_down"].tolist())
+        ref = [2.5 * a + b for a, b in zip(acc, s)]
+        assert np.allclose(out["y"][t], ref, rtol=1e-12, atol=1e-14)
+    # the sum over the selection is not 1 (it is with normalisation on)
+    assert np.all(np.abs(out["topk_w"].sum(axis=1) - 1.0) > 1e-3)
+
+
 # ---------------------------------------------------------------- invariants
 
 def test_token_permutation_equivariance():

@@ -1,11 +1,12 @@
 """moe_permute_static: the expert-order permutation without a workspace.
 
 Callers that cannot allocate device memory (code inside another runtime's
-memory pool, plugins whose host process owns all device memory, or work being
-captured into a CUDA graph) get the permutation from this entry point, whose
-scratch is a static device array inside the library.  Its output must be
-identical to moe_permute's on the same input, call after call (the array keeps
-the previous call's contents, which must not leak into the next one).
+memory pool, or plugins whose host process owns all device memory) get the
+permutation from this entry point, whose scratch is a static device array
+inside the library.  Its output must be identical to moe_permute's on the same
+input, call after call (the array keeps the previous call's contents, which
+must not leak into the next one), and a call must not change how much device
+memory is in use.
 """
 import ctypes
 
@@ -14,6 +15,8 @@ import pytest
 
 from sparse_moe_layer_select_b200 import build as B
 from sparse_moe_layer_select_b200 import moe as M
+
+SCRATCH = 512 * 1024
 
 
 def _p(t):
@@ -27,40 +30,113 @@ def _routing(T, E, k, seed):
     return np.stack([rng.choice(E, size=k, replace=False, p=pop) for _ in range(T)]).astype(np.int32)
 
 
+def _chunk_entries(n):
+    if n <= 4096:
+        return 4096
+    c = 1024
+    while c < 4096 and c * 48 < n:
+        c *= 2
+    return c
+
+
+def _static_bytes(n, E):
+    """Scratch bytes of one call for n = T * k pairs (the size rule stated in moe.h)."""
+    r = lambda b: (b + 255) // 256 * 256
+    nchunks = max(-(-n // _chunk_entries(n)), 1)
+    return 256 + r(4 * E * nchunks) + r(16 * (-(-n // 128) + E))
+
+
+def test_size_rule_limits_match_the_header():
+    for E, n_max in [(256, 1_384_448), (512, 823_296)]:
+        assert _static_bytes(n_max, E) <= SCRATCH < _static_bytes(n_max + 1, E)
+        assert all(_static_bytes(n, E) <= SCRATCH for n in range(1, n_max + 1, 997))
+
+
 def test_rejects_dims_beyond_the_static_scratch():
+    import torch
     B.build()
     L = M.lib()
-    big = M.make_dims(262144, 2048, 256, 8, 512, 512)   # T*k = 2,097,152 pairs
-    rc = L.moe_permute_static(ctypes.byref(big), ctypes.c_void_p(256), ctypes.c_void_p(512),
-                              ctypes.c_void_p(768), ctypes.c_void_p(1024), None)
-    assert rc == M.MOE_ERR_UNSUPPORTED_SHAPE
+    # fake 16-byte-aligned device addresses: rejected calls never dereference them
+    fake = [ctypes.c_void_p(a) for a in (256, 512, 768, 1024)]
+    for E, n_max in [(256, 1_384_448), (512, 823_296)]:
+        for k in (8, 16):
+            T = n_max // k + 1                        # T * k just past the limit
+            d = M.make_dims(T, 2048, E, k, 512, 512)
+            assert L.moe_permute_static(ctypes.byref(d), *fake, None) == M.MOE_ERR_UNSUPPORTED_SHAPE
+            assert M.last_launch_count() == 0
+        if not torch.cuda.is_available():
+            # at the limit the size check passes and the call reaches CUDA (absent here)
+            d = M.make_dims(n_max // 8, 2048, E, 8, 512, 512)
+            assert L.moe_permute_static(ctypes.byref(d), *fake, None) == M.MOE_ERR_CUDA
+
+
+def _run(L, dims, idx, E, T, k, use_static, stream):
+    import torch
+    counts = torch.full((E,), -7, dtype=torch.int32, device="cuda")
+    offsets = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    perm = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    if use_static:
+        rc = L.moe_permute_static(ctypes.byref(dims), _p(idx), _p(counts), _p(offsets), _p(perm),
+                                  ctypes.c_void_p(stream.cuda_stream))
+        assert rc == M.MOE_OK, M.status_string(rc)
+        assert M.last_launch_count() == (1 if T * k <= 4096 else 2)
+    else:
+        ws = M.alloc_workspace(dims)
+        M.permute(dims, idx, counts, offsets, perm, ws)
+    torch.cuda.synchronize()
+    return counts.cpu().numpy(), offsets.cpu().numpy(), perm.cpu().numpy()
 
 
 @pytest.mark.gpu
-def test_static_scratch_permute_matches_workspace_permute_twice():
+def test_static_scratch_permute_matches_workspace_permute_call_after_call():
     import torch
     B.build()
     L = M.lib()
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
-    # two calls in a row with different sizes: the second must not see the first's scratch
-    for (T, E, k, seed) in [(4096, 256, 8, 1), (1000, 64, 6, 2)]:
+    # single-chunk (decode-sized) and multi-chunk batches, larger then smaller, the same size
+    # twice and smaller then larger: no call may see the previous call's scratch
+    cases = [(4096, 256, 8, 1), (1000, 64, 6, 2), (1000, 64, 6, 3), (4096, 256, 8, 4),
+             (64, 256, 8, 5), (6000, 64, 6, 6), (512, 16, 8, 7), (40000, 256, 8, 8)]
+    for (T, E, k, seed) in cases:
         idx = torch.from_numpy(_routing(T, E, k, seed)).cuda()
         dims = M.make_dims(T, 256, E, k, 128, 128)
-        outs = []
-        for use_static in (False, True):
-            counts = torch.full((E,), -7, dtype=torch.int32, device="cuda")
-            offsets = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
-            perm = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
-            if use_static:
-                rc = L.moe_permute_static(ctypes.byref(dims), _p(idx), _p(counts), _p(offsets),
-                                          _p(perm), ctypes.c_void_p(stream.cuda_stream))
-                assert rc == M.MOE_OK, M.status_string(rc)
-            else:
-                ws = M.alloc_workspace(dims)
-                M.permute(dims, idx, counts, offsets, perm, ws)
-            torch.cuda.synchronize()
-            outs.append((counts.cpu().numpy(), offsets.cpu().numpy(), perm.cpu().numpy()))
-        for a, b in zip(outs[0], outs[1]):
-            assert np.array_equal(a, b)
-        assert outs[1][1][-1] == T * k and sorted(outs[1][2].tolist()) == list(range(T * k))
+        ref = _run(L, dims, idx, E, T, k, False, stream)
+        got = _run(L, dims, idx, E, T, k, True, stream)
+        for a, b in zip(ref, got):
+            assert np.array_equal(a, b), (T, E, k)
+        assert got[1][-1] == T * k and sorted(got[2].tolist()) == list(range(T * k))
+
+
+@pytest.mark.gpu
+def test_static_scratch_permute_allocates_nothing():
+    import torch
+    B.build()
+    L = M.lib()
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    sizes = [(64, 256, 8), (20000, 256, 8)]      # the single-CTA and the multi-chunk index
+    bufs = []
+    for (T, E, k) in sizes:
+        idx = torch.from_numpy(_routing(T, E, k, 11)).cuda()
+        out = (torch.empty(E, dtype=torch.int32, device="cuda"),
+               torch.empty(E + 1, dtype=torch.int32, device="cuda"),
+               torch.empty(T * k, dtype=torch.int32, device="cuda"))
+        bufs.append((M.make_dims(T, 256, E, k, 128, 128), idx, out))
+
+    def call(dims, idx, out):
+        rc = L.moe_permute_static(ctypes.byref(dims), _p(idx), *[_p(t) for t in out],
+                                  ctypes.c_void_p(stream.cuda_stream))
+        assert rc == M.MOE_OK, M.status_string(rc)
+
+    for b in bufs:          # first calls: symbol lookup and module loading happen here
+        call(*b)
+    torch.cuda.synchronize()
+    torch_before = torch.cuda.memory_allocated()
+    free_before, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        for b in bufs:
+            call(*b)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == torch_before
+    assert torch.cuda.mem_get_info()[0] == free_before
