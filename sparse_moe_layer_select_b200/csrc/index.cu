@@ -27,8 +27,11 @@
 //                         experts from __match_any_sync (stable, deterministic)
 // With a single chunk (decode-sized batches) one CTA does all three steps in
 // one launch (index_single_kernel), or, inside a layer forward with E <= 256,
-// the last CTA of the router's selection kernel does (router_cc.cu).  The
-// device steps themselves are in index_common.cuh.
+// the last CTA of the router's selection kernel does (router_cc.cu).  With up
+// to as many chunks as can be resident at once, one cooperative launch does
+// them (index_coop_kernel, a grid barrier between the histograms and the
+// scatter); beyond that the two kernels above run.  The device steps
+// themselves are in index_common.cuh.
 #include "index_common.cuh"
 #include "kernels.h"
 #include "status.cuh"
@@ -80,6 +83,106 @@ __global__ void __launch_bounds__(kIdxWarps * 32)
   chunk_warp_scatter(topk_idx, n, E, blockIdx.x, h, perm, inv, sub);
 }
 
+// All of the above in one cooperative launch (every chunk's CTA resident at
+// once): each CTA keeps its per-warp histograms in shared memory, publishes its
+// chunk totals and waits at a grid barrier (an arrival counter in the workspace
+// header, a bounded spin); then every CTA derives its own chunk's base row of
+// each expert from the totals (the sum over the chunks before it plus the
+// expert's offset, an exclusive scan over experts that each CTA repeats), CTA
+// 0 writes counts, offsets and the tile lists, and every CTA scatters its
+// entries.  One launch and no second pass over the routing instead of two.
+__global__ void __launch_bounds__(512)
+    index_coop_kernel(const int32_t *__restrict__ topk_idx, int n, int E, int T, int with_shared,
+                      int *__restrict__ chunk_hist, int32_t *__restrict__ counts,
+                      int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                      int32_t *__restrict__ inv, Tile *__restrict__ tiles,
+                      Tile *__restrict__ tiles_pair, int *__restrict__ header, int sub) {
+  __shared__ int h[kIdxWarps * kMaxE];
+  __shared__ int warp_sums[32];
+  __shared__ int totals[3];
+  __shared__ int go;
+  const int nchunks = gridDim.x;
+  chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, header, sub);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) s += h[w * E + e];
+    chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = s;
+  }
+  __threadfence();  // this chunk's totals are visible before its arrival
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int *arrived = &reinterpret_cast<WsHeader *>(header)->index_arrived;
+    atomicAdd(arrived, 1);
+    const long long t0 = clock64();
+    int ok = 1;
+    while (*reinterpret_cast<volatile int *>(arrived) < nchunks) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        record_status(header, MOE_ERR_DEVICE_TIMEOUT, SITE_INDEX_GRID_BARRIER);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    go = ok;
+  }
+  __syncthreads();
+  if (!go) return;
+  // this chunk's base row of each expert: offset of the expert + rows in earlier chunks
+  const int e = threadIdx.x;
+  int total = 0, before = 0;
+  if (e < E) {
+    int c = 0;
+    for (; c + 8 <= nchunks; c += 8) {  // eight independent loads in flight
+      int v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __ldcg(&chunk_hist[static_cast<size_t>(c + q) * E + e]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        total += v[q];
+        before += (c + q) < static_cast<int>(blockIdx.x) ? v[q] : 0;
+      }
+    }
+    for (; c < nchunks; ++c) {
+      const int v = __ldcg(&chunk_hist[static_cast<size_t>(c) * E + e]);
+      total += v;
+      before += c < static_cast<int>(blockIdx.x) ? v : 0;
+    }
+  }
+  const int off = block_exclusive_scan(e < E ? total : 0, warp_sums, &totals[0]);
+  if (blockIdx.x == 0) {
+    if (e < E) {
+      counts[e] = total;
+      offsets[e] = off;
+    }
+    if (e == 0) offsets[E] = totals[0];
+    const int n1 = write_tiles(e, total, off, E, T, with_shared, kBlockM, tiles, warp_sums,
+                               &totals[1]);
+    int n2 = 0;
+    if (tiles_pair != nullptr)
+      n2 = write_tiles(e, total, off, E, T, with_shared, 2 * kBlockM, tiles_pair, warp_sums,
+                       &totals[2]);
+    if (threadIdx.x == 0) {
+      reinterpret_cast<WsHeader *>(header)->n_tiles = n1;
+      reinterpret_cast<WsHeader *>(header)->n_tiles_pair = n2;
+    }
+  }
+  // per-warp first rows of this chunk (the shared-memory histograms of phase 1)
+  if (e < E) {
+    int run = off + before;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) {
+      const int c = h[w * E + e];
+      h[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  // the chunk's entries belong to its first kIdxWarps warps (sub entries each); the
+  // CTA's other warps only took part in the scans
+  if ((threadIdx.x >> 5) < kIdxWarps) chunk_warp_scatter(topk_idx, n, E, blockIdx.x, h, perm, inv, sub);
+}
+
 // All of the above for a single chunk (n <= kIndexChunk), in one CTA of 512
 // threads.
 __global__ void __launch_bounds__(512)
@@ -97,6 +200,24 @@ __global__ void __launch_bounds__(512)
 
 }  // namespace
 
+// How many index_coop_kernel CTAs can be resident at once on the current
+// device (0 if the query fails): the one-launch builder is used only for up to
+// that many chunks.
+int coop_index_max_ctas() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, index_coop_kernel, 512, 0) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    cached[dev] = per_sm * sms > 0 ? per_sm * sms : -1;
+  }
+  return cached[dev] > 0 ? cached[dev] : 0;
+}
+
 cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_shared,
                          int *chunk_hist, Tile *tiles, int *status, int32_t *counts,
                          int32_t *offsets, int32_t *perm, cudaStream_t s, int *launches,
@@ -109,6 +230,22 @@ cudaError_t launch_index(const int32_t *topk_idx, int T, int k, int E, int with_
                                           offsets, perm, inv, tiles, tiles_pair, status);
     *launches += 1;
     return cudaGetLastError();
+  }
+  if (E <= 512 && nchunks <= coop_index_max_ctas()) {
+    // one cooperative launch: all chunk CTAs are resident together
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nchunks);
+    cfg.blockDim = dim3(512);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeCooperative;
+    attr.val.cooperative = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const int sub = chunk / kIdxWarps;
+    *launches += 1;
+    return cudaLaunchKernelEx(&cfg, index_coop_kernel, topk_idx, n, E, T, with_shared, chunk_hist,
+                              counts, offsets, perm, inv, tiles, tiles_pair, status, sub);
   }
   index_hist_scan_kernel<<<nchunks, 512, 0, s>>>(topk_idx, n, E, nchunks, T, with_shared,
                                                   chunk_hist, counts, offsets, tiles, tiles_pair,

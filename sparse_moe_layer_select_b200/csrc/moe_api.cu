@@ -206,11 +206,17 @@ WsLayout ws_layout(const Dims &D) {
 }
 
 // Width of one part of an FFN of width f in the fused kernel: f split into the
-// fewest equal parts of at most 512 columns; 0 if a part is not a multiple of 128.
-int fused_part(int f) {
+// fewest equal parts of at most 512 columns (and at least min_parts parts, as
+// far as parts of whole 128-column chunks allow); 0 if no such split exists.
+int fused_part(int f, int min_parts = 1) {
   if (f <= 0 || f % 128 != 0) return 0;
-  const int parts = (f + 511) / 512;
-  return (f % parts == 0 && (f / parts) % 128 == 0) ? f / parts : 0;
+  int parts = (f + 511) / 512;
+  while (parts <= f / 128 && (f % parts != 0 || (f / parts) % 128 != 0)) ++parts;
+  if (parts > f / 128) return 0;
+  int best = parts;
+  for (int q = parts; q <= f / 128 && best < min_parts; ++q)
+    if (f % q == 0 && (f / q) % 128 == 0) best = q;
+  return f / best;
 }
 
 moe_status check_dims(const moe_dims_t *dims, Dims *D) {
@@ -656,9 +662,20 @@ moe_status forward_impl(const Dims &D, const moe_weights_t *w, const moe_fp8_wei
     GemmParams p = base;
     p.tiles = tiles;
     p.n_tiles_dev = n_tiles;
-    p.fp = fused_part(D.F);
+    // Items are (row tile, FFN part).  With few tiles (small batches: about one tile
+    // per touched expert) the FFN is cut into more parts so that the persistent grid
+    // has about three items per SM; each part adds its partial down projection into
+    // the token rows, so more parts cost more reduce-adds (cheap at these sizes).
+    const int64_t tiles_est = std::min<int64_t>(D.E, static_cast<int64_t>(D.T) * D.k) +
+                              (static_cast<int64_t>(D.T) * D.k + kBlockM - 1) / kBlockM;
+    const int want_parts = static_cast<int>(std::min<int64_t>(
+        D.F / 128, (3 * static_cast<int64_t>(sms) + tiles_est - 1) / std::max<int64_t>(tiles_est, 1)));
+    p.fp = fused_part(D.F, want_parts);
     p.n_parts = D.F / p.fp;
-    p.fp_sh = D.Fs > 0 ? fused_part(D.Fs) : 128;
+    // The shared expert's tiles come last in the tile list, so with few of them their
+    // items are cut to single 128-column chunks and do not trail the routed ones.
+    const int sh_tiles = (D.T + kBlockM - 1) / kBlockM;
+    p.fp_sh = D.Fs > 0 ? fused_part(D.Fs, sh_tiles < sms ? D.Fs / 128 : want_parts) : 128;
     p.n_parts_sh = D.Fs > 0 ? D.Fs / p.fp_sh : 0;
     p.n_ntiles = std::max(p.n_parts, p.n_parts_sh);
     p.x = static_cast<const uint16_t *>(x);

@@ -14,11 +14,12 @@
 //              cp.async arrivals)
 //   gather     GEMM1's A rows are copied by warps 7.. (each a share of the
 //              128 rows, gemm_common.cuh); warp 0 issues the TMA loads
-//   relay      warp 6 of each CTA forwards each completed stage to the
-//              leader's full[s] (two arrivals per phase), after a proxy fence
-//              for the cp.async-written rows; each CTA can therefore always
-//              drain its own copies
-//   full[s]    leader: both halves of stage s are in shared memory
+//   relay      warp 6 of the peer CTA forwards each of its completed stages
+//              to the leader's full[s], after a proxy fence for the
+//              cp.async-written rows; each CTA can therefore always drain its
+//              own copies
+//   full[s]    leader: the peer's half of stage s is in shared memory (the
+//              leader's MMA thread waits on its own lfull[s] for its half)
 //   empty[s]   per CTA: the leader's MMAs of stage s completed (commit
 //              multicast to both CTAs)
 //   acc_full   per CTA: an accumulator is complete (commit multicast)
@@ -93,7 +94,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
-      mbar_init(&full[s], 2);
+      mbar_init(&full[s], 1);  // the peer's relayed arrival (the leader waits on its own lfull)
       // own loads: one expect_tx arrival (+ one cp.async arrival per gathering lane)
       mbar_init(&lfull[s], BASE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
       mbar_init(&empty[s], 1);
@@ -216,8 +217,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
     }
   } else if (warp == 6) {
-    // ------------------------------------------------------------ relay (both CTAs)
-    if (lane == 0) {
+    // ------------------------------------------------------------ relay (peer CTA)
+    // The leader's MMA thread waits on the leader's own lfull; only the peer's
+    // completed stages are forwarded, one remote arrival each on the leader's full.
+    if (lane == 0 && !leader) {
       const uint32_t leader_full0 = map_shared_rank(smem_u32(&full[0]), 0);
       int s = 0;
       uint32_t ph = 0;
@@ -265,11 +268,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kPAccStride;
         for (int kb = 0; kb < it.nk; ++kb) {
-          if (!mbar_wait(&full[s], ph, status, SITE_GEMM_MMA_FULL)) {
+          // this CTA's half of the stage (its loads), then the peer's (relayed)
+          if (!mbar_wait(&lfull[s], ph, status, SITE_GEMM_MMA_FULL) ||
+              !mbar_wait(&full[s], ph, status, SITE_GEMM_MMA_FULL)) {
             ok = false;
             break;
           }
           MOE_TRACE_AT(p, TR_FULL, consumed);
+          if (BASE == MODE_GEMM1) fence_proxy_async_smem();  // own rows written by cp.async
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kPABytes);
           const uint32_t b0 = smem_u32(sB + s * kPBBytes);

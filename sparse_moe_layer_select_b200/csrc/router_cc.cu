@@ -12,10 +12,12 @@
 //                         loads of W_r, fp32 FMA, warp butterfly reduction).
 //   router_select_kernel  one warp per token, for both logit paths: the E
 //                         logits sit in registers (E/32 per lane) as
-//                         order-preserving integer keys; k+1 rounds of a warp
-//                         arg-max (a max- then a min-reduction, ties to the
-//                         lower expert index) pick the experts in descending
-//                         order; tokens whose
+//                         order-preserving integer keys; each lane keeps the
+//                         top three of its keys (rebuilt when all three are
+//                         taken), and k+1 rounds of a warp arg-max over the
+//                         lanes' heads (a max- then a min-reduction, ties to
+//                         the lower expert index) pick the experts in
+//                         descending order; tokens whose
 //                         k-th and (k+1)-th logits are within kRefineBand get
 //                         the experts near that boundary re-decided on float64
 //                         logits; sigmoid and normalisation in fp32.  When
@@ -186,10 +188,10 @@ __device__ __forceinline__ float key_logit(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
-// One warp per token: each lane sorts its NPL = E/32 logits once (odd-even
-// transposition network, registers only); each of the k+1 rounds then takes
-// the warp arg-max of the 32 list heads (ties to the lower expert id) and the
-// winning lane pops its head.  Tokens whose k-th and (k+1)-th logits are
+// One warp per token: each lane keeps the top three of its NPL = E/32 logits
+// (registers only); each of the k+1 rounds then takes the warp arg-max of the
+// 32 list heads (ties to the lower expert id) and the winning lane pops its
+// head, rebuilding its list from its remaining logits when it runs empty.  Tokens whose k-th and (k+1)-th logits are
 // within kRefineBand get the experts near that boundary re-decided on
 // float64 logits.  Then sigmoid scores and post-top-k normalisation (Laguna
 // M.1/XS.2 Technical Report summary, Key claims, report §3.1; Laguna-M.1-base
@@ -204,106 +206,22 @@ struct RefineScratch {
   float out_l[16];
 };
 
-template <int NPL>
-__device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
-                                             float *__restrict__ logits, int nsplit, int T,
-                                             const uint16_t *__restrict__ x,
-                                             const uint16_t *__restrict__ w_router,
-                                             const float *__restrict__ bias,
-                                             const float *__restrict__ sel_bias, int d, int E,
-                                             int k, int norm_topk, int32_t *__restrict__ topk_idx,
-                                             float *__restrict__ topk_w) {
-  float *row = logits + static_cast<size_t>(t) * E;
-  // This lane's logits (experts lane + 32 i): all loads first, one memory
-  // round trip.  With K slices (nsplit <= 4) the partial planes are summed in
-  // slice order and the sum is written back into plane 0, where the rest of
-  // the selection (and any later reader) finds the logits.
-  float lv[NPL];
-  {
-    const size_t plane = static_cast<size_t>(T) * E;
-    float part[4][NPL];
-#pragma unroll
-    for (int sl = 0; sl < 4; ++sl)
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        part[sl][i] = (sl < nsplit && e < E) ? row[sl * plane + e] : 0.f;
-      }
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      float l = part[0][i];
-#pragma unroll
-      for (int sl = 1; sl < 4; ++sl)
-        if (sl < nsplit) l += part[sl][i];
-      lv[i] = l;
-    }
-    if (nsplit > 1) {
-#pragma unroll
-      for (int i = 0; i < NPL; ++i)
-        if (lane + 32 * i < E) row[lane + 32 * i] = lv[i];
-      __syncwarp();
-    }
-  }
-  // The selection value of expert e with logit l: l, or with a selection-only
-  // bias sigmoid(l) + b_e (the weights below always use the logit).
-  auto sel_of = [&](int e, float l) -> float {
+// The float64 re-decision of a token whose k-th and (k+1)-th selection values
+// (lk, lk1) are within kRefineBand: the band's experts are ranked on float64
+// values and fill the places after the experts above the band (my_l / my_e of
+// lanes 0..k-1 are updated).  Kept out of line: it runs for few tokens, and
+// inlined its float64 state would crowd the registers of every token's path.
+__device__ __noinline__ void refine_band(int t, int lane, RefineScratch *rs, const float *row,
+                                         const uint16_t *__restrict__ x,
+                                         const uint16_t *__restrict__ w_router,
+                                         const float *__restrict__ bias,
+                                         const float *__restrict__ sel_bias, int d, int E, int k,
+                                         float lk, float lk1, float &my_l, int &my_e) {
+  auto sel_value = [&](int e) -> float {
+    const float l = row[e];
     return sel_bias ? 1.f / (1.f + expf(-l)) + sel_bias[e] : l;
   };
-  auto sel_value = [&](int e) -> float { return sel_of(e, row[e]); };
-  // Keys: an order-preserving map of the fp32 logit to uint32 (larger logit,
-  // larger key; +0 and -0 equal; NaN and the padding slots past E lowest).
-  uint32_t key[NPL];
-  int ev[NPL];
-#pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    ev[i] = lane + 32 * i;
-    key[i] = ev[i] < E ? logit_key(sel_of(ev[i], lv[i])) : 0u;
-  }
-  // Sort each lane's list descending by key.  The list starts in ascending
-  // expert id and the odd-even transposition network swaps only strictly
-  // smaller keys forward, so equal keys stay in ascending id (stable).
-#pragma unroll
-  for (int r = 0; r < NPL; ++r) {
-#pragma unroll
-    for (int i = r & 1; i + 1 < NPL; i += 2) {
-      if (key[i] < key[i + 1]) {
-        const uint32_t tk = key[i];
-        const int te = ev[i];
-        key[i] = key[i + 1];
-        ev[i] = ev[i + 1];
-        key[i + 1] = tk;
-        ev[i + 1] = te;
-      }
-    }
-  }
-  float my_l = 0.f;  // lane j < k keeps the j-th selected logit and expert
-  int my_e = 0;
-  float lk = 0.f, lk1 = -INFINITY;
-  const int rounds = k < E ? k + 1 : k;
-  for (int j = 0; j < rounds; ++j) {
-    // the largest head key, then the lowest expert id among the heads holding it
-    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key[0]);
-    const uint32_t ewin =
-        __reduce_min_sync(0xffffffffu, key[0] == kmax ? static_cast<uint32_t>(ev[0]) : 0xffffffffu);
-    if (static_cast<uint32_t>(ev[0]) == ewin) {  // pop the head
-#pragma unroll
-      for (int i = 0; i + 1 < NPL; ++i) {
-        key[i] = key[i + 1];
-        ev[i] = ev[i + 1];
-      }
-      key[NPL - 1] = 0u;
-      ev[NPL - 1] = 0x7fffffff;
-    }
-    const float lv = key_logit(kmax);
-    if (j < k && lane == j) {
-      my_l = lv;
-      my_e = static_cast<int>(ewin);
-    }
-    if (j == k - 1) lk = lv;
-    if (j == k) lk1 = lv;
-  }
 
-  if (k < E && lk - lk1 < kRefineBand) {
     // The fp32 selection values are within kRefineBand / 4 of their float64
     // values, so with mid the midpoint of the k-th and (k+1)-th values:
     // experts above mid + kRefineBand are in the float64 top k, those below
@@ -421,6 +339,121 @@ __device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
       }
     }
   }
+
+template <int NPL>
+__device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
+                                             float *__restrict__ logits, int nsplit, int T,
+                                             const uint16_t *__restrict__ x,
+                                             const uint16_t *__restrict__ w_router,
+                                             const float *__restrict__ bias,
+                                             const float *__restrict__ sel_bias, int d, int E,
+                                             int k, int norm_topk, int32_t *__restrict__ topk_idx,
+                                             float *__restrict__ topk_w) {
+  float *row = logits + static_cast<size_t>(t) * E;
+  // This lane's logits (experts lane + 32 i): all loads first, one memory
+  // round trip.  With K slices (nsplit <= 4) the partial planes are summed in
+  // slice order and the sum is written back into plane 0, where the rest of
+  // the selection (and any later reader) finds the logits.
+  float lv[NPL];
+  if (nsplit == 1) {
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      lv[i] = e < E ? row[e] : 0.f;
+    }
+  } else {
+    const size_t plane = static_cast<size_t>(T) * E;
+    float part[4][NPL];
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        part[sl][i] = (sl < nsplit && e < E) ? row[sl * plane + e] : 0.f;
+      }
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      float l = part[0][i];
+#pragma unroll
+      for (int sl = 1; sl < 4; ++sl)
+        if (sl < nsplit) l += part[sl][i];
+      lv[i] = l;
+    }
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (lane + 32 * i < E) row[lane + 32 * i] = lv[i];
+    __syncwarp();
+  }
+  // The selection value of expert e with logit l: l, or with a selection-only
+  // bias sigmoid(l) + b_e (the weights below always use the logit).
+  auto sel_of = [&](int e, float l) -> float {
+    return sel_bias ? 1.f / (1.f + expf(-l)) + sel_bias[e] : l;
+  };
+  auto sel_value = [&](int e) -> float { return sel_of(e, row[e]); };
+  // Keys: an order-preserving map of the fp32 selection value to uint32, plus
+  // one (larger value, larger key; +0 and -0 equal; NaN the lowest value, key
+  // 1); 0 marks an empty entry (and the padding slots past E).
+  uint32_t key[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? logit_key(sel_of(e, lv[i])) + 1u : 0u;
+  }
+  // Each lane keeps the top three of its remaining slots in (key descending,
+  // slot ascending) order -- slot i holds expert lane + 32 i, so equal keys keep
+  // the lower expert id first.  "Remaining" are the slots after the last one
+  // this lane gave up; when all three are taken the list is rebuilt from them.
+  uint32_t hk0, hk1, hk2;
+  int hi0, hi1, hi2;
+  auto build = [&](uint32_t last_k, int last_i) {
+    hk0 = hk1 = hk2 = 0u;
+    hi0 = hi1 = hi2 = NPL;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const uint32_t u = key[i];
+      if (!(u < last_k || (u == last_k && i > last_i))) continue;
+      if (u > hk0) {
+        hk2 = hk1; hi2 = hi1;
+        hk1 = hk0; hi1 = hi0;
+        hk0 = u;   hi0 = i;
+      } else if (u > hk1) {
+        hk2 = hk1; hi2 = hi1;
+        hk1 = u;   hi1 = i;
+      } else if (u > hk2) {
+        hk2 = u;   hi2 = i;
+      }
+    }
+  };
+  build(0xffffffffu, -1);
+  float my_l = 0.f;  // lane j < k keeps the j-th selected logit and expert
+  int my_e = 0;
+  float lk = 0.f, lk1 = -INFINITY;
+  const int rounds = k < E ? k + 1 : k;
+  for (int j = 0; j < rounds; ++j) {
+    // the largest head key, then the lowest expert id among the heads holding it
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, hk0);
+    const uint32_t mine = (hk0 == kmax && hk0 != 0u) ? static_cast<uint32_t>(lane + 32 * hi0)
+                                                     : 0xffffffffu;
+    const uint32_t ewin = __reduce_min_sync(0xffffffffu, mine);
+    if (mine == ewin) {  // this lane's head is taken
+      const uint32_t tk = hk0;
+      const int ti = hi0;
+      hk0 = hk1; hi0 = hi1;
+      hk1 = hk2; hi1 = hi2;
+      hk2 = 0u;  hi2 = NPL;
+      if (hk0 == 0u) build(tk, ti);
+    }
+    const float lj = key_logit(kmax - 1u);
+    if (j < k && lane == j) {
+      my_l = lj;
+      my_e = static_cast<int>(ewin);
+    }
+    if (j == k - 1) lk = lj;
+    if (j == k) lk1 = lj;
+  }
+
+  if (k < E && lk - lk1 < kRefineBand)
+    refine_band(t, lane, rs, row, x, w_router, bias, sel_bias, d, E, k, lk, lk1, my_l, my_e);
 
   // With a selection-only bias the rounds carried sigmoid(l) + b: the weights
   // take the selected experts' own logits.

@@ -18,6 +18,7 @@ enum Site : int {
   SITE_GEMM_EPI_ACC_FULL = 13,
   SITE_GEMM_DRAIN = 14,
   SITE_PERMUTE_EXPERT_ID = 20,
+  SITE_INDEX_GRID_BARRIER = 21,  // the one-launch index builder's wait for all chunk histograms
   SITE_H_FP16_RANGE = 30,        // SwiGLU activation beyond the fp16 range
   SITE_SLOT_FP16_RANGE = 31,     // scaled expert contribution beyond the fp16 range
   SITE_WEIGHT_FP16_RANGE = 32,   // down-projection weight beyond the fp16 range
@@ -31,7 +32,8 @@ struct WsHeader {
   int n_tiles;    // 128-row tiles in the expert tile list (written by the index builder)
   int n_tiles_pair;  // 256-row tiles in the second list, when one is built
   int index_done;    // index builder: histogram CTAs finished (the last one scans)
-  int pad[59];
+  int index_arrived; // one-launch index builder: CTAs past their histogram (grid barrier)
+  int pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 

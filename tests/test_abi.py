@@ -66,16 +66,18 @@ def test_workspace_size_and_shape_limits(L):
 
 
 def test_fused_and_reduce_combine_shape_rules_and_workspace(L):
-    """The fused kernel needs F, Fs, d multiples of 128 and FFN parts (<= 512 columns, equal)
-    of whole 128-column chunks; its workspace holds no h and no fp16 contribution rows, only
-    the fp32 token rows (so does the reduce combine's, which keeps h)."""
+    """The fused kernel needs F, Fs, d multiples of 128 (an FFN runs in equal parts of whole
+    128-column chunks, at most 512 columns each: 640 as five parts of 128); its workspace
+    holds no h and no fp16 contribution rows, only the fp32 token rows (so does the reduce
+    combine's, which keeps h)."""
     F_ = M.MOE_FLAG_FUSED_EXPERTS
     R_ = M.MOE_FLAG_COMBINE_REDUCE
     for ok in [(4096, 2048, 256, 8, 512, 512), (64, 256, 16, 4, 1024, 1024),
-               (64, 256, 16, 4, 768, 0), (64, 256, 16, 4, 1536, 128)]:
+               (64, 256, 16, 4, 768, 0), (64, 256, 16, 4, 1536, 128),
+               (64, 256, 16, 4, 640, 128)]:
         assert M.workspace_size(M.make_dims(*ok, flags=F_)) > 0, ok
-    for bad in [(64, 256, 16, 4, 640, 128),    # two parts of 320: not whole 128-column chunks
-                (64, 256, 16, 4, 192, 128),    # F not a multiple of 128
+    for bad in [(64, 256, 16, 4, 192, 128),    # F not a multiple of 128
+                (64, 256, 16, 4, 128, 320),    # Fs not a multiple of 128
                 (64, 192, 16, 4, 128, 128)]:   # d not a multiple of 128
         assert M.workspace_size(M.make_dims(*bad, flags=F_)) == 0, bad
     T, d, E, k, F, Fs = 4096, 2048, 256, 8, 512, 512

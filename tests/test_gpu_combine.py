@@ -9,8 +9,7 @@ kernel that also runs the gate/up GEMM and keeps h in tensor memory.
 The same rules as the default path: routing bit-exact up to the exempt
 near-ties, y within relative Frobenius 1e-2 and |dy| <= 2e-2 (|y| + 0.05) per
 element.  The order of a token's additions is not fixed, so repeated runs are
-compared within the redundant-run bound |dy| <= 1e-3 (|y| + 0.05) instead of
-bit for bit.
+compared up to one bf16 step per element instead of bit for bit.
 """
 import numpy as np
 import pytest
@@ -44,8 +43,12 @@ def _small(w):
     return h, G.host_to_device(h)
 
 
-def _close(a, b, rel=1e-3):
-    return np.all(np.abs(a - b) <= rel * (np.abs(b) + 0.05))
+def _bf16_steps_apart(a, b):
+    """Per element, how many bf16 steps apart two bf16 tensors (bit patterns) are."""
+    def ordered(u):
+        u = u.astype(np.int32)
+        return np.where(u & 0x8000, -(u & 0x7FFF), u)
+    return np.abs(ordered(a) - ordered(b))
 
 
 @pytest.mark.parametrize("flags", VARIANTS)
@@ -96,22 +99,29 @@ def test_reduce_combine_padding_mask_and_no_shared_expert(Fs, flags):
 
 @pytest.mark.parametrize("flags", [RED, FUSED])
 def test_reduce_combine_runs_agree_with_each_other_and_the_default_path(flags):
-    """Five runs of the same inputs: routing and permutation identical bit for bit, y within
-    the redundant-run bound of each other and of the deterministic default combine."""
+    """Five runs of the same inputs: routing and permutation identical bit for bit to each
+    other and to the default path; y of any two runs at most one bf16 step apart per element
+    (the fp32 sums differ in their last bits with the order of the additions, which can move
+    the final rounding to bf16 by one step) and every run within the oracle's bound.
+    (Against the default path, which rounds h and every contribution to fp16 where these
+    keep fp32 sums, y differs at that rounding's level: both are held to the oracle's
+    bound.)"""
     import torch
     w = I.get("c1_tiny").with_(T=1000)
-    _, dev = _small(w)
+    h, dev = _small(w)
     y0, r0, _ = G.run_forward(w, dev)
-    base = G.y_numpy(y0)
+    ref = G.oracle_forward(w, h)
     outs = []
     for _ in range(5):
         y, routing, _ = G.run_forward(w, dev, flags=flags)
-        outs.append((G.y_numpy(y), routing["topk_idx"].cpu().numpy(),
-                     routing["perm"].cpu().numpy()))
-    for yv, idx, perm in outs:
+        outs.append((P.to_numpy_bf16(y), routing["topk_idx"].cpu().numpy(),
+                     routing["perm"].cpu().numpy(), G.y_numpy(y)))
+    for bits, idx, perm, yv in outs:
         assert np.array_equal(idx, r0["topk_idx"].cpu().numpy())
         assert np.array_equal(perm, r0["perm"].cpu().numpy())
-        assert _close(yv, outs[0][0]) and _close(yv, base)
+        assert int(_bf16_steps_apart(bits, outs[0][0]).max()) <= 1
+        G.check_output(yv, ref["y"], what="reduce run")
+    G.check_output(G.y_numpy(y0), ref["y"], what="default run")
     torch.cuda.synchronize()
 
 
@@ -131,10 +141,11 @@ def test_reduce_combine_full_size_sample(name, flags):
     G.check_output(G.y_numpy(y)[rows], ref["y"], rows_ok=same, what=f"{name} sample")
 
 
-@pytest.mark.parametrize("F,Fs", [(1024, 1024), (768, 256), (256, 1536)])
+@pytest.mark.parametrize("F,Fs", [(1024, 1024), (768, 256), (256, 1536), (640, 128)])
 def test_fused_kernel_ffn_parts(F, Fs):
-    """FFN widths above 512 run in equal parts of at most 512 columns (1024: 2 x 512, 768:
-    2 x 384, 1536: 3 x 512) whose partial down projections add into the same rows."""
+    """FFN widths above 512 run in equal parts of whole 128-column chunks, at most 512
+    columns each (narrower ones when the batch has few row tiles), whose partial down
+    projections add into the same token rows."""
     w = I.get("c1_tiny").with_(T=300, moe_intermediate_size=F, shared_intermediate_size=Fs)
     h, dev = _small(w)
     y, routing, _ = G.run_forward(w, dev, flags=FUSED)

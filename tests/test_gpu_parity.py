@@ -678,11 +678,11 @@ def test_select_kernel_builds_the_decode_index(T, Fs):
     ref = G.oracle_forward(w, h, rows=rows)
     same = P.same_selection_mask(gidx[rows], ref["topk_idx"])
     G.check_output(G.y_numpy(y)[rows], ref["y"], rows_ok=same, what=f"T={T} Fs={Fs}")
-    # router logits, selection (+ index when fused), [two index kernels], W_down and (with
-    # a shared expert) its W_down converted to fp16 (bf16 weights passed), gate/up, down,
-    # combine
+    # router logits, selection (+ index when fused), [the one-launch index builder], W_down
+    # and (with a shared expert) its W_down converted to fp16 (bf16 weights passed),
+    # gate/up, down, combine
     fused = T * w.k <= 4096
-    expected = 2 + (0 if fused else 2) + (2 if Fs else 1) + 3
+    expected = 2 + (0 if fused else 1) + (2 if Fs else 1) + 3
     assert launches == expected, (launches, expected)
 
 
