@@ -220,7 +220,8 @@ __device__ __forceinline__ void scan_and_tiles(int *__restrict__ chunk_hist, int
 
 // The whole index of a single chunk (n <= kIndexChunk entries) in one CTA of
 // at least max(E, 256) threads: warps 0..7 do the histogram and the scatter,
-// all warps the scan.  h: kIdxWarps * kMaxE ints of shared memory.
+// all warps the scan; the counts and bases never leave shared memory.  h:
+// kIdxWarps * kMaxE ints of shared memory.
 __device__ __forceinline__ void index_single_cta(const int32_t *__restrict__ topk_idx, int n,
                                                  int E, int T, int with_shared,
                                                  int *__restrict__ chunk_hist,
@@ -231,21 +232,42 @@ __device__ __forceinline__ void index_single_cta(const int32_t *__restrict__ top
                                                  Tile *__restrict__ tiles,
                                                  Tile *__restrict__ tiles_pair, int *header, int *h,
                                                  int *warp_sums, int *totals) {
+  (void)chunk_hist;  // one chunk: its totals and bases stay in shared memory
   const int warp = threadIdx.x >> 5;
   // entries per warp: the chunk spread over all eight warps, in whole warps of entries
   const int sub = max(32, (n + kIdxWarps * 32 - 1) / (kIdxWarps * 32) * 32);
   chunk_warp_hist(topk_idx, n, E, 0, h, header, sub);  // warps 0..7
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int s = 0;
+  // one thread per expert: its count, the exclusive scan over experts, and each
+  // warp's first row of the expert (in place of the per-warp counts in h)
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < E) {
 #pragma unroll
-    for (int w = 0; w < kIdxWarps; ++w) s += h[w * E + e];
-    chunk_hist[e] = s;
+    for (int w = 0; w < kIdxWarps; ++w) cnt += h[w * E + e];
   }
-  __syncthreads();
-  scan_and_tiles(chunk_hist, 1, E, T, with_shared, counts, offsets, tiles, tiles_pair, header,
-                 warp_sums, totals);
-  __syncthreads();
-  warp_bases(E, chunk_hist, h);
+  const int off = block_exclusive_scan(e < E ? cnt : 0, warp_sums, &totals[0]);
+  if (e < E) {
+    counts[e] = cnt;
+    offsets[e] = off;
+    int run = off;
+#pragma unroll
+    for (int w = 0; w < kIdxWarps; ++w) {
+      const int c = h[w * E + e];
+      h[w * E + e] = run;
+      run += c;
+    }
+  }
+  if (e == 0) offsets[E] = totals[0];
+  const int n1 = write_tiles(e, cnt, off, E, T, with_shared, kBlockM, tiles, warp_sums, &totals[1]);
+  int n2 = 0;
+  if (tiles_pair != nullptr)
+    n2 = write_tiles(e, cnt, off, E, T, with_shared, 2 * kBlockM, tiles_pair, warp_sums,
+                     &totals[2]);
+  if (threadIdx.x == 0 && header) {
+    reinterpret_cast<WsHeader *>(header)->n_tiles = n1;
+    reinterpret_cast<WsHeader *>(header)->n_tiles_pair = n2;
+  }
+  __syncthreads();  // the bases in h are complete
   if (warp < kIdxWarps) chunk_warp_scatter(topk_idx, n, E, 0, h, perm, inv, sub);
 }
 

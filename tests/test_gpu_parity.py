@@ -151,6 +151,32 @@ def test_padding_mask_forward(T, frac, engine):
     G.check_output(G.y_numpy(y), ref["y"], what=f"mask T={T} frac={frac}")
 
 
+@pytest.mark.parametrize("T,router", [(3000, M.MOE_FLAG_ROUTER_CUDA_CORE),
+                                      (12000, M.MOE_FLAG_ROUTER_TENSOR)])
+def test_padding_mask_multi_chunk_index(T, router):
+    """Masked batches whose T * k entries span several index chunks, with the logits from
+    either router (one plane at T=3000 on CUDA cores, K-sliced planes summed by the select
+    kernel at T=12000): padding tokens are left unrouted, routed tokens match the oracle."""
+    w = I.get("c1_tiny").with_(T=T)
+    h, dev = _small(w)
+    mask = (np.random.default_rng(T).random(T) >= 0.3).astype(np.uint8)
+    y, routing = _mask_run(w, h, dev, mask, router)
+    ref = O.moe_forward(h["x"], h["w_router"], h["w_gate"], h["w_up"], h["w_down"], w.k,
+                        ws_gate=h["ws_gate"], ws_up=h["ws_up"], ws_down=h["ws_down"],
+                        routed_scaling_factor=w.routed_scaling_factor, token_mask=mask)
+    gidx = routing["topk_idx"].cpu().numpy()
+    gw = routing["topk_w"].cpu().numpy()
+    pad = mask == 0
+    assert np.all(gidx[pad] == M.MOE_NOT_ROUTED) and np.all(gw[pad] == 0.0)
+    keep = ~pad
+    G.check_routing(gidx[keep], gw[keep], {"topk_idx": ref["topk_idx"][keep],
+                                           "topk_w": ref["topk_w"][keep],
+                                           "scores": ref["scores"][keep]}, w.k)
+    same = np.ones(T, dtype=bool)
+    same[keep] = P.same_selection_mask(gidx[keep], ref["topk_idx"][keep])
+    G.check_output(G.y_numpy(y), ref["y"], rows_ok=same, what=f"mask, multi-chunk index T={T}")
+
+
 def test_padding_mask_permute_and_gather():
     import torch
     w = I.get("c1_tiny").with_(T=500)
