@@ -300,6 +300,20 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    if (MODE == MODE_GEMM2_F8 && warp == 2 && lane == 0) {
+      // The FP8 down epilogue multiplies by one scale per output column, read
+      // from the [E, d] (and [d]) float32 tables as each item starts; each CTA
+      // asks L2 for its share of the tables up front, so that those reads,
+      // on the epilogue's critical path, find them there.
+      const size_t total = static_cast<size_t>(p.E) * p.d * 4;
+      const size_t share = ((total + gridDim.x - 1) / gridDim.x + 15) & ~static_cast<size_t>(15);
+      const size_t off = static_cast<size_t>(blockIdx.x) * share;
+      if (off < total)
+        prefetch_l2_bulk(reinterpret_cast<const char *>(p.sb0) + off,
+                         static_cast<uint32_t>(total - off < share ? total - off : share));
+      if (blockIdx.x == 0 && p.Fs > 0 && p.sb0_sh != nullptr)
+        prefetch_l2_bulk(p.sb0_sh, static_cast<uint32_t>(p.d) * 4);
+    }
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row_local = q * 32 + lane;
     EpiStage st{smem + SmemLayout::epi_off + (warp - 2) * kEpiBytesPerWarp, 0};

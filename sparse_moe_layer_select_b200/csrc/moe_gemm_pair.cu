@@ -10,16 +10,19 @@
 // gate rows and its peer the up rows of the same column block.
 //
 // Synchronisation (all waits bounded, as in moe_gemm.cu):
-//   lfull[s]   per CTA: its own loads of stage s have landed (TMA bytes and
-//              cp.async arrivals)
+//   lfull[s]   GEMM1, per CTA: its own loads of stage s have landed (TMA bytes
+//              and cp.async arrivals)
 //   gather     GEMM1's A rows are copied by warps 7.. (each a share of the
 //              128 rows, gemm_common.cuh); warp 0 issues the TMA loads
-//   relay      warp 6 of the peer CTA forwards each of its completed stages
-//              to the leader's full[s], after a proxy fence for the
-//              cp.async-written rows; each CTA can therefore always drain its
-//              own copies
-//   full[s]    leader: the peer's half of stage s is in shared memory (the
-//              leader's MMA thread waits on its own lfull[s] for its half)
+//   relay      GEMM1: warp 6 of the peer CTA forwards each of its completed
+//              stages to the leader's full[s], after a proxy fence for the
+//              cp.async-written rows (a cp.async completion can only arrive on
+//              a barrier of its own CTA)
+//   full[s]    GEMM1, leader: the peer's half of stage s is in shared memory
+//              (the leader's MMA thread waits on its own lfull[s] for its
+//              half).  GEMM2 (all loads by TMA), leader: both halves are in
+//              shared memory -- each CTA's TMA loads complete on the leader's
+//              full[s] (.cta_group::2), the leader arms it for both CTAs' bytes
 //   empty[s]   per CTA: the leader's MMAs of stage s completed (commit
 //              multicast to both CTAs)
 //   acc_full   per CTA: an accumulator is complete (commit multicast)
@@ -94,7 +97,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
-      mbar_init(&full[s], 1);  // the peer's relayed arrival (the leader waits on its own lfull)
+      // GEMM1: the peer's relayed arrival (the leader waits on its own lfull);
+      // GEMM2: the leader's expect-tx arrival for both CTAs' bytes
+      mbar_init(&full[s], 1);
       // own loads: one expect_tx arrival (+ one cp.async arrival per gathering lane)
       mbar_init(&lfull[s], BASE == MODE_GEMM1 ? 1 + 32 * kGatherWarps : 1);
       mbar_init(&empty[s], 1);
@@ -137,6 +142,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                             : (kTmaWarpGathers ? 1 : 0) + (warp - kPairGather2Warp);
     const bool gathers = BASE == MODE_GEMM1 && gw >= 0;
     if (tma_warp || gathers) {
+      // GEMM2: both CTAs' TMA loads complete on the leader's full[s]
+      const uint32_t leader_full0 = map_shared_rank(smem_u32(&full[0]), 0);
       int s = 0;
       uint32_t ph = 0;
       long long issued = 0;
@@ -163,7 +170,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (tma_warp && lane == 0) MOE_TRACE_AT(p, TR_PWAIT, issued);
           if (lane == 0) {
             good = mbar_wait(&empty[s], ph ^ 1, status, SITE_GEMM_PRODUCER_EMPTY);
-            if (good && tma_warp) mbar_arrive_expect_tx(&lfull[s], bytes);
+            if (good && tma_warp) {
+              if (BASE == MODE_GEMM1) mbar_arrive_expect_tx(&lfull[s], bytes);
+              else if (leader) mbar_arrive_expect_tx(&full[s], 2 * bytes);  // equal boxes per CTA
+            }
           }
           good = __shfl_sync(0xffffffffu, good, 0);
           if (!good) {
@@ -182,9 +192,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                   leader ? (shared ? &tm_b0_sh : &tm_b0) : (shared ? &tm_b1_sh : &tm_b1);
               tma_load_2d(b_dst, tm, &lfull[s], kc, brow);
             } else {
-              tma_load_2d(a_dst, shared ? &tm_a_sh : &tm_a, &lfull[s], kc, it.row0);
+              const uint32_t bar = leader_full0 + s * 8;
+              tma_load_2d_pair(a_dst, shared ? &tm_a_sh : &tm_a, bar, kc, it.row0);
               const int brow = (shared ? 0 : it.group * p.d) + it.j * p.n_tile + rank * half_b_rows;
-              tma_load_2d(b_dst, shared ? &tm_b0_sh : &tm_b0, &lfull[s], kc, brow);
+              tma_load_2d_pair(b_dst, shared ? &tm_b0_sh : &tm_b0, bar, kc, brow);
             }
           }
           if (gathers) gather_a_stage<MODE>(p, tok, lane, gw, a_dst, &lfull[s], kc);
@@ -207,12 +218,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         walk.next();
       }
-      // Every stage filled must have landed before the CTA exits.
+      // Every stage filled must have landed before the CTA exits.  GEMM2: the
+      // leader's full[] counts both CTAs' bytes, and the peer stays until the
+      // leader reaches the closing cluster barrier.
       if (gathers) cp_async_wait_all();
-      if (tma_warp && lane == 0) {
+      if (tma_warp && lane == 0 && (BASE == MODE_GEMM1 || leader)) {
+        uint64_t *landed = BASE == MODE_GEMM1 ? lfull : full;
         for (long long n = (issued > kPairStages ? issued - kPairStages : 0); n < issued; ++n)
-          if (!mbar_wait(&lfull[n % kPairStages], static_cast<uint32_t>((n / kPairStages) & 1), status,
-                         SITE_GEMM_DRAIN))
+          if (!mbar_wait(&landed[n % kPairStages], static_cast<uint32_t>((n / kPairStages) & 1),
+                         status, SITE_GEMM_DRAIN))
             break;
       }
     }
@@ -220,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // ------------------------------------------------------------ relay (peer CTA)
     // The leader's MMA thread waits on the leader's own lfull; only the peer's
     // completed stages are forwarded, one remote arrival each on the leader's full.
-    if (lane == 0 && !leader) {
+    if (BASE == MODE_GEMM1 && lane == 0 && !leader) {
       const uint32_t leader_full0 = map_shared_rank(smem_u32(&full[0]), 0);
       int s = 0;
       uint32_t ph = 0;
@@ -269,7 +283,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint32_t d_tmem = tmem_base + acc * kPAccStride;
         for (int kb = 0; kb < it.nk; ++kb) {
           // this CTA's half of the stage (its loads), then the peer's (relayed)
-          if (!mbar_wait(&lfull[s], ph, status, SITE_GEMM_MMA_FULL) ||
+          if ((BASE == MODE_GEMM1 && !mbar_wait(&lfull[s], ph, status, SITE_GEMM_MMA_FULL)) ||
               !mbar_wait(&full[s], ph, status, SITE_GEMM_MMA_FULL)) {
             ok = false;
             break;
