@@ -138,8 +138,9 @@ constexpr int kSelectCtasPerSm = 4;
 
 // float64 logits of up to four experts e[0..n) for one token: exact bf16
 // products, float64 sums (lane-strided, then a butterfly in fixed order), plus
-// the bias.  The token row is read once per group, all loads of the group
-// are independent, so the group costs about one memory round trip.
+// the bias.  The token row is read once per group; the loads of a batch of
+// chunks are issued before any is used (the register budget of the selection
+// kernels bounds the batch).
 __device__ __forceinline__ void logits_f64_x4(const uint16_t *__restrict__ x,
                                               const uint16_t *__restrict__ w_router,
                                               const float *__restrict__ bias, int t,
@@ -152,20 +153,51 @@ __device__ __forceinline__ void logits_f64_x4(const uint16_t *__restrict__ x,
     wr[g] = reinterpret_cast<const uint4 *>(w_router + static_cast<size_t>(g < n ? e[g] : e[0]) * d);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
   const int nvec = d / 8;
+  if (n <= 2) {
+    // The usual band of one or two experts: four of the lane's chunks of the
+    // three rows in flight at once (the loads of a batch are issued before any
+    // is used), so the rows cost two memory round trips at d = 2048.
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+    for (int c0 = lane; c0 < nvec; c0 += 4 * 32) {
+      uint4 xv[4], wv0[4], wv1[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int c = c0 + 32 * b;
+        xv[b] = c < nvec ? xr[c] : zero;
+        wv0[b] = c < nvec ? wr[0][c] : zero;
+        wv1[b] = (c < nvec && n > 1) ? wr[1][c] : zero;
+      }
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float xf[8], wf0[8], wf1[8];
+        bf16x8_to_f32(xv[b], xf);
+        bf16x8_to_f32(wv0[b], wf0);
+        bf16x8_to_f32(wv1[b], wf1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          acc[0] = fma(static_cast<double>(xf[i]), static_cast<double>(wf0[i]), acc[0]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          acc[1] = fma(static_cast<double>(xf[i]), static_cast<double>(wf1[i]), acc[1]);
+      }
+    }
+  } else {
 #pragma unroll 4
-  for (int c = lane; c < nvec; c += 32) {
-    float xf[8];
-    bf16x8_to_f32(xr[c], xf);
-    uint4 wv[4];
+    for (int c = lane; c < nvec; c += 32) {
+      float xf[8];
+      bf16x8_to_f32(xr[c], xf);
+      uint4 wv[4];
 #pragma unroll
-    for (int g = 0; g < 4; ++g) wv[g] = wr[g][c];
+      for (int g = 0; g < 4; ++g) wv[g] = wr[g][c];
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      float wf[8];
-      bf16x8_to_f32(wv[g], wf);
+      for (int g = 0; g < 4; ++g) {
+        float wf[8];
+        bf16x8_to_f32(wv[g], wf);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        acc[g] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[g]);
+        for (int i = 0; i < 8; ++i)
+          acc[g] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[g]);
+      }
     }
   }
 #pragma unroll
@@ -233,13 +265,22 @@ __device__ __noinline__ void refine_band(int t, int lane, RefineScratch *rs, con
     const int above = __popc(__ballot_sync(0xffffffffu, lane < k && my_l > hi));
     const unsigned lt = (1u << lane) - 1u;
     const int nslice = (E + 31) / 32;
-    int nband = 0;
-    for (int i = 0; i < nslice; ++i) {  // band members in ascending id
+    // this lane's selection values (E <= 512: at most 16), every load issued
+    // before the first is used, so the band costs one memory round trip
+    float sv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
       const int e_lane = lane + 32 * i;
-      float v = 0.f;
+      sv[i] = (i < nslice && e_lane < E) ? row[e_lane] : 0.f;
+    }
+    int nband = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {  // band members in ascending id
+      if (i >= nslice) break;
+      const int e_lane = lane + 32 * i;
       bool in = false;
       if (e_lane < E) {
-        v = sel_value(e_lane);
+        const float v = sel_bias ? 1.f / (1.f + expf(-sv[i])) + sel_bias[e_lane] : sv[i];
         in = v >= lo && v <= hi;
       }
       const unsigned b = __ballot_sync(0xffffffffu, in);
