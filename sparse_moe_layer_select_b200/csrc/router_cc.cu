@@ -239,16 +239,18 @@ struct RefineScratch {
 };
 
 // The float64 re-decision of a token whose k-th and (k+1)-th selection values
-// (lk, lk1) are within kRefineBand: the band's experts are ranked on float64
-// values and fill the places after the experts above the band (my_l / my_e of
-// lanes 0..k-1 are updated).  Kept out of line: it runs for few tokens, and
-// inlined its float64 state would crowd the registers of every token's path.
+// (lk, lk1) are within kRefineBand: the band's experts (nband of them, the
+// first 32 in rs->ids in ascending id, found by the caller from the values it
+// holds) are ranked on float64 values and fill the places after the experts
+// above the band (my_l / my_e of lanes 0..k-1 are updated).  Kept out of line:
+// it runs for few tokens, and inlined its float64 state would crowd the
+// registers of every token's path.
 __device__ __noinline__ void refine_band(int t, int lane, RefineScratch *rs, const float *row,
                                          const uint16_t *__restrict__ x,
                                          const uint16_t *__restrict__ w_router,
                                          const float *__restrict__ bias,
                                          const float *__restrict__ sel_bias, int d, int E, int k,
-                                         float lk, float lk1, float &my_l, int &my_e) {
+                                         float lk, float lk1, int nband, float &my_l, int &my_e) {
   auto sel_value = [&](int e) -> float {
     const float l = row[e];
     return sel_bias ? 1.f / (1.f + expf(-l)) + sel_bias[e] : l;
@@ -263,31 +265,7 @@ __device__ __noinline__ void refine_band(int t, int lane, RefineScratch *rs, con
     const float mid = 0.5f * (lk + lk1);
     const float lo = mid - kRefineBand, hi = mid + kRefineBand;
     const int above = __popc(__ballot_sync(0xffffffffu, lane < k && my_l > hi));
-    const unsigned lt = (1u << lane) - 1u;
     const int nslice = (E + 31) / 32;
-    // this lane's selection values (E <= 512: at most 16), every load issued
-    // before the first is used, so the band costs one memory round trip
-    float sv[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int e_lane = lane + 32 * i;
-      sv[i] = (i < nslice && e_lane < E) ? row[e_lane] : 0.f;
-    }
-    int nband = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {  // band members in ascending id
-      if (i >= nslice) break;
-      const int e_lane = lane + 32 * i;
-      bool in = false;
-      if (e_lane < E) {
-        const float v = sel_bias ? 1.f / (1.f + expf(-sv[i])) + sel_bias[e_lane] : sv[i];
-        in = v >= lo && v <= hi;
-      }
-      const unsigned b = __ballot_sync(0xffffffffu, in);
-      const int pos = nband + __popc(b & lt);
-      if (in && pos < 32) rs->ids[pos] = e_lane;
-      nband += __popc(b);
-    }
     __syncwarp();
     if (nband <= 32) {
       for (int g0 = 0; g0 < nband; g0 += 4) {
@@ -493,8 +471,26 @@ __device__ __forceinline__ void select_token(int t, int lane, RefineScratch *rs,
     if (j == k) lk1 = lj;
   }
 
-  if (k < E && lk - lk1 < kRefineBand)
-    refine_band(t, lane, rs, row, x, w_router, bias, sel_bias, d, E, k, lk, lk1, my_l, my_e);
+  if (k < E && lk - lk1 < kRefineBand) {
+    // The band's members in ascending id, from the selection values this lane
+    // holds as keys (no memory round trip); the first 32 go to rs->ids.
+    const float mid = 0.5f * (lk + lk1);
+    const float lo = mid - kRefineBand, hi = mid + kRefineBand;
+    const unsigned lt = (1u << lane) - 1u;
+    int nband = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const float v = key_logit(key[i] - 1u);
+      const bool in = key[i] != 0u && v >= lo && v <= hi;
+      const unsigned b = __ballot_sync(0xffffffffu, in);
+      const int pos = nband + __popc(b & lt);
+      if (in && pos < 32) rs->ids[pos] = lane + 32 * i;
+      nband += __popc(b);
+    }
+    __syncwarp();
+    refine_band(t, lane, rs, row, x, w_router, bias, sel_bias, d, E, k, lk, lk1, nband, my_l,
+                my_e);
+  }
 
   // With a selection-only bias the rounds carried sigmoid(l) + b: the weights
   // take the selected experts' own logits.
