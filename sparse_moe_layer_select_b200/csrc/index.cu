@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(512)
   __shared__ int warp_sums[32];
   __shared__ int totals[3];
   __shared__ int go;
+  __shared__ int s_first[kMaxE], s_row0[kMaxE], s_cnt[kMaxE];
   const int nchunks = gridDim.x;
   chunk_warp_hist(topk_idx, n, E, blockIdx.x, h, header, sub);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -150,22 +151,26 @@ __global__ void __launch_bounds__(512)
     }
   }
   const int off = block_exclusive_scan(e < E ? total : 0, warp_sums, &totals[0]);
+  // CTA 0 writes counts, offsets and the 128-row tile list, CTA 1 (CTA 0 with
+  // a single chunk) the 256-row list, each spread over the CTA's threads.
+  const int pair_writer = nchunks > 1 ? 1 : 0;
   if (blockIdx.x == 0) {
     if (e < E) {
       counts[e] = total;
       offsets[e] = off;
     }
     if (e == 0) offsets[E] = totals[0];
-    const int n1 = write_tiles(e, total, off, E, T, with_shared, kBlockM, tiles, warp_sums,
-                               &totals[1]);
-    int n2 = 0;
-    if (tiles_pair != nullptr)
-      n2 = write_tiles(e, total, off, E, T, with_shared, 2 * kBlockM, tiles_pair, warp_sums,
-                       &totals[2]);
+    const int n1 = write_tiles_spread(e, total, off, E, T, with_shared, kBlockM, tiles, warp_sums,
+                                      &totals[1], s_first, s_row0, s_cnt);
     if (threadIdx.x == 0) {
       reinterpret_cast<WsHeader *>(header)->n_tiles = n1;
-      reinterpret_cast<WsHeader *>(header)->n_tiles_pair = n2;
+      if (tiles_pair == nullptr) reinterpret_cast<WsHeader *>(header)->n_tiles_pair = 0;
     }
+  }
+  if (tiles_pair != nullptr && static_cast<int>(blockIdx.x) == pair_writer) {
+    const int n2 = write_tiles_spread(e, total, off, E, T, with_shared, 2 * kBlockM, tiles_pair,
+                                      warp_sums, &totals[2], s_first, s_row0, s_cnt);
+    if (threadIdx.x == 0) reinterpret_cast<WsHeader *>(header)->n_tiles_pair = n2;
   }
   // per-warp first rows of this chunk (the shared-memory histograms of phase 1)
   if (e < E) {

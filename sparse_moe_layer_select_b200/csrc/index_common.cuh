@@ -78,6 +78,21 @@ __device__ __forceinline__ void chunk_warp_hist(const int32_t *__restrict__ topk
   __syncthreads();
 }
 
+// The lanes of the warp whose id equals this lane's (ids in [-1, 1023)): an
+// AND over ten bit-plane ballots, the same mask __match_any_sync returns at a
+// fraction of its cost (one ballot per bit of the id).
+__device__ __forceinline__ unsigned lanes_with_same_id(int e) {
+  const unsigned v = static_cast<unsigned>(e) & 0x3ffu;  // -1 -> 1023, above every expert id
+  unsigned m = 0xffffffffu;
+#pragma unroll
+  for (int b = 0; b < 10; ++b) {
+    const unsigned bit = (v >> b) & 1u;
+    const unsigned votes = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? votes : ~votes;
+  }
+  return m;
+}
+
 // Each warp places its `sub` consecutive entries (512 in a multi-chunk
 // batch; fewer, spread over all eight warps, in a single small chunk):
 // fill[warp][e] holds its next row of e.
@@ -103,7 +118,7 @@ __device__ __forceinline__ void chunk_warp_scatter(const int32_t *__restrict__ t
     if (r >= sub || base + r >= n) break;  // warp-uniform
     int e = ids[q];
     if (e < 0 || e >= E) e = -1;
-    const unsigned m = __match_any_sync(0xffffffffu, e);
+    const unsigned m = lanes_with_same_id(e);
     const int rank = __popc(m & lt);
     if (e >= 0) {
       const int pos = fw[e] + rank;
@@ -158,6 +173,51 @@ __device__ __forceinline__ int write_tiles(int e, int cnt, int off, int E, int T
     tiles[*total + i] = t;
   }
   return *total + nshared;
+}
+
+// The same tile list as write_tiles, with the routed tiles written by every
+// thread of the CTA -- tile ti's expert found by a binary search over the
+// experts' first tiles -- so that a skewed expert's many tiles are not one
+// thread's serial stores.  s_first, s_row0, s_cnt: shared arrays of E ints.
+__device__ __forceinline__ int write_tiles_spread(int e, int cnt, int off, int E, int T,
+                                                  int with_shared, int tile_rows,
+                                                  Tile *__restrict__ tiles, int *warp_sums,
+                                                  int *total, int *s_first, int *s_row0,
+                                                  int *s_cnt) {
+  const int ntile = e < E ? (cnt + tile_rows - 1) / tile_rows : 0;
+  const int toff = block_exclusive_scan(ntile, warp_sums, total);
+  if (e < E) {
+    s_first[e] = toff;
+    s_row0[e] = off;
+    s_cnt[e] = cnt;
+  }
+  __syncthreads();
+  const int nrouted = *total;
+  for (int ti = threadIdx.x; ti < nrouted; ti += blockDim.x) {
+    int lo = 0, hi = E - 1;  // the last expert whose first tile is <= ti
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_first[mid] <= ti) lo = mid;
+      else hi = mid - 1;
+    }
+    const int i = ti - s_first[lo];
+    Tile t;
+    t.group = lo;
+    t.row0 = s_row0[lo] + i * tile_rows;
+    t.nrows = min(tile_rows, s_cnt[lo] - i * tile_rows);
+    t.pad = 0;
+    tiles[ti] = t;
+  }
+  const int nshared = with_shared ? (T + tile_rows - 1) / tile_rows : 0;
+  for (int i = threadIdx.x; i < nshared; i += blockDim.x) {
+    Tile t;
+    t.group = E;
+    t.row0 = i * tile_rows;
+    t.nrows = min(tile_rows, T - i * tile_rows);
+    t.pad = 0;
+    tiles[nrouted + i] = t;
+  }
+  return nrouted + nshared;
 }
 
 // Expert sums over chunks, exclusive scan over experts, chunk bases and the
