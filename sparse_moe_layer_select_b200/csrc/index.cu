@@ -134,12 +134,12 @@ __global__ void __launch_bounds__(512)
   int total = 0, before = 0;
   if (e < E) {
     int c = 0;
-    for (; c + 16 <= nchunks; c += 16) {  // sixteen independent loads in flight
-      int v[16];
+    for (; c + 32 <= nchunks; c += 32) {  // 32 independent loads in flight
+      int v[32];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) v[q] = __ldcg(&chunk_hist[static_cast<size_t>(c + q) * E + e]);
+      for (int q = 0; q < 32; ++q) v[q] = __ldcg(&chunk_hist[static_cast<size_t>(c + q) * E + e]);
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
+      for (int q = 0; q < 32; ++q) {
         total += v[q];
         before += (c + q) < static_cast<int>(blockIdx.x) ? v[q] : 0;
       }
