@@ -521,7 +521,8 @@ def run_ours(args):
     # end to end through the C ABI: pinned host batch in, host output back, every step
     e2e = None
     if not args.no_e2e:
-        e2e = end_to_end(M, torch, layer, w, dev["x"], ring, steps, world)
+        e2e = end_to_end(M, torch, layer, w, dev["x"], ring, steps, world,
+                         copy_streams=args.copy_streams)
 
     # the materialised permutation (moe_permute with x_perm) at this batch's routing
     permute = None
@@ -633,11 +634,12 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def end_to_end(M, torch, layer, w, x_buf, ring, steps, world):
+def end_to_end(M, torch, layer, w, x_buf, ring, steps, world, copy_streams=1):
     """Through the public API with host buffers: every step copies its own input from
-    pinned host memory and reads its own output back.  Three streams (input copy, layer,
-    output copy) and two device buffers overlap step i's copies with the layer of steps
-    i-1 / i+1."""
+    pinned host memory and reads its own output back.  The input copy, the layer and the
+    output copy run on their own streams with two device buffers, so step i's copies
+    overlap the layer of steps i-1 / i+1; each copy is split into `copy_streams` row
+    blocks on as many streams, so that several copy engines share a direction."""
     decode = ring is not None
     n_host = min(steps, 64) if decode else 1
     hx = torch.empty((n_host, w.T, w.d_model), dtype=torch.bfloat16, pin_memory=True)
@@ -645,30 +647,38 @@ def end_to_end(M, torch, layer, w, x_buf, ring, steps, world):
     hy = [torch.empty((w.T, w.d_model), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
     xd = [torch.empty_like(x_buf) for _ in range(2)]
     yd = [torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    nc = max(1, min(copy_streams, w.T))
+    s_in = [torch.cuda.Stream() for _ in range(nc)]
+    s_out = [torch.cuda.Stream() for _ in range(nc)]
     s_c = torch.cuda.current_stream()
+    cuts = [w.T * c // nc for c in range(nc + 1)]
 
     def run_e2e(n):
-        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_in = [[torch.cuda.Event() for _ in range(nc)] for _ in range(n)]
         ev_c = [torch.cuda.Event() for _ in range(n)]
-        ev_out = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [[torch.cuda.Event() for _ in range(nc)] for _ in range(n)]
         for i in range(n):
             b = i % 2
+            for c in range(nc):
+                lo, hi = cuts[c], cuts[c + 1]
+                if i >= 2:
+                    s_in[c].wait_event(ev_c[i - 2])      # the layer of step i-2 has read xd[b]
+                with torch.cuda.stream(s_in[c]):
+                    xd[b][lo:hi].copy_(hx[i % n_host][lo:hi], non_blocking=True)
+                ev_in[i][c].record(s_in[c])
+                s_c.wait_event(ev_in[i][c])
             if i >= 2:
-                s_in.wait_event(ev_c[i - 2])      # the layer of step i-2 has read xd[b]
-            with torch.cuda.stream(s_in):
-                xd[b].copy_(hx[i % n_host], non_blocking=True)
-            ev_in[i].record(s_in)
-            s_c.wait_event(ev_in[i])
-            if i >= 2:
-                s_c.wait_event(ev_out[i - 2])     # yd[b] of step i-2 is back on the host
+                for c in range(nc):
+                    s_c.wait_event(ev_out[i - 2][c])  # yd[b] of step i-2 is back on the host
             layer.forward(xd[b], yd[b], stream=s_c)
             ev_c[i].record(s_c)
-            s_out.wait_event(ev_c[i])
-            with torch.cuda.stream(s_out):
-                hy[b].copy_(yd[b], non_blocking=True)
-            ev_out[i].record(s_out)
-        return ev_out[-1]
+            for c in range(nc):
+                lo, hi = cuts[c], cuts[c + 1]
+                s_out[c].wait_event(ev_c[i])
+                with torch.cuda.stream(s_out[c]):
+                    hy[b][lo:hi].copy_(yd[b][lo:hi], non_blocking=True)
+                ev_out[i][c].record(s_out[c])
+        return [ev_out[-1][c] for c in range(nc)]
 
     run_e2e(2)
     torch.cuda.synchronize()
@@ -677,17 +687,19 @@ def end_to_end(M, torch, layer, w, x_buf, ring, steps, world):
         dist.barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(s_in)
-    s_c.wait_event(a)
-    s_out.wait_event(a)
+    a.record(s_c)
+    for st in s_in + s_out:
+        st.wait_event(a)
     last = run_e2e(steps)
-    s_out.wait_event(last)
-    b.record(s_out)
+    for ev in last:
+        s_c.wait_event(ev)
+    b.record(s_c)
     torch.cuda.synchronize()
     te = max_over_ranks(a.elapsed_time(b) / 1e3, world)
     return {"value": job_tokens_per_s(w.T, steps, world, te), "unit": "tokens/s",
             "h2d_bytes_per_step": w.T * w.d_model * 2, "d2h_bytes_per_step": w.T * w.d_model * 2,
-            "overlap": "input copy, layer and output copy on three streams, two buffers"}
+            "overlap": f"input copy, layer and output copy on their own streams, two buffers; "
+                       f"each copy in {nc} row blocks on {nc} streams"}
 
 
 def time_permute(M, torch, layer, w, x, steps, peaks):
@@ -810,6 +822,9 @@ def main():
                          "the down GEMM adds into fp32 token rows (MOE_FLAG_COMBINE_REDUCE)")
     ap.add_argument("--fused", action="store_true",
                     help="the fused expert kernel (h in tensor memory; MOE_FLAG_FUSED_EXPERTS)")
+    ap.add_argument("--copy-streams", type=int, default=1,
+                    help="streams (row blocks) each end-to-end host<->device copy is split over "
+                         "(2 or 4 measured slower than 1 at the T=32768 prefill)")
     ap.add_argument("--fp8", action="store_true",
                     help="FP8 (e4m3) expert weights: moe_prepare_fp8 + moe_forward_fp8")
     args = ap.parse_args()
