@@ -24,7 +24,7 @@
 //   index_scatter_kernel  per chunk: per-warp histograms and their scan give
 //                         each warp its first row per expert; each warp then
 //                         places its entries in order, ranks among equal
-//                         experts from __match_any_sync (stable, deterministic)
+//                         experts from bit-plane ballots (stable, deterministic)
 // With a single chunk (decode-sized batches) one CTA does all three steps in
 // one launch (index_single_kernel), or, inside a layer forward with E <= 256,
 // the last CTA of the router's selection kernel does (router_cc.cu).  With up
