@@ -166,8 +166,8 @@ size_t moe_workspace_size(const moe_dims_t *dims);
 
 /* Router: sigmoid scores, top-k with ties to the lower expert index, and
  * post-top-k normalisation (Laguna M.1/XS.2 Technical Report summary, Key
- * claims, report §3.1; Laguna-M.1-base spec sheet, Mixture of experts:
- * "Router score", "Renormalize top-k").  Selection is made on the logits
+ * claims, report §3.1; Laguna-M.1-base spec sheet, Mixture of experts: the
+ * router score is a sigmoid, the top-k weights are renormalised).  Selection is made on the logits
  * (equivalent to selection on the scores, since the sigmoid is increasing):
  * fp32 logits, and for tokens whose k-th and (k+1)-th logits are closer than
  * 2e-4, float64 logits for the experts at that boundary.

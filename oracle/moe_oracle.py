@@ -10,12 +10,13 @@ What the layer computes, and where the pages say so:
 
 * Router: sigmoid scores over the experts, token-choice top-k, and
   normalisation of the selected scores to sum to one
-  (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1:
-  "sigmoid router with post-top-k normalization"; Laguna-M.1-base spec sheet,
-  Mixture of experts: "Router score: sigmoid", "Renormalize top-k: Yes").
+  (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1: a
+  sigmoid router whose top-k scores are normalised after the selection;
+  Laguna-M.1-base spec sheet, Mixture of experts: sigmoid router scores,
+  top-k renormalisation on).
 * Experts: SwiGLU feed-forward blocks without bias
-  (Laguna-M.1-base spec sheet, Feed-forward: "Activation: SwiGLU",
-  "FFN bias: No", gate_proj / up_proj / down_proj projections).
+  (Laguna-M.1-base spec sheet, Feed-forward: SwiGLU activation, no FFN
+  bias, gate_proj / up_proj / down_proj projections).
 * Combine: the routed sum is multiplied by the modulation factor 2.5 and then
   added to an always-on shared expert
   (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1;
@@ -23,7 +24,7 @@ What the layer computes, and where the pages say so:
   1 for M.1, 2.5 introduced in XS.2).
 * Expert order: tokens are laid out expert by expert before the grouped GEMM
   (Laguna M.1/XS.2 Technical Report summary, Key claims, report §3.1.2,
-  Fig. 2: tokens are copied "in expert order").
+  Fig. 2: the tokens are copied so that each expert's rows are contiguous).
 
 Readings where the pages are silent:
 

@@ -2,8 +2,9 @@
 // the grouped expert GEMMs.
 //
 // The grouped GEMM takes tokens laid out expert by expert (Laguna M.1/XS.2
-// Technical Report summary, Key claims, report §3.1.2, Fig. 2: tokens are
-// copied "in expert order").  Here that order is an index, not a copy:
+// Technical Report summary, Key claims, report §3.1.2, Fig. 2: the tokens are
+// copied so that each expert's rows are contiguous).  Here that order is an
+// index, not a copy:
 //
 //   counts[e]  rows of expert e;  offsets = exclusive prefix sum (E + 1)
 //   perm[r]    = t * k + j for the r-th row in expert order, rows of one

@@ -4,7 +4,7 @@
 //
 // Sigmoid router with post-top-k normalisation (Laguna M.1/XS.2 Technical
 // Report summary, Key claims, report §3.1; Laguna-M.1-base spec sheet,
-// Mixture of experts: "Router score: sigmoid", "Renormalize top-k: Yes").
+// Mixture of experts: sigmoid router scores, top-k renormalisation on).
 //
 //   router_logits_kernel  fp32 logits[T, E] = x . W_r^T (+ b): a CTA stages
 //                         8 token rows in shared memory; each warp computes
