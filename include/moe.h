@@ -303,7 +303,7 @@ moe_status moe_profile_next_forward(void **events, int32_t n_events);
  * E = 256, 823,296 at E = 512.  Dims that need more return
  * MOE_ERR_UNSUPPORTED_SHAPE, and nothing is launched.  The first call on each
  * device looks up the array's device address (cudaGetSymbolAddress, with that
- * device current): make that first call before any stream capture.  Every
+ * device current).  Every
  * call uses the same array, so calls that overlap on the GPU (other streams,
  * or other host threads) race; serialise them.  An expert id outside [0, E)
  * is skipped on the device and is not reported by this entry point.  It
