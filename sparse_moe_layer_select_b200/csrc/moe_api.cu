@@ -132,14 +132,19 @@ bool use_tensor_router(const Dims &D);
 // K slices of the tensor-core router GEMM: with few 128-token tiles, up to 4
 // slices of d (each slice's CTAs write partial logits, summed in slice order
 // by the select kernel), so that about one CTA per SM streams its share of x
-// once instead of a few CTAs streaming whole rows.  A function of the
-// dimensions only, since the workspace holds one logit plane per slice.
+// once instead of a few CTAs streaming whole rows.  Four slices only up to 18
+// tiles (T <= 2304): at T = 4096 two slices measured faster than four (router
+// GEMM + select 28.0 against 30.4 us, ncu), the select kernel summing half as
+// many planes.  A function of the dimensions only, since the workspace holds
+// one logit plane per slice.
 constexpr int kRouterSplitSms = 148;
 int router_ksplit(const Dims &D) {
   if (!use_tensor_router(D)) return 1;
   const int tiles = (D.T + kBlockM - 1) / kBlockM;
+  const int max_ks = tiles <= kRouterSplitSms / 8 ? 4 : 2;
   int ks = 1;
-  while (ks < 4 && tiles * ks * 2 <= kRouterSplitSms && (D.d / kBlockK) % (ks * 2) == 0) ks *= 2;
+  while (ks < max_ks && tiles * ks * 2 <= kRouterSplitSms && (D.d / kBlockK) % (ks * 2) == 0)
+    ks *= 2;
   return ks;
 }
 

@@ -90,18 +90,19 @@ def test_fused_and_reduce_combine_shape_rules_and_workspace(L):
 
 
 def test_workspace_holds_one_logit_plane_per_router_slice(L):
-    """The tensor-core router (T >= 1024 at E = 256) cuts d into 4 K slices up to 37 token
-    tiles (T <= 4736), 2 up to 74 (T <= 9472), none above, and the workspace holds one fp32
+    """The tensor-core router (T >= 1024 at E = 256) cuts d into 4 K slices up to 18 token
+    tiles (T <= 2304), 2 up to 74 (T <= 9472), none above, and the workspace holds one fp32
     [T, E] logit plane per slice: the size jumps by about three planes at T = 1024 (no slices
-    on the CUDA-core router below) and drops by about two planes just past T = 4736 and
-    about one just past T = 9472."""
+    on the CUDA-core router below) and drops by about two planes just past T = 2304 and
+    about one just past T = 9472; T = 4736 -> 4737 (37 -> 38 tiles) keeps two."""
     def ws(T):
         return M.workspace_size(M.make_dims(T, 2048, 256, 8, 512, 512))
     plane = lambda T: T * 256 * 4
     per_token = ws(2001) - ws(2000)          # growth of everything else, per token
     assert 0 < per_token < 200_000
     assert ws(1024) - ws(1023) > 3 * plane(1023) - 2 * per_token
-    assert ws(4736) - ws(4737) > 2 * plane(4736) - 2 * per_token
+    assert ws(2304) - ws(2305) > 2 * plane(2304) - 2 * per_token
+    assert abs((ws(4737) - ws(4736)) - (per_token - 2 * 256 * 4)) < 4096
     assert ws(9472) - ws(9473) > plane(9472) - 2 * per_token
     # T = 2000 grows by four planes per token, T = 20000 by one (256-byte section alignment)
     assert abs((ws(20001) - ws(20000)) - (per_token - 3 * 256 * 4)) < 2048

@@ -536,7 +536,7 @@ def test_router_logits_error_against_float64(flags):
 
 @pytest.mark.parametrize("T", [1024, 4096, 6000, 10000])
 def test_router_k_slices_against_float64(T):
-    """The tensor-core router splits d into 4 slices (T <= 4736), 2 (T <= 9472) or none; the
+    """The tensor-core router splits d into 4 slices (T <= 2304), 2 (T <= 9472) or none; the
     select kernel sums the slices' partial logits.  The summed logits against the oracle's
     float64 logits, and the routing against the oracle's, at each split (XS.2 widths)."""
     import torch
