@@ -290,8 +290,8 @@ moe_status moe_profile_next_forward(void **events, int32_t n_events);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
  * memory (code that runs inside another runtime's memory pool, or plugins
- * whose host process owns all device memory).  The paper has no counterpart
- * to this entry point; it is a deployment convenience.
+ * whose host process owns all device memory).  The source pages describe no
+ * counterpart to this entry point; it is a deployment convenience.
  * Same outputs as moe_permute without x / x_perm: counts [E], offsets [E + 1],
  * perm [T * k].  Its scratch is one static device array of
  * MOE_STATIC_SCRATCH_BYTES per GPU, held from library load to process exit.
