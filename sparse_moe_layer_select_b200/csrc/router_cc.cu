@@ -63,6 +63,24 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   const int nt = min(kTokPerCta, T - t0);
   const int vec_per_row = d / 8;
   const int n_vec = kTokPerCta * vec_per_row;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // This lane's weight vectors of an expert row, kWLoads loads in flight at a time.
+  constexpr int kWLoads = 8;
+  uint4 wv[kWLoads];
+  auto load_w = [&](const uint4 *wr, int c0) {
+#pragma unroll
+    for (int u = 0; u < kWLoads; ++u) {
+      const int c = c0 + 32 * u;
+      wv[u] = c < vec_per_row ? wr[c] : make_uint4(0, 0, 0, 0);
+    }
+  };
+  // The first expert's first batch of weights is requested before the token
+  // rows are staged, so that the two memory round trips overlap.
+  const int e_first = blockIdx.y * kWarpsPerCta + warp;
+  if (e_first < E)
+    load_w(reinterpret_cast<const uint4 *>(w_router + static_cast<size_t>(e_first) * d), lane);
+  bool have_w = e_first < E;
   // Stage the tokens: each thread's loads are issued together (kStageLoads at
   // a time), then stored, so the staging costs about one memory round trip.
   constexpr int kStageLoads = 8;
@@ -81,22 +99,14 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
       if (i0 + u * blockDim.x < n_vec) xs4[i0 + u * blockDim.x] = v[u];
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  for (int e = blockIdx.y * kWarpsPerCta + warp; e < E; e += gridDim.y * kWarpsPerCta) {
+  for (int e = e_first; e < E; e += gridDim.y * kWarpsPerCta) {
     const uint4 *wr = reinterpret_cast<const uint4 *>(w_router + static_cast<size_t>(e) * d);
     float acc[kTokPerCta];
 #pragma unroll
     for (int r = 0; r < kTokPerCta; ++r) acc[r] = 0.f;
-    // this lane's weight vectors of the expert row, kWLoads loads in flight at a time
-    constexpr int kWLoads = 8;
     for (int c0 = lane; c0 < vec_per_row; c0 += 32 * kWLoads) {
-      uint4 wv[kWLoads];
-#pragma unroll
-      for (int u = 0; u < kWLoads; ++u) {
-        const int c = c0 + 32 * u;
-        wv[u] = c < vec_per_row ? wr[c] : make_uint4(0, 0, 0, 0);
-      }
+      if (!have_w) load_w(wr, c0);
+      have_w = false;
 #pragma unroll
       for (int u = 0; u < kWLoads; ++u) {
         const int c = c0 + 32 * u;
