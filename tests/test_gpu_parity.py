@@ -534,6 +534,33 @@ def test_router_logits_error_against_float64(flags):
     assert err < 1e-4 / 4, err
 
 
+@pytest.mark.parametrize("d", [4096, 7296])
+def test_cuda_core_router_wide_rows(d):
+    """The CUDA-core router stages 8 bf16 token rows per CTA in shared memory; beyond d = 3072
+    that takes more than the default 48 KB (the opt-in launch attribute).  Against the oracle's
+    float64 logits and routing, on a ragged batch (43 tokens: five full groups of 8 and 3)."""
+    import torch
+    w = I.get("c2_xs2_small").with_(T=43, d_model=d)
+    h = {"x": I.generate_numpy((w.T, d), w.seed, I.TID_X, w.sigma_x),
+         "w_router": I.generate_numpy((w.E, d), w.seed, I.TID_W_ROUTER, w.sigma_router)}
+    dev = G.host_to_device(h)
+    dims = M.dims_for(w, flags=M.MOE_FLAG_ROUTER_CUDA_CORE)
+    ws = M.alloc_workspace(dims)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((w.T, w.k), dtype=torch.float32, device="cuda")
+    M.route(dims, dev["x"], dev["w_router"], None, idx, wt, ws)
+    torch.cuda.synchronize()
+    code, site = M.read_device_status(ws)
+    assert code == 0, (M.status_string(code), site)
+    off = M.logits_offset(dims)
+    got = ws[off:off + w.T * w.E * 4].view(torch.float32).view(w.T, w.E).cpu().numpy()
+    ref_l = O.router_logits(h["x"], h["w_router"], None)
+    assert float(np.abs(got - ref_l).max()) < 1e-4 / 4
+    ref = O.route(h["x"], h["w_router"], None, w.k)
+    G.check_routing(idx.cpu().numpy(), wt.cpu().numpy(),
+                    {"topk_idx": ref[0], "topk_w": ref[1], "scores": ref[2]}, w.k)
+
+
 @pytest.mark.parametrize("T", [1024, 4096, 6000, 10000])
 def test_router_k_slices_against_float64(T):
     """The tensor-core router splits d into 4 slices (T <= 2304), 2 (T <= 9472) or none; the
