@@ -122,8 +122,9 @@ size_t gemm_pair_smem_bytes();
 cudaError_t launch_gemm_pair(int mode, const GemmParams &p, const GemmMaps &m, int grid,
                              cudaStream_t s);
 
+// CUDA-core router logits; sms: the device's SM count (grid shape choice).
 cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
-                             float *logits, int T, int d, int E, cudaStream_t s);
+                             float *logits, int T, int d, int E, int sms, cudaStream_t s);
 // Warp-per-token selection over the fp32 logits of every token.
 // Expert id of a (token, slot) pair that is not routed (a padding token).
 constexpr int kNotRouted = -1;

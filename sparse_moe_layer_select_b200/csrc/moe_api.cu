@@ -330,7 +330,7 @@ moe_status route_impl(const Dims &D, const void *x, const void *w_router, const 
     return MOE_OK;
   }
   if (launch_router_cc(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(w_router),
-                       bias, logits, D.T, D.d, D.E, s) != cudaSuccess)
+                       bias, logits, D.T, D.d, D.E, sms, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (launch_router_select(logits, 1, static_cast<const uint16_t *>(x),
                            static_cast<const uint16_t *>(w_router), bias, sel_bias, token_mask,

@@ -8,7 +8,7 @@
 //
 //   router_logits_kernel  fp32 logits[T, E] = x . W_r^T (+ b): a CTA stages
 //                         8 token rows in shared memory; each warp computes
-//                         one expert's logits for those 8 tokens (16-byte
+//                         two experts' logits for those 8 tokens (16-byte
 //                         loads of W_r, fp32 FMA, warp butterfly reduction).
 //   router_select_kernel  one warp per token, for both logit paths: the E
 //                         logits sit in registers (E/32 per lane) as
@@ -54,6 +54,10 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
   }
 }
 
+// kExpPerWarp experts per warp: 2 when the whole grid fits on the SMs at one
+// CTA each (small batches; 142 registers), else 1 (84 registers, several CTAs
+// per SM to hide the memory round trips of many CTA waves).
+template <int kExpPerWarp>
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
     router_logits_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w_router,
                          const float *__restrict__ bias, float *__restrict__ logits, int T, int d,
@@ -65,21 +69,25 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   const int n_vec = kTokPerCta * vec_per_row;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // This lane's weight vectors of an expert row, kWLoads loads in flight at a time.
+  // This lane's weight vectors of the warp's kExpPerWarp expert rows,
+  // kWLoads per row in flight at a time.
   constexpr int kWLoads = 8;
-  uint4 wv[kWLoads];
-  auto load_w = [&](const uint4 *wr, int c0) {
+  uint4 wv[kExpPerWarp][kWLoads];
+  auto load_w = [&](int e0, int c0) {
 #pragma unroll
-    for (int u = 0; u < kWLoads; ++u) {
-      const int c = c0 + 32 * u;
-      wv[u] = c < vec_per_row ? wr[c] : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < kExpPerWarp; ++j) {
+      const uint4 *wr = reinterpret_cast<const uint4 *>(w_router + static_cast<size_t>(e0 + j) * d);
+#pragma unroll
+      for (int u = 0; u < kWLoads; ++u) {
+        const int c = c0 + 32 * u;
+        wv[j][u] = (e0 + j < E && c < vec_per_row) ? wr[c] : make_uint4(0, 0, 0, 0);
+      }
     }
   };
-  // The first expert's first batch of weights is requested before the token
+  // The first experts' first batch of weights is requested before the token
   // rows are staged, so that the two memory round trips overlap.
-  const int e_first = blockIdx.y * kWarpsPerCta + warp;
-  if (e_first < E)
-    load_w(reinterpret_cast<const uint4 *>(w_router + static_cast<size_t>(e_first) * d), lane);
+  const int e_first = (blockIdx.y * kWarpsPerCta + warp) * kExpPerWarp;
+  if (e_first < E) load_w(e_first, lane);
   bool have_w = e_first < E;
   // Stage the tokens: each thread's loads are issued together (kStageLoads at
   // a time), then stored, so the staging costs about one memory round trip.
@@ -99,37 +107,52 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
       if (i0 + u * blockDim.x < n_vec) xs4[i0 + u * blockDim.x] = v[u];
   }
   __syncthreads();
-  for (int e = e_first; e < E; e += gridDim.y * kWarpsPerCta) {
-    const uint4 *wr = reinterpret_cast<const uint4 *>(w_router + static_cast<size_t>(e) * d);
-    float acc[kTokPerCta];
+  // Each staged x vector read from shared memory feeds all kExpPerWarp
+  // experts (the reads, not the FMAs, bound this loop); every logit keeps the
+  // same products in the same order.
+  for (int e0 = e_first; e0 < E; e0 += gridDim.y * kWarpsPerCta * kExpPerWarp) {
+    float acc[kExpPerWarp][kTokPerCta];
 #pragma unroll
-    for (int r = 0; r < kTokPerCta; ++r) acc[r] = 0.f;
+    for (int j = 0; j < kExpPerWarp; ++j)
+#pragma unroll
+      for (int r = 0; r < kTokPerCta; ++r) acc[j][r] = 0.f;
     for (int c0 = lane; c0 < vec_per_row; c0 += 32 * kWLoads) {
-      if (!have_w) load_w(wr, c0);
+      if (!have_w) load_w(e0, c0);
       have_w = false;
 #pragma unroll
       for (int u = 0; u < kWLoads; ++u) {
         const int c = c0 + 32 * u;
         if (c >= vec_per_row) break;
-        float wf[8];
-        bf16x8_to_f32(wv[u], wf);
+        float wf[kExpPerWarp][8];
+#pragma unroll
+        for (int j = 0; j < kExpPerWarp; ++j) bf16x8_to_f32(wv[j][u], wf[j]);
 #pragma unroll
         for (int r = 0; r < kTokPerCta; ++r) {
           float xf[8];
           bf16x8_to_f32(xs4[r * vec_per_row + c], xf);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[r] = fmaf(xf[i], wf[i], acc[r]);
+          for (int j = 0; j < kExpPerWarp; ++j)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[j][r] = fmaf(xf[i], wf[j][i], acc[j][r]);
         }
       }
     }
 #pragma unroll
-    for (int r = 0; r < kTokPerCta; ++r) {
+    for (int j = 0; j < kExpPerWarp; ++j)
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], off);
-    }
+      for (int r = 0; r < kTokPerCta; ++r) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          acc[j][r] += __shfl_xor_sync(0xffffffffu, acc[j][r], off);
+      }
     if (lane == 0) {
-      const float b = bias ? bias[e] : 0.f;
-      for (int r = 0; r < nt; ++r) logits[static_cast<size_t>(t0 + r) * E + e] = acc[r] + b;
+#pragma unroll
+      for (int j = 0; j < kExpPerWarp; ++j) {
+        const int e = e0 + j;
+        if (e >= E) break;
+        const float b = bias ? bias[e] : 0.f;
+        for (int r = 0; r < nt; ++r) logits[static_cast<size_t>(t0 + r) * E + e] = acc[j][r] + b;
+      }
     }
   }
 }
@@ -588,24 +611,34 @@ __global__ void __launch_bounds__(kSelectWarps * 32, kSelectCtasPerSm)
                         warp_sums, totals);
 }
 
-}  // namespace
-
-cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
-                             float *logits, int T, int d, int E, cudaStream_t s) {
-  const int gx = (T + kTokPerCta - 1) / kTokPerCta;
-  // spread experts over enough CTAs to fill the GPU when T is small
-  int gy = (E + kWarpsPerCta - 1) / kWarpsPerCta;
-  if (gx >= 256) gy = 1;
+template <int kExpPerWarp>
+cudaError_t launch_router_logits(const uint16_t *x, const uint16_t *w_router, const float *bias,
+                                 float *logits, int T, int d, int E, int gx, int gy,
+                                 cudaStream_t s) {
   const size_t smem = static_cast<size_t>(kTokPerCta) * d * 2;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(router_logits_kernel,
+    cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<kExpPerWarp>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  router_logits_kernel<<<dim3(gx, gy), kWarpsPerCta * 32, smem, s>>>(x, w_router, bias, logits,
-                                                                      T, d, E);
+  router_logits_kernel<kExpPerWarp><<<dim3(gx, gy), kWarpsPerCta * 32, smem, s>>>(
+      x, w_router, bias, logits, T, d, E);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_router_cc(const uint16_t *x, const uint16_t *w_router, const float *bias,
+                             float *logits, int T, int d, int E, int sms, cudaStream_t s) {
+  const int gx = (T + kTokPerCta - 1) / kTokPerCta;
+  // spread experts over enough CTAs to fill the GPU when T is small
+  const int gy2 = (E + 2 * kWarpsPerCta - 1) / (2 * kWarpsPerCta);
+  if (static_cast<int64_t>(gx) * gy2 <= sms)
+    return launch_router_logits<2>(x, w_router, bias, logits, T, d, E, gx, gy2, s);
+  int gy = (E + kWarpsPerCta - 1) / kWarpsPerCta;
+  if (gx >= 256) gy = 1;
+  return launch_router_logits<1>(x, w_router, bias, logits, T, d, E, gx, gy, s);
 }
 
 cudaError_t launch_router_select(float *logits, int nsplit, const uint16_t *x,
