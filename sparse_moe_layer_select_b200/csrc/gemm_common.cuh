@@ -114,10 +114,12 @@ struct ItemWalk {
 // instruction moves 4 whole 128-byte rows).  One warp issues such copies at
 // about one instruction per 15 ns, slower than the tensor cores consume a
 // stage, so the rows are split across warps on all four SM sub-partitions.
-// (TMA tile::gather4 moves the same 4 rows per instruction; measured in
-// place of, and beside, cp.async it was slower: one, the other or any split
-// of the rows between them took 2.34 to 2.99 ms for the gate/up GEMM of the
-// skewed T=32768 prefill with one gathering warp.)
+// Even so the copies arrive at only ~16 KB per 0.5 us per SM, which bounds
+// the gate/up GEMM at large batches.  (TMA tile::gather4 moves the same 4
+// rows per instruction but was slower: with one gathering warp, gather4 for
+// all or part of the rows took 2.34 to 2.99 ms for the gate/up GEMM of the
+// skewed T=32768 prefill; beside these eight warps, gather4 for 32 or 64 of
+// the 128 rows took 1.70 or 2.15 ms against 1.08 ms.)
 #ifndef MOE_GATHER_WARPS
 #define MOE_GATHER_WARPS 8
 #endif
