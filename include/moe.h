@@ -27,7 +27,10 @@
  *   moe_read_device_status, so the sequence can be captured in a CUDA graph.
  * - Every device pointer must be 16-byte aligned.  Shape limits: d_model a
  *   multiple of 64; F and Fs multiples of 64 (Fs = 0: no shared expert);
- *   1 <= k <= min(E, 16); E <= 512.  Anything else returns
+ *   1 <= k <= min(E, 16); E <= 512.  The calls that route (moe_route*,
+ *   moe_forward*) also need d_model <= 14528 when the router runs on CUDA
+ *   cores (T < 1024, E not a multiple of 16 or above 256, or
+ *   MOE_FLAG_ROUTER_CUDA_CORE).  Anything else returns
  *   MOE_ERR_UNSUPPORTED_SHAPE before anything is launched.
  * - T = 0 is a no-op that returns MOE_OK.
  * - Errors: argument errors return synchronously and launch nothing; a failed

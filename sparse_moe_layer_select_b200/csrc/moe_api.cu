@@ -257,6 +257,15 @@ moe_status check_dims(const moe_dims_t *dims, Dims *D) {
   return MOE_OK;
 }
 
+// Shapes the router itself cannot take: a batch routed on CUDA cores stages
+// 8 bf16 token rows per CTA in shared memory (227 KB at most; router_cc.cu),
+// so d is capped on that path.
+constexpr int kRouterCcMaxD = 232448 / (8 * 2);
+moe_status check_router_dims(const Dims &D) {
+  if (!use_tensor_router(D) && D.d > kRouterCcMaxD) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 moe_status check_ws(const Dims &D, const void *ws, size_t ws_bytes) {
@@ -398,6 +407,7 @@ moe_status moe_route_masked(const moe_dims_t *dims, const void *x, const void *w
   Dims D;
   moe_status st = check_dims(dims, &D);
   if (st != MOE_OK) return st;
+  if ((st = check_router_dims(D)) != MOE_OK) return st;
   if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(topk_idx) || !aligned16(topk_w) ||
       (router_bias && !aligned16(router_bias)))
@@ -462,6 +472,7 @@ moe_status moe_forward_masked(const moe_dims_t *dims, const moe_weights_t *w, co
   Dims D;
   moe_status st = check_dims(dims, &D);
   if (st != MOE_OK) return st;
+  if ((st = check_router_dims(D)) != MOE_OK) return st;
   if (!w || !x || !y || !routing) return MOE_ERR_INVALID_ARG;
   if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
   if (D.Fs > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down)) return MOE_ERR_INVALID_ARG;
@@ -488,6 +499,7 @@ moe_status moe_forward_fp8(const moe_dims_t *dims, const moe_weights_t *w,
   Dims D;
   moe_status st = check_dims(dims, &D);
   if (st != MOE_OK) return st;
+  if ((st = check_router_dims(D)) != MOE_OK) return st;
   if (!(D.flags & MOE_FLAG_FP8_EXPERTS) ||
       (D.flags & (MOE_FLAG_COMBINE_REDUCE | MOE_FLAG_FUSED_EXPERTS)))
     return MOE_ERR_INVALID_ARG;

@@ -132,6 +132,13 @@ def test_argument_errors_return_before_any_launch(L):
     # forced tensor-core router with an E it cannot take
     f = M.make_dims(64, 256, 24, 4, 128, 128, flags=M.MOE_FLAG_ROUTER_TENSOR)
     assert _call_forward(f) == M.MOE_ERR_UNSUPPORTED_SHAPE
+    # the CUDA-core router (small batches, or E outside the tensor router's range) stages
+    # 8 bf16 token rows per CTA in 227 KB of shared memory: d <= 14528 on that path only
+    wide = M.make_dims(64, 14592, 256, 8, 512, 512)
+    assert M.workspace_size(wide) > 0                 # a permute-only caller can size it
+    assert _call_forward(wide) == M.MOE_ERR_UNSUPPORTED_SHAPE
+    assert _call_forward(M.make_dims(2048, 14592, 264, 8, 512, 512)) == M.MOE_ERR_UNSUPPORTED_SHAPE
+    assert _call_forward(wide, x=0) == M.MOE_ERR_UNSUPPORTED_SHAPE  # shape checks come first
 
 
 def _fp8_struct(missing=None):
