@@ -40,14 +40,29 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 2 ** 20
 
 
-def load_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
+def load_peaks(path=None):
+    """Roofline denominators: the measured figures where MEASURED_PEAKS.json gives them
+    (numbers at the top level), the fallback figures for any it lacks; "source" names
+    which were measured."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peaks = dict(FALLBACK_PEAKS)
+    if not os.path.exists(path):
+        return peaks
+    try:
         with open(path) as f:
-            p = json.load(f)
-        p["source"] = "measured"
-        return p
-    return dict(FALLBACK_PEAKS)
+            got = json.load(f)
+    except (OSError, ValueError):
+        return peaks
+    keys = ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")
+    measured = [k for k in keys
+                if isinstance(got, dict) and isinstance(got.get(k), (int, float)) and got[k] > 0]
+    for k in measured:
+        peaks[k] = float(got[k])
+    if len(measured) == len(keys):
+        peaks["source"] = "measured"
+    elif measured:
+        peaks["source"] = "measured " + ", ".join(measured) + "; fallback for the rest"
+    return peaks
 
 
 def _code_tokens(text):

@@ -129,3 +129,25 @@ def test_stage_work_of_the_t4096_workload():
     assert f8["gemm1_swiglu"]["bytes"] == (1073741824 + 4194304) // 2 + 16777216 + \
         4 * (256 * 2 * 512 + 2 * 512)
     assert f8["gemm2_down_scale"]["bytes"] == (536870912 + 2097152) // 2 + 4 * (256 * 2048 + 2048)
+
+
+def test_peaks_measured_where_given_fallback_for_the_rest(tmp_path):
+    sys.path.insert(0, ROOT)
+    import bench
+    full = tmp_path / "full.json"
+    full.write_text(json.dumps({"hbm_gbs": 6537.3, "bf16_tflops": 1602.0,
+                                "bf16_tflops_sustained": 1391.0, "clocks": {"sm": 1965}}))
+    p = bench.load_peaks(str(full))
+    assert (p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"]) == (6537.3, 1602.0, 1391.0)
+    assert p["source"] == "measured"
+    part = tmp_path / "part.json"
+    part.write_text(json.dumps({"hbm_gbs": 6537.3, "bf16_tflops": "n/a"}))
+    p = bench.load_peaks(str(part))
+    assert p["hbm_gbs"] == 6537.3
+    assert p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    assert p["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert p["source"].startswith("measured hbm_gbs") and "fallback" in p["source"]
+    bad = tmp_path / "bad.json"
+    bad.write_text("{not json")
+    assert bench.load_peaks(str(bad)) == bench.FALLBACK_PEAKS
+    assert bench.load_peaks(str(tmp_path / "missing.json")) == bench.FALLBACK_PEAKS
